@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of the SALR linear layer Y = X (M.W)^T + (X A_cat) B_cat on B200.
+
+One step is one salr_linear call on the decode q_proj workload (W 4096 x 4096 bf16, 50%
+per-row magnitude pruned and bitmap-encoded, adapters 64 + 16 stacked to R = 80,
+X 16 x 4096).  Prints one JSON line (see --help).  Timing: W warm-up steps, then K steps
+queued behind a short GPU sleep so that host launch overhead does not leave gaps, each
+bracketed by CUDA events on the launching stream; the weight/adapter set rotates over
+enough copies that the working set exceeds L2 (no step finds its weights in L2).
+
+--impl reference times the fp64 CPU oracle on the same workload instead (one full layer
+per step on the host cores).  Under torchrun every rank runs an independent replica
+(the layer has no data-path exchange); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import salr_synth as synth  # noqa: E402
+
+METRIC = "SALR linear tokens/s + achieved fraction of HBM/tensor roofline on 1 B200"
+WORKLOAD = "q_proj"
+M_TOKENS = 16
+L2_BYTES = 126 * 1024 * 1024
+KERNEL_SOURCES = ["sm100.cuh", "salr_codec.cuh", "salr_linear.cuh", "salr_api.cu"]
+
+
+def algorithmic_bytes(N, K, R, M, keep):
+    """Bytes the layer must move: bitmap, kept values, offset table, adapters (once),
+    activations in and outputs out (padding and L2 re-reads excluded)."""
+    return (N * K / 8 + 2 * N * keep + (N // 128) * (K // 64) * 4 + 2 * R * (K + N)
+            + 2 * M * K + 2 * M * N)
+
+
+def algorithmic_flops(N, K, R, M):
+    return 2 * M * N * K + 2 * M * K * R + 2 * M * R * N
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "sparse_rank_linear_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            p = [v.strip() for v in line.split(",")]
+            if len(p) >= 9:
+                rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def oracle_step_fn(wl, M):
+    """The fp64 oracle on one full step of the workload (inputs prepared untimed)."""
+    import oracle
+    w = synth.weight(wl)
+    wp = oracle.prune(w, oracle.magnitude_mask(w, wl.sparsity))
+    x = synth.activations(wl, M)
+    ad = synth.adapters(wl)
+    return lambda: oracle.linear(x, wp, ad)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(wl, M, steps=None, budget_s=10.0):
+    step = oracle_step_fn(wl, M)
+    step()  # warm
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        step()
+        n += 1
+        el = time.perf_counter() - t0
+        if (steps is not None and n >= steps) or (steps is None and el >= budget_s):
+            break
+    return n, el
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[WORKLOAD]
+    step = oracle_step_fn(wl, M_TOKENS)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = args.steps * M_TOKENS / el
+    cores = blas_threads()
+    sample = f"full {WORKLOAD} layer (M={M_TOKENS}) per step, fp64 numpy oracle"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD} N=4096 K=4096 R=80 M={M_TOKENS} s=0.5"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def traffic_for(kname, workload):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kname}|{workload}")
+    if not e or e.get("kernel_hash") != kernel_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["salr", "reference"], default="salr")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from sparse_rank_linear_b200.build import build
+    import sparse_rank_linear_b200 as salr
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    if rank == 0:
+        build()
+    if ws > 1:
+        dist.barrier()
+    lib = salr.load_library()
+
+    wl = synth.WORKLOADS[WORKLOAD]
+    N, K, R, M = wl.N, wl.K, wl.R, M_TOKENS
+    keep = K - int(np.floor(wl.sparsity * K))
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+    w_bits = synth.weight(wl)
+    W = dev(w_bits)
+    ad = synth.adapters(wl)
+    a_cat = np.concatenate([a for a, _ in ad], axis=1)
+    b_cat = np.concatenate([b for _, b in ad], axis=0)
+    x_bits = synth.activations(wl, M)
+    X = dev(x_bits)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+
+    # rotate over enough independent weight + adapter copies to exceed 2x L2
+    first = salr.encode(W, wl.sparsity)
+    per_copy = first.info()["bytes"] + 2 * R * (K + N)
+    ncopies = max(2, int(np.ceil(2 * L2_BYTES / per_copy)))
+    handles = [first] + [salr.encode(W, wl.sparsity) for _ in range(ncopies - 1)]
+    A = [dev(a_cat) for _ in range(ncopies)]
+    B = [dev(b_cat) for _ in range(ncopies)]
+    del W
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    sp = salr.binding._stream_ptr(stream)
+    import ctypes
+
+    def launch(i):
+        c = i % ncopies
+        rc = lib.salr_linear(ctypes.c_void_p(X.data_ptr()), M, handles[c].handle,
+                             ctypes.c_void_p(A[c].data_ptr()), ctypes.c_void_p(B[c].data_ptr()),
+                             R, ctypes.c_void_p(Y.data_ptr()), sp)
+        if rc:
+            raise RuntimeError(salr.status_string(rc))
+
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    for h in handles[:1]:
+        if h.sync_status() != 0:
+            raise RuntimeError("device status after warm-up")
+
+    # ---------------- device-resident timed region
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        torch.cuda._sleep(int(2e9 * 40e-6 * args.steps) + 10_000_000)
+        for i in range(args.steps):
+            ev_s[i].record(stream)
+            launch(i)
+            ev_e[i].record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    per_launch_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
+    total_ms = ev_s[0].elapsed_time(ev_e[-1])
+    if ws > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    status = handles[0].sync_status()
+    if status != 0:
+        raise RuntimeError(f"device status {salr.status_string(status)}")
+
+    # ---------------- end to end: host activations in, host outputs back, per step
+    xh = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = args.steps
+
+    def launch_host(i):
+        c = i % ncopies
+        rc = lib.salr_linear_host(ctypes.c_void_p(xh.data_ptr()), M, handles[c].handle,
+                                  ctypes.c_void_p(A[c].data_ptr()), ctypes.c_void_p(B[c].data_ptr()),
+                                  R, ctypes.c_void_p(yh.data_ptr()), sp)
+        if rc:
+            raise RuntimeError(salr.status_string(rc))
+
+    for i in range(args.warmup):
+        launch_host(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e9 * 60e-6 * e2e_steps) + 10_000_000)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        launch_host(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    peaks, peak_src = measured_peaks()
+    kern_ms = statistics.mean(per_launch_ms)
+    abytes = algorithmic_bytes(N, K, R, M, keep)
+    aflops = algorithmic_flops(N, K, R, M)
+    t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = aflops / (peaks["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        achieved = abytes / (kern_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        achieved = aflops / (kern_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
+    kname = "salr_linear_kernel<16>"
+    roof["traffic"] = traffic_for(kname, WORKLOAD)
+    roof["peak_source"] = peak_src
+    roof["kernel"] = kname
+    roof["kernel_ms"] = kern_ms
+    roof["algorithmic_bytes"] = abytes
+    roof["algorithmic_flops"] = aflops
+
+    value = ws * args.steps * M / (total_ms * 1e-3)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD} N={N} K={K} R={R} (64+16) M={M} sparsity=0.5",
+                       "model": "SALR linear layer (decode q_proj shape)", "global_batch": M * ws,
+                       "parallelism": f"replicas x{ws}",
+                       "l2": f"rotating {ncopies} weight+adapter copies "
+                             f"({ncopies * per_copy / 2**20:.0f} MiB > 2x L2)"},
+            "roofline": roof,
+            "e2e": {"value": ws * e2e_steps * M / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N},
+            "gpu_launches": args.steps,
+            "clocks": clocks.summary(),
+            "kernel_ms_p10_p50_p90": [float(np.percentile(per_launch_ms, q)) for q in (10, 50, 90)]}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        n, el = time_oracle(wl, M)
+        line["cpu_baseline"] = {"value": n * M / el, "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} full {WORKLOAD} layers (M={M}) in {el:.1f} s, "
+                                          "fp64 numpy oracle"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for h in handles:
+        h.free()
+    if ws > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,156 @@
+/*
+ * salr.h - C ABI of the SALR sparse + low-rank inference linear layer for NVIDIA B200.
+ *
+ * The layer (SALR, "Sparsity-Aware Low-Rank Representation for Efficient Fine-Tuning of
+ * Large Language Models"; the authors' abstract and the gist.science technical summary):
+ *
+ *     Y = X (M (.) W)^T + X A_cat B_cat
+ *
+ * W (N x K, out x in) is the frozen base weight, statically magnitude-pruned per row
+ * (technical summary, Methodology 1) and stored as a bitmap plus a compact array of the
+ * kept values with a per-block offset table (Methodology 4, "Bitmap Encoding" and the
+ * lookup table read by "Stage 1").  A_cat (K x R) and B_cat (R x N) are the low-rank
+ * adapters (task LoRAs and the truncated-SVD residual adapter) stacked along rank into
+ * one GEMM on the shared input (Methodology 3).  salr_linear runs the two-stage
+ * pipeline of Methodology 4: bitmap blocks are expanded on CUDA cores while tensor cores
+ * consume the previously expanded blocks.
+ *
+ * Conventions for every entry point
+ *   - Matrices are row-major; bf16 is passed as its 16-bit pattern (uint16).
+ *   - "device" pointers are CUDA device memory of the device current at the call;
+ *     "host" pointers are page-locked host memory (cudaHostAlloc / cudaHostRegister).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  All
+ *     calls are stream-ordered unless stated otherwise.
+ *   - Every call returns a salr_status.  Argument errors are detected on the host before
+ *     any work is queued; nothing is written in that case.
+ *   - The library never traps or spins without a bound on the GPU.  Errors found on the
+ *     device (a NaN in W, a pipeline wait that ran out of time) are recorded in the
+ *     handle's status word; salr_encode reports them itself, salr_sync_status reads them.
+ *
+ * Shape rules (v1): N % 128 == 0, K % 64 == 0, 64 <= K <= 32768, R % 8 == 0, R <= 128,
+ * M >= 1, all pointers 16-byte aligned.
+ */
+#ifndef SALR_H_
+#define SALR_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SALR_API __attribute__((visibility("default")))
+#else
+#define SALR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct salr_weight_s* salr_handle; /* opaque; owns its device buffers */
+
+typedef enum {
+  SALR_OK = 0,
+  SALR_ERR_INVALID = 1,     /* bad argument, bad handle, NaN in W, bad sparsity      */
+  SALR_ERR_UNSUPPORTED = 2, /* shape or alignment outside the v1 rules above         */
+  SALR_ERR_CUDA = 3,        /* a CUDA runtime/driver call or a launch failed         */
+  SALR_ERR_OOM = 4,         /* a device or host allocation failed                    */
+  SALR_ERR_TIMEOUT = 5      /* a bounded wait inside a kernel gave up                */
+} salr_status;
+
+/*
+ * salr_encode - prune W by magnitude and store it in the bitmap block format.
+ *
+ * Defined by: technical summary, Methodology 1 (static magnitude mask on the frozen base,
+ * adapters stay dense) and Methodology 4 (bitmap + compact values + lookup table).
+ *
+ * W        device, N x K bf16, read only; may be freed once the call returns.
+ * sparsity fraction pruned per row, 0 <= sparsity < 1.  Each row keeps
+ *          keep = K - floor(sparsity * K) entries: those of largest |w|, and among equal
+ *          |w| those of lowest column index.  |+0| = |-0|; +-Inf rank highest; a NaN
+ *          makes the call fail with SALR_ERR_INVALID.
+ * out      receives a new handle on SALR_OK (unchanged otherwise).
+ *
+ * Synchronises `stream` once (to size the value array and to read the NaN check).
+ *
+ * Encoded format (also readable through salr_format_view): W is cut into blocks of
+ * 128 rows x 64 columns; block b = i * (K/64) + j covers rows 128i..128i+127 and
+ * columns 64j..64j+63 and starts at byte 16 * offsets[b] of the blob.  A block holds
+ * 128 little-endian uint64 words (word r: bit c set when W[128i+r, 64j+c] is kept),
+ * then the kept values as bf16 in row-major order (a kept -0 stays -0), then zero
+ * bytes up to a multiple of 16.  offsets has nblocks + 1 uint32 entries; the last is
+ * the blob size in 16-byte units.
+ */
+SALR_API int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* stream,
+                salr_handle* out);
+
+/*
+ * salr_decode - expand an encoded weight back to dense M (.) W, for checking.
+ *
+ * W_out device, N x K bf16, caller-allocated, fully overwritten; pruned entries are
+ *       +0.0 (0x0000), kept entries bit-identical to W.
+ */
+SALR_API int salr_decode(salr_handle h, void* W_out, void* stream);
+
+/*
+ * salr_linear - Y = X (M (.) W)^T + (X A_cat) B_cat, one kernel launch.
+ *
+ * Defined by: technical summary, Methodology 3 (one concatenated adapter GEMM on the
+ * shared input) and Methodology 4 (two-stage pipelined bitmap decoding + tensor-core
+ * GEMM).
+ *
+ * X     device, M x K bf16.
+ * M     number of tokens, >= 1.
+ * A_cat device, K x R bf16; B_cat device, R x N bf16.  R == 0 means no adapter; the
+ *       pointers are then ignored and may be NULL.
+ * Y     device, M x N bf16, overwritten (no accumulation into Y).
+ *
+ * Arithmetic: products of bf16 inputs accumulate in fp32 on the tensor cores.  The
+ * adapter's inner product t = X A_cat is accumulated in fp32 and rounded once to bf16
+ * before it multiplies B_cat.  The order of the fp32 sums is not fixed (split K), so
+ * results are not bitwise reproducible between calls with different M, but always
+ * satisfy ||Y - Y*||_F <= 4e-3 ||Y*||_F and |Y - Y*| <= 1e-2 * sum|products| against the
+ * exact result Y*.
+ *
+ * The handle holds the split-K workspace used by this call; it is grown on demand
+ * (a cudaMalloc) and is not safe to share between calls running concurrently on
+ * different streams.
+ */
+SALR_API int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat,
+                const void* B_cat, int64_t R, void* Y, void* stream);
+
+/*
+ * salr_linear_host - salr_linear with the activations in host memory.
+ *
+ * X_host (M x K bf16) and Y_host (M x N bf16) are page-locked host buffers; A_cat and
+ * B_cat are device buffers as for salr_linear (adapters are weights and stay resident).
+ * Queues the host-to-device copy of X, the layer and the device-to-host copy of Y on
+ * `stream` through staging buffers owned by the handle; Y_host is valid once the
+ * stream has been synchronised.
+ */
+SALR_API int salr_linear_host(const void* X_host, int64_t M, salr_handle h, const void* A_cat,
+                     const void* B_cat, int64_t R, void* Y_host, void* stream);
+
+/* salr_free - release a handle and every device buffer it owns.  Freeing an unknown or
+ * already freed handle returns SALR_ERR_INVALID and touches nothing. */
+SALR_API int salr_free(salr_handle h);
+
+/* salr_info - shape and size of an encoded weight.  Any output pointer may be NULL.
+ * nnz = number of kept entries; bytes = blob bytes + offset-table bytes. */
+SALR_API int salr_info(salr_handle h, int64_t* N, int64_t* K, int64_t* nnz, int64_t* bytes);
+
+/* salr_format_view - read-only device pointers to the encoded format described under
+ * salr_encode (blob and offset table), owned by the handle. */
+SALR_API int salr_format_view(salr_handle h, const void** blob, int64_t* blob_bytes,
+                     const void** offsets, int64_t* n_offsets);
+
+/* salr_sync_status - synchronise `stream`, return the first device-side error recorded
+ * for this handle since the last call (SALR_OK if none) and clear it. */
+SALR_API int salr_sync_status(salr_handle h, void* stream);
+
+/* salr_status_string - static, human-readable name of a status code. */
+SALR_API const char* salr_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SALR_H_ */

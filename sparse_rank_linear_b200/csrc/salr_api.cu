@@ -1,0 +1,450 @@
+// salr_api.cu - host side of the SALR C ABI declared in include/salr.h: argument checks,
+// the weight handle and its device buffers, tensor maps, schedule choice and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <unordered_set>
+
+#include "../../include/salr.h"
+#include "salr_codec.cuh"
+#include "salr_linear.cuh"
+
+using namespace salr;
+
+namespace {
+
+constexpr uint64_t kMagic = 0x53414c5257454754ull;  // "SALRWEGT"
+
+struct Workspace {
+  float* ws = nullptr;
+  size_t ws_elems = 0;
+  uint32_t* counters = nullptr;
+  size_t n_counters = 0;
+};
+
+}  // namespace
+
+struct salr_weight_s {
+  uint64_t magic;
+  int device;
+  int64_t N, K, keep, nnz;
+  float sparsity;
+  uint8_t* blob;
+  int64_t blob_bytes;
+  uint32_t* offsets;
+  int64_t nblocks;
+  int* status;  // device status word (DEV_ERR_* bits)
+  Workspace work;
+  uint8_t* x_stage;  // salr_linear_host staging
+  size_t x_cap;
+  uint8_t* y_stage;
+  size_t y_cap;
+};
+
+namespace {
+
+std::mutex g_mu;
+std::unordered_set<salr_weight_s*>& live() {
+  static std::unordered_set<salr_weight_s*> s;
+  return s;
+}
+
+bool valid_handle(salr_handle h) {
+  std::lock_guard<std::mutex> g(g_mu);
+  return h && live().count(h) && h->magic == kMagic;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SALR_OK;
+  return e == cudaErrorMemoryAllocation ? SALR_ERR_OOM : SALR_ERR_CUDA;
+}
+
+#define SALR_TRY(expr)                      \
+  do {                                      \
+    const cudaError_t e_ = (expr);          \
+    if (e_ != cudaSuccess) return cuda_status(e_); \
+  } while (0)
+
+bool fake_oom() {
+  const char* v = getenv("SALR_FAKE_OOM");
+  return v && v[0] == '1';
+}
+
+cudaError_t dev_alloc(void** p, size_t bytes) {
+  if (fake_oom()) return cudaErrorMemoryAllocation;
+  return cudaMalloc(p, bytes);
+}
+
+int device_sms(int dev) {
+  static int cache[64] = {0};
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n > 0 ? n : 1;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map with 128-byte swizzle; out-of-range elements read as zero.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+              uint32_t box_inner, uint32_t box_outer) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+void release(salr_weight_s* h) {
+  cudaFree(h->blob);
+  cudaFree(h->offsets);
+  cudaFree(h->status);
+  cudaFree(h->work.ws);
+  cudaFree(h->work.counters);
+  cudaFree(h->x_stage);
+  cudaFree(h->y_stage);
+  h->magic = 0;
+  delete h;
+}
+
+// Grow the split-K workspace to hold `elems` floats and `ctrs` counters (both zeroed).
+int ensure_workspace(salr_weight_s* h, size_t elems, size_t ctrs, cudaStream_t st) {
+  if (elems > h->work.ws_elems) {
+    if (h->work.ws) {
+      SALR_TRY(cudaStreamSynchronize(st));
+      cudaFree(h->work.ws);
+      h->work.ws = nullptr;
+      h->work.ws_elems = 0;
+    }
+    void* p = nullptr;
+    SALR_TRY(dev_alloc(&p, elems * sizeof(float)));
+    h->work.ws = static_cast<float*>(p);
+    h->work.ws_elems = elems;
+    SALR_TRY(cudaMemsetAsync(p, 0, elems * sizeof(float), st));
+  }
+  if (ctrs > h->work.n_counters) {
+    if (h->work.counters) {
+      SALR_TRY(cudaStreamSynchronize(st));
+      cudaFree(h->work.counters);
+      h->work.counters = nullptr;
+      h->work.n_counters = 0;
+    }
+    void* p = nullptr;
+    SALR_TRY(dev_alloc(&p, ctrs * sizeof(uint32_t)));
+    h->work.counters = static_cast<uint32_t*>(p);
+    h->work.n_counters = ctrs;
+    SALR_TRY(cudaMemsetAsync(p, 0, ctrs * sizeof(uint32_t), st));
+  }
+  return SALR_OK;
+}
+
+struct Schedule {
+  int bnt, tt, splits;
+};
+
+Schedule choose_schedule(int64_t M, int64_t N, int64_t K, int sms) {
+  Schedule s;
+  s.bnt = M <= 16 ? 16 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  s.tt = static_cast<int>((M + s.bnt - 1) / s.bnt);
+  const int64_t tiles = (N / 128) * s.tt;
+  const int kblocks = static_cast<int>(K / 64);
+  int splits = 1;
+  if (tiles < sms) {
+    splits = static_cast<int>(sms / tiles);
+    if (splits > kblocks) splits = kblocks;
+    if (splits < 1) splits = 1;
+  }
+  s.splits = splits;
+  return s;
+}
+
+template <int BNT>
+int launch_linear(const LinParams& p, const CUtensorMap& tx, const CUtensorMap& ta,
+                  const CUtensorMap& tb, int grid, cudaStream_t st) {
+  constexpr int smem = LinLayout<BNT>::kSmemBytes;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
+  if (!attr_set[dev]) {
+    SALR_TRY(cudaFuncSetAttribute(salr_linear_kernel<BNT>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr_set[dev] = true;
+  }
+  salr_linear_kernel<BNT><<<grid, kLinThreads, smem, st>>>(p, tx, ta, tb);
+  SALR_TRY(cudaGetLastError());
+  return SALR_OK;
+}
+
+int check_linear_args(const void* X, int64_t M, salr_handle h, const void* A, const void* B,
+                      int64_t R, const void* Y) {
+  if (!valid_handle(h)) return SALR_ERR_INVALID;
+  if (!X || !Y || M < 1) return SALR_ERR_INVALID;
+  if (R < 0) return SALR_ERR_INVALID;
+  if (R > 0 && (!A || !B)) return SALR_ERR_INVALID;
+  if (R % 8 != 0 || R > 128) return SALR_ERR_UNSUPPORTED;
+  if (M > (1ll << 24)) return SALR_ERR_UNSUPPORTED;
+  if (!aligned16(X) || !aligned16(Y) || (R > 0 && (!aligned16(A) || !aligned16(B))))
+    return SALR_ERR_UNSUPPORTED;
+  return SALR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* salr_status_string(int status) {
+  switch (status) {
+    case SALR_OK: return "SALR_OK";
+    case SALR_ERR_INVALID: return "SALR_ERR_INVALID";
+    case SALR_ERR_UNSUPPORTED: return "SALR_ERR_UNSUPPORTED";
+    case SALR_ERR_CUDA: return "SALR_ERR_CUDA";
+    case SALR_ERR_OOM: return "SALR_ERR_OOM";
+    case SALR_ERR_TIMEOUT: return "SALR_ERR_TIMEOUT";
+    default: return "SALR_ERR_UNKNOWN";
+  }
+}
+
+int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* stream,
+                salr_handle* out) {
+  if (!W || !out) return SALR_ERR_INVALID;
+  if (!(sparsity >= 0.0f && sparsity < 1.0f)) return SALR_ERR_INVALID;
+  if (N < 128 || K < 64 || N % 128 || K % 64 || K > 64 * kMaxKBlocks) return SALR_ERR_UNSUPPORTED;
+  if (N > (1ll << 22)) return SALR_ERR_UNSUPPORTED;
+  if (!aligned16(W)) return SALR_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t keep = K - static_cast<int64_t>(std::floor(static_cast<double>(sparsity) * K));
+  const int64_t nwords = K / 64;
+  const int64_t nblocks = (N / 128) * nwords;
+
+  salr_weight_s* h = new (std::nothrow) salr_weight_s();
+  if (!h) return SALR_ERR_OOM;
+  std::memset(h, 0, sizeof(*h));
+  cudaGetDevice(&h->device);
+  h->N = N;
+  h->K = K;
+  h->keep = keep;
+  h->sparsity = sparsity;
+  h->nblocks = nblocks;
+
+  uint64_t* bits = nullptr;
+  uint32_t* size16 = nullptr;
+  unsigned long long* nnz_d = nullptr;
+  auto fail = [&](int code) {
+    cudaStreamSynchronize(st);
+    cudaFree(bits);
+    cudaFree(size16);
+    cudaFree(nnz_d);
+    release(h);
+    return code;
+  };
+  cudaError_t e;
+  if ((e = dev_alloc(reinterpret_cast<void**>(&h->status), sizeof(int))) != cudaSuccess ||
+      (e = dev_alloc(reinterpret_cast<void**>(&h->offsets), (nblocks + 1) * sizeof(uint32_t))) !=
+          cudaSuccess ||
+      (e = dev_alloc(reinterpret_cast<void**>(&bits), N * nwords * sizeof(uint64_t))) !=
+          cudaSuccess ||
+      (e = dev_alloc(reinterpret_cast<void**>(&size16), nblocks * sizeof(uint32_t))) !=
+          cudaSuccess ||
+      (e = dev_alloc(reinterpret_cast<void**>(&nnz_d), sizeof(unsigned long long))) != cudaSuccess)
+    return fail(cuda_status(e));
+  if ((e = cudaMemsetAsync(h->status, 0, sizeof(int), st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(nnz_d, 0, sizeof(unsigned long long), st)) != cudaSuccess)
+    return fail(cuda_status(e));
+
+  encode_mask_kernel<<<static_cast<unsigned>(N), kEncThreads, K * sizeof(uint16_t), st>>>(
+      static_cast<const uint16_t*>(W), static_cast<int>(K), static_cast<int>(keep), bits,
+      h->status);
+  encode_count_kernel<<<static_cast<unsigned>((nblocks + 7) / 8), 256, 0, st>>>(
+      bits, static_cast<int>(nwords), static_cast<int>(nblocks), size16, nnz_d);
+  encode_scan_kernel<<<1, 1024, 0, st>>>(size16, static_cast<int>(nblocks), h->offsets, h->status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return fail(cuda_status(e));
+
+  uint32_t total16 = 0;
+  int status = 0;
+  unsigned long long nnz = 0;
+  if ((e = cudaMemcpyAsync(&total16, h->offsets + nblocks, sizeof(uint32_t),
+                           cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(&status, h->status, sizeof(int), cudaMemcpyDeviceToHost, st)) !=
+          cudaSuccess ||
+      (e = cudaMemcpyAsync(&nnz, nnz_d, sizeof(unsigned long long), cudaMemcpyDeviceToHost,
+                           st)) != cudaSuccess ||
+      (e = cudaStreamSynchronize(st)) != cudaSuccess)
+    return fail(cuda_status(e));
+  if (status & DEV_ERR_NAN) return fail(SALR_ERR_INVALID);
+  if (status & DEV_ERR_RANGE) return fail(SALR_ERR_UNSUPPORTED);
+
+  h->nnz = static_cast<int64_t>(nnz);
+  h->blob_bytes = static_cast<int64_t>(total16) * 16;
+  if ((e = dev_alloc(reinterpret_cast<void**>(&h->blob), h->blob_bytes)) != cudaSuccess)
+    return fail(cuda_status(e));
+  encode_scatter_kernel<<<static_cast<unsigned>(nblocks), kBlockRows, 0, st>>>(
+      static_cast<const uint16_t*>(W), static_cast<int>(K), bits, h->offsets, h->blob);
+  if ((e = cudaGetLastError()) != cudaSuccess || (e = cudaStreamSynchronize(st)) != cudaSuccess)
+    return fail(cuda_status(e));
+  cudaFree(bits);
+  cudaFree(size16);
+  cudaFree(nnz_d);
+  h->magic = kMagic;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    live().insert(h);
+  }
+  *out = h;
+  return SALR_OK;
+}
+
+int salr_decode(salr_handle h, void* W_out, void* stream) {
+  if (!valid_handle(h) || !W_out) return SALR_ERR_INVALID;
+  if (!aligned16(W_out)) return SALR_ERR_UNSUPPORTED;
+  decode_kernel<<<static_cast<unsigned>(h->nblocks), kBlockRows, 0,
+                  static_cast<cudaStream_t>(stream)>>>(h->blob, h->offsets, static_cast<int>(h->K),
+                                                       static_cast<uint16_t*>(W_out));
+  SALR_TRY(cudaGetLastError());
+  return SALR_OK;
+}
+
+int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, const void* B_cat,
+                int64_t R, void* Y, void* stream) {
+  int rc = check_linear_args(X, M, h, A_cat, B_cat, R, Y);
+  if (rc != SALR_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Schedule sc = choose_schedule(M, h->N, h->K, device_sms(h->device));
+  LinParams p{};
+  p.blob = h->blob;
+  p.offsets = h->offsets;
+  p.Y = static_cast<uint16_t*>(Y);
+  p.status = h->status;
+  p.N = static_cast<int>(h->N);
+  p.K = static_cast<int>(h->K);
+  p.M = static_cast<int>(M);
+  p.R = static_cast<int>(R);
+  p.R16 = static_cast<int>((R + 15) / 16 * 16);
+  p.kblocks = static_cast<int>(h->K / 64);
+  p.TT = sc.tt;
+  p.splits = sc.splits;
+  if (sc.splits > 1) {
+    rc = ensure_workspace(h, static_cast<size_t>(sc.tt) * sc.bnt * h->N,
+                          static_cast<size_t>(h->N / 128) * sc.tt, st);
+    if (rc != SALR_OK) return rc;
+    p.ws = h->work.ws;
+    p.counters = h->work.counters;
+  }
+  CUtensorMap tx, ta, tb;
+  std::memset(&ta, 0, sizeof(ta));
+  std::memset(&tb, 0, sizeof(tb));
+  if (!make_map(&tx, X, h->K, M, 64, sc.bnt)) return SALR_ERR_CUDA;
+  if (R > 0) {
+    if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
+    if (!make_map(&tb, B_cat, h->N, R, 64, p.R16)) return SALR_ERR_CUDA;
+  }
+  const int grid = static_cast<int>((h->N / 128) * sc.tt * sc.splits);
+  switch (sc.bnt) {
+    case 16: return launch_linear<16>(p, tx, ta, tb, grid, st);
+    case 64: return launch_linear<64>(p, tx, ta, tb, grid, st);
+    case 128: return launch_linear<128>(p, tx, ta, tb, grid, st);
+    default: return launch_linear<256>(p, tx, ta, tb, grid, st);
+  }
+}
+
+int salr_linear_host(const void* X_host, int64_t M, salr_handle h, const void* A_cat,
+                     const void* B_cat, int64_t R, void* Y_host, void* stream) {
+  if (!valid_handle(h) || !X_host || !Y_host || M < 1) return SALR_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(M) * h->K * 2, yb = static_cast<size_t>(M) * h->N * 2;
+  if (xb > h->x_cap) {
+    SALR_TRY(cudaStreamSynchronize(st));
+    cudaFree(h->x_stage);
+    h->x_stage = nullptr;
+    h->x_cap = 0;
+    SALR_TRY(dev_alloc(reinterpret_cast<void**>(&h->x_stage), xb));
+    h->x_cap = xb;
+  }
+  if (yb > h->y_cap) {
+    SALR_TRY(cudaStreamSynchronize(st));
+    cudaFree(h->y_stage);
+    h->y_stage = nullptr;
+    h->y_cap = 0;
+    SALR_TRY(dev_alloc(reinterpret_cast<void**>(&h->y_stage), yb));
+    h->y_cap = yb;
+  }
+  SALR_TRY(cudaMemcpyAsync(h->x_stage, X_host, xb, cudaMemcpyHostToDevice, st));
+  const int rc = salr_linear(h->x_stage, M, h, A_cat, B_cat, R, h->y_stage, stream);
+  if (rc != SALR_OK) return rc;
+  SALR_TRY(cudaMemcpyAsync(Y_host, h->y_stage, yb, cudaMemcpyDeviceToHost, st));
+  return SALR_OK;
+}
+
+int salr_free(salr_handle h) {
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    if (!h || !live().count(h) || h->magic != kMagic) return SALR_ERR_INVALID;
+    live().erase(h);
+  }
+  cudaDeviceSynchronize();
+  release(h);
+  return SALR_OK;
+}
+
+int salr_info(salr_handle h, int64_t* N, int64_t* K, int64_t* nnz, int64_t* bytes) {
+  if (!valid_handle(h)) return SALR_ERR_INVALID;
+  if (N) *N = h->N;
+  if (K) *K = h->K;
+  if (nnz) *nnz = h->nnz;
+  if (bytes) *bytes = h->blob_bytes + (h->nblocks + 1) * static_cast<int64_t>(sizeof(uint32_t));
+  return SALR_OK;
+}
+
+int salr_format_view(salr_handle h, const void** blob, int64_t* blob_bytes, const void** offsets,
+                     int64_t* n_offsets) {
+  if (!valid_handle(h)) return SALR_ERR_INVALID;
+  if (blob) *blob = h->blob;
+  if (blob_bytes) *blob_bytes = h->blob_bytes;
+  if (offsets) *offsets = h->offsets;
+  if (n_offsets) *n_offsets = h->nblocks + 1;
+  return SALR_OK;
+}
+
+int salr_sync_status(salr_handle h, void* stream) {
+  if (!valid_handle(h)) return SALR_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int status = 0;
+  SALR_TRY(cudaStreamSynchronize(st));
+  SALR_TRY(cudaMemcpy(&status, h->status, sizeof(int), cudaMemcpyDeviceToHost));
+  SALR_TRY(cudaMemset(h->status, 0, sizeof(int)));
+  if (status == 0) return SALR_OK;
+  // a kernel that gave up may have left partial sums behind: start the next call clean
+  if (h->work.ws) SALR_TRY(cudaMemset(h->work.ws, 0, h->work.ws_elems * sizeof(float)));
+  if (h->work.counters)
+    SALR_TRY(cudaMemset(h->work.counters, 0, h->work.n_counters * sizeof(uint32_t)));
+  if (status & DEV_ERR_TIMEOUT) return SALR_ERR_TIMEOUT;
+  if (status & DEV_ERR_NAN) return SALR_ERR_INVALID;
+  return SALR_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

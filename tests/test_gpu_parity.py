@@ -1,0 +1,268 @@
+"""GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+encode/decode must match the oracle bit for bit (format bytes included); salr_linear
+must satisfy ||Y - Y*||_F <= 4e-3 ||Y*||_F and |Y - Y*| <= 1e-2 * S elementwise, S the
+sum of |products| feeding each output.  Small and ragged shapes are compared in full;
+the full-size workloads are compared on sampled rows and columns the oracle computes
+one by one, plus properties that hold at any size.
+"""
+import functools
+
+import numpy as np
+import pytest
+
+import oracle
+import salr_synth as synth
+from salr_synth import bf16_bits_to_f64
+from gpu_util import assert_close, to_bits, to_dev
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+salr = pytest.importorskip("sparse_rank_linear_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    from sparse_rank_linear_b200.build import build
+    build()
+    assert torch.cuda.is_available()
+    return salr.load_library()
+
+
+@functools.lru_cache(maxsize=None)
+def weight(name):
+    return synth.weight(synth.WORKLOADS[name])
+
+
+@functools.lru_cache(maxsize=None)
+def encoded(name, sparsity=0.5):
+    W = to_dev(weight(name))
+    h = salr.encode(W, sparsity)
+    torch.cuda.synchronize()
+    return h, W
+
+
+@functools.lru_cache(maxsize=None)
+def adapters_dev(name):
+    ad = synth.adapters(synth.WORKLOADS[name])
+    acat = np.concatenate([a for a, _ in ad], axis=1)  # caller-side layout: stack along rank
+    bcat = np.concatenate([b for _, b in ad], axis=0)
+    return ad, to_dev(acat), to_dev(bcat)
+
+
+def sample_idx(n, extra, seed, count):
+    rng = np.random.default_rng(seed)
+    idx = set(int(v) for v in extra if 0 <= v < n)
+    idx |= set(rng.integers(0, n, size=count).tolist())
+    return np.array(sorted(idx))
+
+
+# ---------------------------------------------------------------- codec
+
+@pytest.mark.parametrize("name", ["tiny", "q_proj"])
+def test_encode_bytes_and_decode_bitexact_full(name):
+    wl = synth.WORKLOADS[name]
+    w = weight(name)
+    m = oracle.magnitude_mask(w, 0.5)
+    wp = oracle.prune(w, m)
+    offs, blob = oracle.encode_format(wp, m)
+    h, _ = encoded(name)
+    gblob, goffs = h.format_tensors()
+    assert (goffs.cpu().numpy().view(np.uint32) == offs).all()
+    assert gblob.numel() == blob.size and (gblob.cpu().numpy() == blob).all()
+    assert (to_bits(h.decode()) == wp).all()
+    inf = h.info()
+    assert inf["nnz"] == wl.N * (wl.K // 2)
+    assert inf["bytes"] == blob.size + 4 * offs.size
+
+
+@pytest.mark.parametrize("name", ["up_proj", "down_proj", "large"])
+def test_encode_decode_full_size_sampled(name):
+    wl = synth.WORKLOADS[name]
+    h, W = encoded(name)
+    dec = h.decode()
+    # at any size: each entry is the weight or +0, exactly keep nonzero-or-kept per row
+    assert bool(((dec.view(torch.int16) == W.view(torch.int16)) |
+                 (dec.view(torch.int16) == 0)).all())
+    assert h.info()["nnz"] == wl.N * (wl.K // 2)
+    rows = sample_idx(wl.N, [0, 1, 127, 128, wl.N // 2, wl.N - 1], 11, 24)
+    w = weight(name)[rows]
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    assert (to_bits(dec[torch.as_tensor(rows, device="cuda")]) == wp).all()
+    # byte image of whole row tiles (first and last) against the oracle's encoder
+    gblob, goffs = h.format_tensors()
+    goffs = goffs.cpu().numpy().view(np.uint32).astype(np.int64)
+    kb = wl.K // 64
+    for tile in (0, wl.N // 128 - 1):
+        wt = weight(name)[128 * tile:128 * (tile + 1)]
+        mt = oracle.magnitude_mask(wt, 0.5)
+        o, b = oracle.encode_format(oracle.prune(wt, mt), mt)
+        lo, hi = goffs[tile * kb], goffs[(tile + 1) * kb]
+        assert (goffs[tile * kb:(tile + 1) * kb + 1] - lo == o).all()
+        assert (gblob[16 * lo:16 * hi].cpu().numpy() == b).all()
+
+
+def test_encode_handworked_block_and_edge_rows():
+    # one block (128 x 64): rows of ties, zeros of both signs, infinities
+    rng = np.random.default_rng(2)
+    vals = rng.choice(np.array([0.0, -0.0, 0.5, -0.5, 1.0, 2.0, -np.inf, np.inf], np.float32),
+                      size=(128, 64))
+    vals[0] = 0.25          # all equal: the first 32 are kept
+    vals[1] = -0.0
+    w = synth.f32_to_bf16_bits(vals)
+    m = oracle.magnitude_mask(w, 0.5)
+    wp = oracle.prune(w, m)
+    h = salr.encode(to_dev(w), 0.5)
+    assert (to_bits(h.decode()) == wp).all()
+    o, b = oracle.encode_format(wp, m)
+    gb, go = h.format_tensors()
+    assert (go.cpu().numpy().view(np.uint32) == o).all() and (gb.cpu().numpy() == b).all()
+    h.free()
+
+
+@pytest.mark.parametrize("s", [0.0, 0.3, 0.75])
+def test_encode_other_sparsities(s):
+    wl = synth.Workload("t", 256, 320, (8,), (4,))
+    w = synth.weight(wl)
+    s32 = float(np.float32(s))
+    m = oracle.magnitude_mask(w, s32)
+    wp = oracle.prune(w, m)
+    h = salr.encode(to_dev(w), s)
+    assert (to_bits(h.decode()) == wp).all()
+    assert h.info()["nnz"] == 256 * oracle.keep_count(320, s32)
+    h.free()
+
+
+def test_encode_rejects_nan():
+    w = synth.weight(synth.Workload("t", 128, 64, (8,), (1,))).copy()
+    w[77, 5] = 0x7FC1
+    with pytest.raises(salr.SalrError) as e:
+        salr.encode(to_dev(w), 0.5)
+    assert e.value.code == 1
+
+
+def test_double_free_rejected():
+    h = salr.encode(to_dev(synth.weight(synth.Workload("t", 128, 64, (8,), (1,)))), 0.5)
+    raw = h.handle
+    h.free()
+    assert salr.load_library().salr_free(raw) == 1
+
+
+# ---------------------------------------------------------------- linear
+
+def run_linear(name, M, rows=None, cols=None, R_on=True):
+    wl = synth.WORKLOADS[name]
+    h, _ = encoded(name)
+    x = synth.activations(wl, M)
+    ad, A, B = adapters_dev(name)
+    Y = salr.linear(to_dev(x), h, A if R_on else None, B if R_on else None)
+    assert h.sync_status() == 0
+    y = to_bits(Y)
+    ad_used = ad if R_on else []
+    if rows is None:
+        w = weight(name)
+        wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+        ystar = oracle.linear(x, wp, ad_used)
+        s = oracle.abs_bound(x, wp, ad_used)
+        return assert_close(y, ystar, s, f"{name} M={M}")
+    w = weight(name)[cols]
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    adc = [(a, b[:, cols]) for a, b in ad_used]
+    ystar = oracle.linear(x[rows], wp, adc)
+    s = oracle.abs_bound(x[rows], wp, adc)
+    return assert_close(y[np.ix_(rows, cols)], ystar, s, f"{name} M={M} sampled")
+
+
+@pytest.mark.parametrize("name,M", [("tiny", 16), ("q_proj", 1), ("q_proj", 16)])
+def test_linear_full_compare(name, M):
+    run_linear(name, M)
+
+
+def test_linear_no_adapter_q_proj():
+    run_linear("q_proj", 16, R_on=False)
+
+
+@pytest.mark.parametrize("name,M", [("up_proj", 2048), ("down_proj", 1), ("down_proj", 128),
+                                    ("down_proj", 4096), ("large", 16), ("large", 8192)])
+def test_linear_full_size_sampled(name, M):
+    wl = synth.WORKLOADS[name]
+    rows = sample_idx(M, [0, M - 1, 255, 256], 3, 40)
+    cols = sample_idx(wl.N, [0, 127, 128, wl.N - 1], 4, 200)
+    run_linear(name, M, rows, cols)
+
+
+@pytest.mark.parametrize("M", [1, 17, 100, 300])
+@pytest.mark.parametrize("R", [0, 8, 72, 128])
+def test_linear_ragged_shapes(M, R):
+    wl = synth.Workload("ragged", 384, 320, (R,) if R else (), (M,))
+    w = synth.weight(wl)
+    x = synth.activations(wl, M)
+    ad = synth.adapters(wl)
+    h = salr.encode(to_dev(w), 0.5)
+    A = to_dev(ad[0][0]) if R else None
+    B = to_dev(ad[0][1]) if R else None
+    Y = salr.linear(to_dev(x), h, A, B)
+    assert h.sync_status() == 0
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    assert_close(to_bits(Y), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad),
+                 f"ragged M={M} R={R}")
+    # a second call on the same handle reuses the (self-clearing) split-K workspace
+    Y2 = salr.linear(to_dev(x), h, A, B)
+    assert_close(to_bits(Y2), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad), "repeat")
+    h.free()
+
+
+@pytest.mark.parametrize("M", [256, 64])
+def test_identity_rows_reproduce_decoded_columns_bitexact(M):
+    # X = rows of the identity, no adapter: every output is a single product
+    K = 256
+    wl = synth.Workload("t", 384, K, (8,), (M,))
+    w = synth.weight(wl)
+    h = salr.encode(to_dev(w), 0.5)
+    x = np.zeros((M, K), np.uint16)
+    x[np.arange(M), np.arange(M)] = 0x3F80
+    Y = salr.linear(to_dev(x), h)
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    y = to_bits(Y)
+    expect = wp.T[:M].copy()
+    # -0 weights give -0 products; a split-K sum of +0 partials may return +0
+    assert ((y == expect) | ((expect == 0x8000) & (y == 0))).all()
+    h.free()
+
+
+def test_sparsity_zero_is_dense_gemm():
+    wl = synth.Workload("t", 256, 256, (16,), (16,))
+    w, x = synth.weight(wl), synth.activations(wl, 16)
+    ad = synth.adapters(wl)
+    h = salr.encode(to_dev(w), 0.0)
+    Y = salr.linear(to_dev(x), h, to_dev(ad[0][0]), to_dev(ad[0][1]))
+    assert_close(to_bits(Y), oracle.linear(x, w, ad), oracle.abs_bound(x, w, ad), "dense")
+    h.free()
+
+
+def test_linear_host_matches_device_path():
+    name, M = "q_proj", 16
+    h, _ = encoded(name)
+    _, A, B = adapters_dev(name)
+    x = synth.activations(synth.WORKLOADS[name], M)
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty(M, 4096, dtype=torch.bfloat16).pin_memory()
+    salr.linear_host(xh, h, A, B, yh)
+    torch.cuda.synchronize()
+    yd = salr.linear(to_dev(x), h, A, B)
+    w = weight(name)
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    ad = synth.adapters(synth.WORKLOADS[name])
+    assert_close(to_bits(yh), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad), "host")
+    assert_close(to_bits(yd), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad), "device")
+
+
+def test_linear_rejects_unsupported_rank():
+    h, _ = encoded("tiny")
+    x = to_dev(synth.activations(synth.WORKLOADS["tiny"], 4))
+    A = torch.zeros(256, 12, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(12, 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(salr.SalrError) as e:
+        salr.linear(x, h, A, B)
+    assert e.value.code == 2
