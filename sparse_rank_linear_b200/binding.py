@@ -150,11 +150,11 @@ class Weight:
 
 
 class _DevArray:
-    """Minimal __cuda_array_interface__ exporter for a read-only device range."""
+    """Minimal __cuda_array_interface__ exporter of a device range (only ever cloned)."""
 
     def __init__(self, ptr: int, n: int, typestr: str):
         self.__cuda_array_interface__ = {"shape": (n,), "typestr": typestr,
-                                         "data": (ptr, True), "version": 2, "strides": None}
+                                         "data": (ptr, False), "version": 2, "strides": None}
 
 
 def _device_view(ptr: int, n: int, typestr: str):
