@@ -14,6 +14,7 @@
 #include "../../include/salr.h"
 #include "salr_codec.cuh"
 #include "salr_linear.cuh"
+#include "salr_stream.cuh"
 
 using namespace salr;
 
@@ -28,6 +29,16 @@ struct Workspace {
   size_t n_counters = 0;
 };
 
+// Scratch of the persistent small-M kernel: partial sums [64 x N], per-row-tile
+// arrival counters, the fp32 t = X A_cat accumulator [64 x 128] and its three flags.
+// All of it is left zeroed by every successful call.
+struct StreamScratch {
+  float* ws = nullptr;
+  uint32_t* counters = nullptr;
+  float* tacc = nullptr;
+  uint32_t* tflags = nullptr;
+};
+
 }  // namespace
 
 struct salr_weight_s {
@@ -40,7 +51,9 @@ struct salr_weight_s {
   uint32_t* offsets;
   int64_t nblocks;
   int* status;  // device status word (DEV_ERR_* bits)
+  uint32_t max16;  // largest encoded block, 16-byte units
   Workspace work;
+  StreamScratch sscr;
   uint8_t* x_stage;  // salr_linear_host staging
   size_t x_cap;
   uint8_t* y_stage;
@@ -121,6 +134,10 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
 }
 
 void release(salr_weight_s* h) {
+  cudaFree(h->sscr.ws);
+  cudaFree(h->sscr.counters);
+  cudaFree(h->sscr.tacc);
+  cudaFree(h->sscr.tflags);
   cudaFree(h->blob);
   cudaFree(h->offsets);
   cudaFree(h->status);
@@ -201,6 +218,82 @@ int launch_linear(const LinParams& p, const CUtensorMap& tx, const CUtensorMap& 
   return SALR_OK;
 }
 
+
+// Persistent small-M path: one CTA per SM (cooperative launch: the adapter's t is
+// shared through global memory, so every CTA must be resident).
+constexpr int kStreamDecoders = 16;
+
+int ensure_stream_scratch(salr_weight_s* h, cudaStream_t st) {
+  if (h->sscr.ws) return SALR_OK;
+  void *a = nullptr, *b = nullptr, *c = nullptr, *d = nullptr;
+  const size_t wsb = static_cast<size_t>(64) * h->N * sizeof(float);
+  const size_t cb = static_cast<size_t>(h->N / 128) * sizeof(uint32_t);
+  const size_t tb = 64 * 128 * sizeof(float);
+  cudaError_t e;
+  if ((e = dev_alloc(&a, wsb)) != cudaSuccess || (e = dev_alloc(&b, cb)) != cudaSuccess ||
+      (e = dev_alloc(&c, tb)) != cudaSuccess || (e = dev_alloc(&d, 4 * sizeof(uint32_t))) != cudaSuccess) {
+    cudaFree(a);
+    cudaFree(b);
+    cudaFree(c);
+    cudaFree(d);
+    return cuda_status(e);
+  }
+  h->sscr.ws = static_cast<float*>(a);
+  h->sscr.counters = static_cast<uint32_t*>(b);
+  h->sscr.tacc = static_cast<float*>(c);
+  h->sscr.tflags = static_cast<uint32_t*>(d);
+  SALR_TRY(cudaMemsetAsync(a, 0, wsb, st));
+  SALR_TRY(cudaMemsetAsync(b, 0, cb, st));
+  SALR_TRY(cudaMemsetAsync(c, 0, tb, st));
+  SALR_TRY(cudaMemsetAsync(d, 0, 4 * sizeof(uint32_t), st));
+  return SALR_OK;
+}
+
+template <int BNT, bool SEL_LUT>
+int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
+                  const CUtensorMap& tb, int sms, cudaStream_t st) {
+  using L = StreamLayout<BNT>;
+  constexpr int kThreads = 32 * (kStreamFixedWarps + kStreamDecoders);
+  p.bcbuf = L::bcat_bytes(p.R16);
+  const int fixed = L::smem_bytes(p.cbuf, p.bcbuf, 0);
+  int stages = (kSmemLimit - fixed) / L::stage_bytes(p.cbuf);
+  if (stages > kStreamMaxStages) stages = kStreamMaxStages;
+  if (stages < 2) return SALR_ERR_UNSUPPORTED;
+  p.stages = stages;
+  const int smem = L::smem_bytes(p.cbuf, p.bcbuf, stages);
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
+  if (!attr_set[dev]) {
+    SALR_TRY(cudaFuncSetAttribute(salr_stream_kernel<BNT, kStreamDecoders, SEL_LUT>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
+    attr_set[dev] = true;
+  }
+  const long long units = p.units;
+  const int grid = static_cast<int>(units < sms ? units : sms);
+  p.tshare = grid < p.kblocks ? grid : p.kblocks;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  // One CTA per SM (the shared-memory footprint admits no second one) and the t-share
+  // work sits in the lowest-numbered CTAs, which wait on nothing before finishing it; so
+  // the only cross-CTA wait (for the complete t) cannot block those CTAs.  A cooperative
+  // launch would guarantee co-residency outright but costs several microseconds per
+  // call; SALR_COOPERATIVE=1 requests it.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  const char* coop = getenv("SALR_COOPERATIVE");
+  cfg.attrs = attr;
+  cfg.numAttrs = (coop && coop[0] == '1') ? 1 : 0;
+  SALR_TRY(cudaLaunchKernelEx(&cfg, salr_stream_kernel<BNT, kStreamDecoders, SEL_LUT>, p, tx, ta,
+                              tb));
+  return SALR_OK;
+}
+
 int check_linear_args(const void* X, int64_t M, salr_handle h, const void* A, const void* B,
                       int64_t R, const void* Y) {
   if (!valid_handle(h)) return SALR_ERR_INVALID;
@@ -254,7 +347,7 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
 
   uint64_t* bits = nullptr;
   uint32_t* size16 = nullptr;
-  unsigned long long* nnz_d = nullptr;
+  unsigned long long* nnz_d = nullptr;  // [0] kept entries, [1] largest block (16 B units)
   auto fail = [&](int code) {
     cudaStreamSynchronize(st);
     cudaFree(bits);
@@ -271,35 +364,38 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
           cudaSuccess ||
       (e = dev_alloc(reinterpret_cast<void**>(&size16), nblocks * sizeof(uint32_t))) !=
           cudaSuccess ||
-      (e = dev_alloc(reinterpret_cast<void**>(&nnz_d), sizeof(unsigned long long))) != cudaSuccess)
+      (e = dev_alloc(reinterpret_cast<void**>(&nnz_d), 2 * sizeof(unsigned long long))) !=
+          cudaSuccess)
     return fail(cuda_status(e));
   if ((e = cudaMemsetAsync(h->status, 0, sizeof(int), st)) != cudaSuccess ||
-      (e = cudaMemsetAsync(nnz_d, 0, sizeof(unsigned long long), st)) != cudaSuccess)
+      (e = cudaMemsetAsync(nnz_d, 0, 2 * sizeof(unsigned long long), st)) != cudaSuccess)
     return fail(cuda_status(e));
 
   encode_mask_kernel<<<static_cast<unsigned>(N), kEncThreads, K * sizeof(uint16_t), st>>>(
       static_cast<const uint16_t*>(W), static_cast<int>(K), static_cast<int>(keep), bits,
       h->status);
   encode_count_kernel<<<static_cast<unsigned>((nblocks + 7) / 8), 256, 0, st>>>(
-      bits, static_cast<int>(nwords), static_cast<int>(nblocks), size16, nnz_d);
+      bits, static_cast<int>(nwords), static_cast<int>(nblocks), size16, nnz_d,
+      reinterpret_cast<unsigned int*>(nnz_d + 1));
   encode_scan_kernel<<<1, 1024, 0, st>>>(size16, static_cast<int>(nblocks), h->offsets, h->status);
   if ((e = cudaGetLastError()) != cudaSuccess) return fail(cuda_status(e));
 
   uint32_t total16 = 0;
   int status = 0;
-  unsigned long long nnz = 0;
+  unsigned long long nnz[2] = {0, 0};
   if ((e = cudaMemcpyAsync(&total16, h->offsets + nblocks, sizeof(uint32_t),
                            cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
       (e = cudaMemcpyAsync(&status, h->status, sizeof(int), cudaMemcpyDeviceToHost, st)) !=
           cudaSuccess ||
-      (e = cudaMemcpyAsync(&nnz, nnz_d, sizeof(unsigned long long), cudaMemcpyDeviceToHost,
+      (e = cudaMemcpyAsync(nnz, nnz_d, 2 * sizeof(unsigned long long), cudaMemcpyDeviceToHost,
                            st)) != cudaSuccess ||
       (e = cudaStreamSynchronize(st)) != cudaSuccess)
     return fail(cuda_status(e));
   if (status & DEV_ERR_NAN) return fail(SALR_ERR_INVALID);
   if (status & DEV_ERR_RANGE) return fail(SALR_ERR_UNSUPPORTED);
 
-  h->nnz = static_cast<int64_t>(nnz);
+  h->nnz = static_cast<int64_t>(nnz[0]);
+  h->max16 = static_cast<uint32_t>(nnz[1]);
   h->blob_bytes = static_cast<int64_t>(total16) * 16;
   if ((e = dev_alloc(reinterpret_cast<void**>(&h->blob), h->blob_bytes)) != cudaSuccess)
     return fail(cuda_status(e));
@@ -334,6 +430,50 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   int rc = check_linear_args(X, M, h, A_cat, B_cat, R, Y);
   if (rc != SALR_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (M <= 64) {
+    rc = ensure_stream_scratch(h, st);
+    if (rc != SALR_OK) return rc;
+    const int bnt = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+    StreamParams sp{};
+    sp.blob = h->blob;
+    sp.offsets = h->offsets;
+    sp.Y = static_cast<uint16_t*>(Y);
+    sp.ws = h->sscr.ws;
+    sp.counters = h->sscr.counters;
+    sp.tacc = h->sscr.tacc;
+    sp.tflags = h->sscr.tflags;
+    sp.status = h->status;
+    sp.N = static_cast<int>(h->N);
+    sp.K = static_cast<int>(h->K);
+    sp.M = static_cast<int>(M);
+    sp.R = static_cast<int>(R);
+    sp.R16 = static_cast<int>((R + 15) / 16 * 16);
+    sp.kblocks = static_cast<int>(h->K / 64);
+    sp.RT = static_cast<int>(h->N / 128);
+    sp.units = sp.RT * sp.kblocks;
+    sp.cbuf = static_cast<int>((h->max16 * 16 + 32 + 1023) / 1024 * 1024);
+    CUtensorMap tx, ta, tb;
+    std::memset(&ta, 0, sizeof(ta));
+    std::memset(&tb, 0, sizeof(tb));
+    if (!make_map(&tx, X, h->K, M, 64, bnt)) return SALR_ERR_CUDA;
+    if (R > 0) {
+      if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
+      if (!make_map(&tb, B_cat, h->N, R, 64, sp.R16)) return SALR_ERR_CUDA;
+    }
+    const int sms = device_sms(h->device);
+    // selector source of the decoder (shared-memory table or registers); registers by
+    // default, SALR_DECODE_LUT=1 selects the table (kept for measurements)
+    const char* lutv = getenv("SALR_DECODE_LUT");
+    const bool use_lut = lutv && lutv[0] == '1';
+    switch (bnt) {
+      case 16: return use_lut ? launch_stream<16, true>(sp, tx, ta, tb, sms, st)
+                              : launch_stream<16, false>(sp, tx, ta, tb, sms, st);
+      case 32: return use_lut ? launch_stream<32, true>(sp, tx, ta, tb, sms, st)
+                              : launch_stream<32, false>(sp, tx, ta, tb, sms, st);
+      default: return use_lut ? launch_stream<64, true>(sp, tx, ta, tb, sms, st)
+                              : launch_stream<64, false>(sp, tx, ta, tb, sms, st);
+    }
+  }
   const Schedule sc = choose_schedule(M, h->N, h->K, device_sms(h->device));
   LinParams p{};
   p.blob = h->blob;
@@ -442,6 +582,12 @@ int salr_sync_status(salr_handle h, void* stream) {
   if (h->work.ws) SALR_TRY(cudaMemset(h->work.ws, 0, h->work.ws_elems * sizeof(float)));
   if (h->work.counters)
     SALR_TRY(cudaMemset(h->work.counters, 0, h->work.n_counters * sizeof(uint32_t)));
+  if (h->sscr.ws) {
+    SALR_TRY(cudaMemset(h->sscr.ws, 0, static_cast<size_t>(64) * h->N * sizeof(float)));
+    SALR_TRY(cudaMemset(h->sscr.counters, 0, static_cast<size_t>(h->N / 128) * sizeof(uint32_t)));
+    SALR_TRY(cudaMemset(h->sscr.tacc, 0, 64 * 128 * sizeof(float)));
+    SALR_TRY(cudaMemset(h->sscr.tflags, 0, 4 * sizeof(uint32_t)));
+  }
   if (status & DEV_ERR_TIMEOUT) return SALR_ERR_TIMEOUT;
   if (status & DEV_ERR_NAN) return SALR_ERR_INVALID;
   return SALR_ERR_UNSUPPORTED;

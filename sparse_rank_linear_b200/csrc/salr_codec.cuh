@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(kEncThreads) encode_mask_kernel(const uint16_t
 // One warp per block: number of kept entries and the block's size in 16-byte units.
 __global__ void encode_count_kernel(const uint64_t* __restrict__ bits, int nwords, int nblocks,
                                     uint32_t* __restrict__ size16,
-                                    unsigned long long* __restrict__ nnz_total) {
+                                    unsigned long long* __restrict__ nnz_total,
+                                    unsigned int* __restrict__ max16) {
   const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= nblocks) return;
@@ -152,6 +153,7 @@ __global__ void encode_count_kernel(const uint64_t* __restrict__ bits, int nword
   if (lane == 0) {
     size16[b] = (kBitmapBytes + 2 * c + 15) / 16;
     atomicAdd(nnz_total, static_cast<unsigned long long>(c));
+    atomicMax(max16, (kBitmapBytes + 2 * c + 15) / 16);
   }
 }
 

@@ -80,10 +80,6 @@ __device__ __forceinline__ bool aborted(Ctrl* c) {
   return *reinterpret_cast<volatile int*>(&c->abort) != 0;
 }
 
-__device__ __forceinline__ void named_bar(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 template <int BNT>
 __global__ void __launch_bounds__(kLinThreads, 1)
     salr_linear_kernel(const __grid_constant__ LinParams p, const __grid_constant__ CUtensorMap tmX,

@@ -1,0 +1,682 @@
+// salr_stream.cuh - persistent SALR layer kernel for small token counts (decode shapes).
+//
+// Same layer as salr_linear_kernel, Y = X (M (.) W)^T + (X A_cat) B_cat, organised for
+// the HBM-bound regime (M <= 64) where decoding the bitmap blocks is the whole cost:
+//
+// * Work split: the weight's 128 x 64 blocks, in storage order, are cut into one
+//   contiguous range per CTA (one CTA per SM, every SM the same number of blocks).  A
+//   range covers one or more row-tile segments; a segment that does not cover a whole
+//   row tile adds its fp32 partial into a workspace, and the last segment of the tile to
+//   arrive (an arrival counter, no waiting) writes the bf16 output.
+// * Stage 1 decode (SALR technical summary, Methodology 4): decoder warps work in
+//   groups, each group on a different block so that several blocks are in flight.  A
+//   warp first turns the bitmap words of its 32 rows into the offset of every (row,
+//   8-column chunk) in the compact value array, then expands one bitmap byte per lane:
+//   an aligned 12-value window is loaded from shared memory, shifted to the chunk's first
+//   value and spread over the eight columns by byte permutes whose selectors come from a
+//   16-entry nibble lookup table.
+// * Stage 2: tcgen05 bf16 MMAs into a double-buffered TMEM accumulator, pipelined
+//   against the decode through shared-memory stages filled by TMA.
+// * Concatenated adapter (Methodology 3): t = X A_cat is computed once per call.  Each
+//   CTA multiplies a share of the K dimension on the tensor cores and adds its part into
+//   an fp32 buffer; when all parts have arrived every row tile reads t back, rounds it to
+//   bf16 once and adds B_cat^T t^T to its accumulator with one more MMA.  This needs all
+//   CTAs resident at once, which the host guarantees with a cooperative launch.
+//
+// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 epilogue (and the
+// adapter's t share), 6.. decoders.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include "salr_codec.cuh"
+#include "sm100.cuh"
+
+namespace salr {
+
+constexpr int kStreamFixedWarps = 6;
+constexpr int kStreamGroups = 4;  // decoder groups, each decodes a different block
+constexpr int kStreamMaxUnitsPerCta = 4096;
+constexpr int kStreamMaxStages = 8;
+
+struct StreamParams {
+  const uint8_t* blob;
+  const uint32_t* offsets;
+  uint16_t* Y;
+  float* ws;           // [BNT x N] fp32 partial sums of split row tiles, zero between calls
+  uint32_t* counters;  // [RT] arrivals per row tile, zero between calls
+  float* tacc;         // [BNT x R16] fp32 accumulator of t = X A_cat, zero between calls
+  uint32_t* tflags;    // [0] t parts arrived, [1] t complete, [2] t readers done
+  int* status;
+  int N, K, M, R, R16;
+  int kblocks;  // K / 64
+  int RT;       // N / 128
+  int units;    // RT * kblocks
+  int tshare;   // CTAs 0 .. tshare-1 compute a share of t (tshare = min(grid, kblocks))
+  int cbuf;     // per-stage bytes for one compact block (bitmap + values), multiple of 1024
+  int bcbuf;    // bytes of the B_cat^T tile / t-share buffer (0 without adapter), x1024
+  int stages;
+};
+
+template <int BNT>
+struct StreamLayout {
+  static constexpr int kAbuf = 16384;
+  static constexpr int kXbuf = BNT * 128;
+  static constexpr int kCs = 4096;                     // 128 rows x 8 chunks: offset | byte << 16
+  static constexpr int kTbuf = BNT * 256;              // t as [BNT x 128] bf16, two chunks
+  // B_cat^T tile [128 x R16] and, at kernel start, the t-share stage (A_cat block + X)
+  __host__ __device__ static int bcat_bytes(int R16) {
+    if (R16 == 0) return 0;
+    const int a = 256 * R16, b = 16384 + kXbuf;
+    return ((a > b ? a : b) + 1023) / 1024 * 1024;
+  }
+  __host__ __device__ static int stage_bytes(int cbuf) { return kAbuf + kXbuf + cbuf + kCs; }
+  __host__ __device__ static int fixed_off(int cbuf, int stages) { return stages * stage_bytes(cbuf); }
+  __host__ __device__ static int smem_bytes(int cbuf, int bcbuf, int stages) {
+    return fixed_off(cbuf, stages) + kTbuf + bcbuf + 4096 /*lut + ctrl*/ + 1024 /*align*/;
+  }
+};
+
+struct StreamCtrl {
+  uint64_t full[kStreamMaxStages], dec[kStreamMaxStages], empty[kStreamMaxStages];
+  uint64_t accfull[2], accempty[2];
+  uint64_t bcfull, bcempty, tready, tsfull, tsfree, tsdone, fin;
+  uint32_t tmem;
+  int abort;
+  int flag;
+  uint32_t lut[32];
+};
+
+__device__ __forceinline__ void stream_timeout(const StreamParams& p, StreamCtrl* c) {
+  atomicOr(p.status, DEV_ERR_TIMEOUT);
+  *reinterpret_cast<volatile int*>(&c->abort) = 1;
+}
+__device__ __forceinline__ bool stream_aborted(StreamCtrl* c) {
+  return *reinterpret_cast<volatile int*>(&c->abort) != 0;
+}
+
+// Bounded wait for a global flag written by another CTA (acquire at gpu scope).
+__device__ __forceinline__ bool wait_global_flag(const uint32_t* flag, uint32_t want) {
+  const long long t0 = clock64();
+  for (;;) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v == want) return true;
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+    __nanosleep(64);
+  }
+}
+
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint2 lds64(const uint8_t* p) {
+  return *reinterpret_cast<const uint2*>(p);
+}
+
+// CTA that owns unit u (block u in storage order) under the even split of U units.
+__device__ __forceinline__ int owner_of(long long u, long long U, int G) {
+  int c = static_cast<int>((u * G) / U);
+  while (c + 1 < G && ((c + 1) * U) / G <= u) ++c;
+  while (c > 0 && (c * U) / G > u) --c;
+  return c;
+}
+
+// Selectors for the nibble lookup table.  For a 4-bit mask t over 4 output columns and
+// a window E0 = (h0, h1), E1 = (h2, h3) holding the nibble's kept values in order:
+//   out0 = prmt(E0, 0, lo) places h0/h1 in columns 0/1 (or zero),
+//   pair = prmt(E0, E1, lo >> 16) brings the next two unused values to the bottom,
+//   out1 = prmt(pair, 0, hi) places them in columns 2/3 (or zero).
+__device__ __forceinline__ uint32_t pat2(uint32_t v) {
+  return v == 0 ? 0x4444u : v == 1 ? 0x4410u : v == 2 ? 0x1044u : 0x3210u;
+}
+
+__device__ __forceinline__ uint32_t funnel16(uint32_t lo, uint32_t hi, uint32_t sh) {
+  return __funnelshift_r(lo, hi, sh);
+}
+
+// Expand one bitmap byte `b` whose values start at halfword p of the block's value
+// array (shared memory, 16-byte aligned, readable 24 bytes past its end).  The window
+// is 8 values from the 8-byte boundary at or below p, plus 4 more only for lanes whose
+// high nibble reaches past them.  SEL_LUT picks the byte-permute selectors from the
+// nibble table in shared memory, otherwise they are built in registers:
+//   PAT(v), v the 2-bit mask of two columns, is 0x4444 / 0x4410 / 0x1044 / 0x3210 (both
+//   zero, first value low, first value high, both values), looked up for all four
+//   column pairs at once by one byte permute of a constant table;
+//   PAIR(s) = 0x3210 + 0x2222 s brings values s, s+1 of a window to the bottom.
+template <bool SEL_LUT>
+__device__ __forceinline__ uint4 expand_byte(const uint8_t* vals, uint32_t p, uint32_t b,
+                                             const uint32_t* lut) {
+  const uint8_t* wp = vals + ((p & ~3u) << 1);
+  const uint2 a0 = lds64(wp), a1 = lds64(wp + 8);
+  const uint32_t o = p & 3u;
+  const uint32_t x = o + __popc(b & 15u);  // first value of the high nibble
+  uint2 a2 = make_uint2(0u, 0u);
+  if (x >= 5u) a2 = lds64(wp + 16);
+  const uint32_t W0 = a0.x, W1 = a0.y, W2 = a1.x, W3 = a1.y, W4 = a2.x, W5 = a2.y;
+  // low nibble: window at halfword o
+  const bool o2 = (o & 2u) != 0;
+  const uint32_t sh0 = (o & 1u) << 4;
+  const uint32_t U0 = o2 ? W1 : W0, U1 = o2 ? W2 : W1, U2 = o2 ? W3 : W2;
+  const uint32_t L0 = funnel16(U0, U1, sh0), L1 = funnel16(U1, U2, sh0);
+  // high nibble: window at halfword x
+  const bool x4 = (x & 4u) != 0, x2 = (x & 2u) != 0;
+  const uint32_t sh1 = (x & 1u) << 4;
+  const uint32_t T0 = x4 ? W2 : W0, T1 = x4 ? W3 : W1, T2 = x4 ? W4 : W2, T3 = x4 ? W5 : W3;
+  const uint32_t V0 = x2 ? T1 : T0, V1 = x2 ? T2 : T1, V2 = x2 ? T3 : T2;
+  const uint32_t H0 = funnel16(V0, V1, sh1), H1 = funnel16(V1, V2, sh1);
+  uint32_t pat01, pat23, pr0, pr1;
+  if constexpr (SEL_LUT) {
+    const uint32_t lo0 = lut[2 * (b & 15u)], hi0 = lut[2 * (b & 15u) + 1];
+    const uint32_t lo1 = lut[2 * (b >> 4)], hi1 = lut[2 * (b >> 4) + 1];
+    pat01 = (lo0 & 0xFFFFu) | (hi0 << 16);
+    pat23 = (lo1 & 0xFFFFu) | (hi1 << 16);
+    pr0 = lo0 >> 16;
+    pr1 = lo1 >> 16;
+  } else {
+    const uint32_t bs = (b & 3u) | ((b & 0xCu) << 6) | ((b & 0x30u) << 12) | ((b & 0xC0u) << 18);
+    const uint32_t idx = bs * 0x22u + 0x10101010u;
+    pat01 = __byte_perm(0x44104444u, 0x32101044u, idx);
+    pat23 = __byte_perm(0x44104444u, 0x32101044u, idx >> 16);
+    pr0 = 0x3210u + 0x2222u * __popc(b & 3u);
+    pr1 = 0x3210u + 0x2222u * __popc(b & 0x30u);
+  }
+  uint4 out;
+  out.x = __byte_perm(L0, 0u, pat01);
+  out.y = __byte_perm(__byte_perm(L0, L1, pr0), 0u, pat01 >> 16);
+  out.z = __byte_perm(H0, 0u, pat23);
+  out.w = __byte_perm(__byte_perm(H0, H1, pr1), 0u, pat23 >> 16);
+  return out;
+}
+
+template <int BNT, int NDEC, bool SEL_LUT>
+__global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
+    salr_stream_kernel(const __grid_constant__ StreamParams p,
+                       const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB) {
+  using L = StreamLayout<BNT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int S = p.stages;
+  const int SB = L::stage_bytes(p.cbuf);
+  auto abuf = [&](int s) { return smem + s * SB; };
+  auto xbuf = [&](int s) { return smem + s * SB + L::kAbuf; };
+  auto cbuf = [&](int s) { return smem + s * SB + L::kAbuf + L::kXbuf; };
+  auto csb = [&](int s) {
+    return reinterpret_cast<uint32_t*>(smem + s * SB + L::kAbuf + L::kXbuf + p.cbuf);
+  };
+  uint8_t* tbuf = smem + L::fixed_off(p.cbuf, S);
+  uint8_t* bcbuf = tbuf + L::kTbuf;  // B_cat^T tile; at kernel start, the t-share stage
+  StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(bcbuf + p.bcbuf);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool adapter = p.R > 0;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const long long U = p.units;
+  const int u0 = static_cast<int>((static_cast<long long>(cta) * U) / G);
+  const int u1 = static_cast<int>((static_cast<long long>(cta + 1) * U) / G);
+  const int KB = p.kblocks;
+  // t share of this CTA: K blocks cta, cta + tshare, ... (only CTAs below tshare)
+  const int nts = (adapter && cta < p.tshare) ? (KB - cta + p.tshare - 1) / p.tshare : 0;
+  constexpr uint32_t kCols = 4 * BNT < 32 ? 32 : 4 * BNT;  // 2 accumulators + t share
+  // the producer's first batch of block offsets is requested before the set-up below
+  uint32_t offv = 0, offx = 0;
+  if (warp == 0) {
+    offv = (u0 + lane <= p.units) ? __ldg(p.offsets + u0 + lane) : 0u;
+    offx = (u0 + 32 <= p.units) ? __ldg(p.offsets + u0 + 32) : 0u;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->dec[s], NDEC / kStreamGroups);
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&ctrl->accfull[x], 1);
+      mbar_init(&ctrl->accempty[x], 4);
+    }
+    mbar_init(&ctrl->bcfull, 1);
+    mbar_init(&ctrl->bcempty, 1);
+    mbar_init(&ctrl->tready, 4);
+    mbar_init(&ctrl->tsfull, 1);
+    mbar_init(&ctrl->tsfree, 1);
+    mbar_init(&ctrl->tsdone, 1);
+    mbar_init(&ctrl->fin, 1);
+    ctrl->abort = 0;
+    ctrl->flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 16) {
+    const uint32_t t = threadIdx.x;
+    ctrl->lut[2 * t] = pat2(t & 3u) | ((0x3210u + 0x2222u * __popc(t & 3u)) << 16);
+    ctrl->lut[2 * t + 1] = pat2(t >> 2);
+  }
+  if (warp == 1) tmem_alloc(&ctrl->tmem, kCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem;
+  const uint32_t tmem_ts = tmem + 2 * BNT;  // t^T share accumulator [128 ranks x BNT]
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    // Warp-uniform loop; lane 0 issues.  Block offsets are fetched 32 at a time by the
+    // whole warp so that no copy waits on a dependent global load.  The t-share rounds
+    // share their buffer with the B_cat tile, so round r+1 is issued once round r has
+    // been consumed and the B_cat tile of a segment only after its last block.
+    const uint32_t xbytes = BNT * 128;
+    int ts_next = 0;  // next t-share round to issue (lane 0)
+    auto issue_ts = [&](int r) {
+      const int kb = cta + r * p.tshare;
+      mbar_arrive_expect_tx(&ctrl->tsfull, (p.R > 64 ? 16384u : 8192u) + xbytes);
+      tma_load_2d(bcbuf, &tmA, 0, kb * 64, &ctrl->tsfull);
+      if (p.R > 64) tma_load_2d(bcbuf + 8192, &tmA, 64, kb * 64, &ctrl->tsfull);
+      tma_load_2d(bcbuf + 16384, &tmX, kb * 64, 0, &ctrl->tsfull);
+    };
+    // blocking: issue every remaining round, then wait until the last one is consumed
+    auto finish_ts = [&]() -> bool {
+      while (ts_next < nts) {
+        if (!mbar_wait(&ctrl->tsfree, (ts_next - 1) & 1)) return false;
+        issue_ts(ts_next++);
+      }
+      return nts == 0 || mbar_wait(&ctrl->tsfree, (nts - 1) & 1);
+    };
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      if (adapter) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+      }
+      if (nts > 0) issue_ts(ts_next++);
+    }
+    int it = 0, nad = 0, obase = u0;
+    bool stop = false, bc_pending = false;
+    for (int u = u0; u < u1 && !stop;) {
+      const int i = u / KB, kba = u % KB;
+      const int kbb = min(KB, kba + (u1 - u));
+      for (int kb = kba; kb < kbb; ++kb, ++it) {
+        const int unit = i * KB + kb;
+        if (unit >= obase + 32) {
+          obase = unit;
+          offv = (obase + lane <= p.units) ? __ldg(p.offsets + obase + lane) : 0u;
+          offx = (obase + 32 <= p.units) ? __ldg(p.offsets + obase + 32) : 0u;
+        }
+        const int k = unit - obase;
+        const uint32_t o0 = __shfl_sync(0xffffffffu, offv, k);
+        const uint32_t o1n = __shfl_sync(0xffffffffu, offv, (k + 1) & 31);
+        const uint32_t o1 = (k + 1 < 32) ? o1n : offx;
+        int fail = 0;
+        if (lane == 0) {
+          if (ts_next < nts && mbar_try_wait(smem_u32(&ctrl->tsfree), (ts_next - 1) & 1))
+            issue_ts(ts_next++);
+          const int s = it % S;
+          if (!mbar_wait(&ctrl->empty[s], ((it / S) & 1) ^ 1) || stream_aborted(ctrl)) {
+            stream_timeout(p, ctrl);
+            fail = 1;
+          } else {
+            const uint32_t cb = (o1 - o0) * 16u;
+            mbar_arrive_expect_tx(&ctrl->full[s], cb + xbytes);
+            bulk_g2s(cbuf(s), p.blob + static_cast<size_t>(o0) * 16, cb, &ctrl->full[s]);
+            tma_load_2d(xbuf(s), &tmX, kb * 64, 0, &ctrl->full[s]);
+          }
+        }
+        if (__shfl_sync(0xffffffffu, fail, 0)) {
+          stop = true;
+          break;
+        }
+      }
+      if (!stop && adapter && kba == 0) {
+        int fail = 0;
+        if (lane == 0) {
+          if (!finish_ts() || !mbar_wait(&ctrl->bcempty, (nad & 1) ^ 1)) {
+            stream_timeout(p, ctrl);
+            fail = 1;
+          } else {
+            mbar_arrive_expect_tx(&ctrl->bcfull, 256u * p.R16);
+            tma_load_2d(bcbuf, &tmB, i * 128, 0, &ctrl->bcfull);
+            tma_load_2d(bcbuf + p.R16 * 128, &tmB, i * 128 + 64, 0, &ctrl->bcfull);
+            bc_pending = true;
+          }
+        }
+        ++nad;
+        if (__shfl_sync(0xffffffffu, fail, 0)) stop = true;
+      }
+      u = i * KB + kbb;
+    }
+    if (lane == 0) {
+      if (!stop && !finish_ts()) stream_timeout(p, ctrl);
+      if (stream_aborted(ctrl)) {
+        // let copies this thread started land before the CTA may exit
+        for (int s = 0; s < S; ++s)
+          if (it > s) mbar_wait(&ctrl->full[(it - 1 - s) % S], ((it - 1 - s) / S) & 1);
+        if (bc_pending) mbar_wait(&ctrl->bcfull, (nad - 1) & 1);
+        if (ts_next > 0) mbar_wait(&ctrl->tsfull, (ts_next - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, BNT, 0, 0);
+      constexpr uint32_t idesc_mn = idesc_bf16(128, BNT, 1, 0);
+      bool ok = true;
+      int ts_done = 0;  // t-share rounds multiplied so far
+      auto mma_ts = [&]() {
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(bcbuf), x0 = smem_u32(bcbuf + 16384);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16_ss(tmem_ts, smem_desc_sw128(a0 + 2048 * k, 8192, 1024),
+                      smem_desc_sw128(x0 + 32 * k, 16, 1024), idesc_mn, (ts_done | k) != 0);
+        mma_commit(&ctrl->tsfree);
+        if (++ts_done == nts) mma_commit(&ctrl->tsdone);
+      };
+      int it = 0, seg = 0, nad = 0;
+      for (int u = u0; u < u1 && ok && !stream_aborted(ctrl); ++seg) {
+        const int i = u / KB, kba = u % KB;
+        const int kbb = min(KB, kba + (u1 - u));
+        const int x = seg & 1;
+        (void)i;
+        if (!mbar_wait(&ctrl->accempty[x], ((seg >> 1) & 1) ^ 1)) {
+          stream_timeout(p, ctrl);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + x * BNT;
+        for (int kb = kba; kb < kbb; ++kb, ++it) {
+          const int s = it % S;
+          if (ts_done < nts && mbar_try_wait(smem_u32(&ctrl->tsfull), ts_done & 1)) mma_ts();
+          if (!mbar_wait(&ctrl->dec[s], (it / S) & 1)) {
+            stream_timeout(p, ctrl);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(abuf(s)), x0 = smem_u32(xbuf(s));
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(acc, smem_desc_sw128(a0 + 32 * k, 16, 1024),
+                        smem_desc_sw128(x0 + 32 * k, 16, 1024), idesc, (kb != kba) || k != 0);
+          mma_commit(&ctrl->empty[s]);
+        }
+        if (!ok) break;
+        if (adapter && kba == 0) {
+          while (ok && ts_done < nts) {
+            if (!mbar_wait(&ctrl->tsfull, ts_done & 1)) {
+              ok = false;
+              break;
+            }
+            mma_ts();
+          }
+          if (!ok || !mbar_wait(&ctrl->tready, 0) || !mbar_wait(&ctrl->bcfull, nad & 1)) {
+            stream_timeout(p, ctrl);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b0 = smem_u32(bcbuf), t0 = smem_u32(tbuf);
+          for (int k = 0; k < p.R16 / 16; ++k)
+            mma_bf16_ss(acc, smem_desc_sw128(b0 + 2048 * k, p.R16 * 128, 1024),
+                        smem_desc_sw128(t0 + (k >> 2) * (BNT * 128) + (k & 3) * 32, 16, 1024),
+                        idesc_mn, 1);
+          mma_commit(&ctrl->bcempty);
+          ++nad;
+        }
+        mma_commit(&ctrl->accfull[x]);
+        u = i * KB + kbb;
+      }
+      while (ok && !stream_aborted(ctrl) && ts_done < nts) {
+        if (!mbar_wait(&ctrl->tsfull, ts_done & 1)) {
+          stream_timeout(p, ctrl);
+          break;
+        }
+        mma_ts();
+      }
+      mma_commit(&ctrl->fin);
+      if (!mbar_wait(&ctrl->fin, 0)) stream_timeout(p, ctrl);
+    }
+  } else if (warp < 6) {
+    // ================================================================ epilogue (warps 2-5)
+    const int q = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    const int r = 32 * q + lane;  // weight row within the tile; rank index for t
+    __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(p.Y);
+    bool ok = true;
+    // ---- 1. this CTA's share of t = X A_cat: drain t^T from TMEM into the fp32 buffer
+    if (nts > 0) {
+      ok = mbar_wait(&ctrl->tsdone, 0);
+      if (!ok) stream_timeout(p, ctrl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        for (int c = 0; c < BNT; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem_ts + lane_base + c, v);
+          tmem_ld_wait();
+          if (r < p.R) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              if (c + e < p.M) atomicAdd(&p.tacc[(c + e) * p.R16 + r], __uint_as_float(v[e]));
+          }
+        }
+      }
+    }
+    if (adapter) {
+      __threadfence();
+      named_bar(1, 128);
+      if (threadIdx.x == 64 && nts > 0) {
+        const uint32_t prev = atomicAdd(&p.tflags[0], 1u);
+        if (prev == static_cast<uint32_t>(p.tshare - 1)) {
+          __threadfence();
+          p.tflags[0] = 0u;
+          st_release(&p.tflags[1], 1u);
+        }
+      }
+    }
+    // ---- 2. if this CTA owns the first block of some row tile, it applies the adapter:
+    //         wait for the complete t, round it to bf16 into shared memory
+    bool has_adapter_seg = false;
+    for (int u = u0; u < u1; u = (u / KB + 1) * KB)
+      if (u % KB == 0) has_adapter_seg = true;
+    bool t_read = false;
+    if (adapter && has_adapter_seg) {
+      if (threadIdx.x == 64) ctrl->flag = wait_global_flag(&p.tflags[1], 1u) ? 1 : 0;
+      named_bar(1, 128);
+      if (*reinterpret_cast<volatile int*>(&ctrl->flag) == 0) {
+        if (threadIdx.x == 64) stream_timeout(p, ctrl);
+      } else {
+        __threadfence();
+        for (int e = threadIdx.x - 64; e < BNT * p.R16; e += 128) {
+          const int m = e / p.R16, j = e % p.R16;
+          float v = 0.0f;
+          if (m < p.M && j < p.R) v = __ldcg(&p.tacc[m * p.R16 + j]);
+          const int chunk = j >> 6, cc = j & 63;
+          uint8_t* dst = tbuf + chunk * (BNT * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
+                         (((cc >> 3) ^ (m & 7)) << 4) + (cc & 7) * 2;
+          *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
+        }
+        fence_proxy_async_smem();
+        t_read = true;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->tready);
+    }
+    // ---- 3. per segment: drain the accumulator, write Y or a partial sum
+    int seg = 0;
+    for (int u = u0; u < u1; ++seg) {
+      const int i = u / KB, kba = u % KB;
+      const int kbb = min(KB, kba + (u1 - u));
+      const int x = seg & 1;
+      bool okw = mbar_wait(&ctrl->accfull[x], (seg >> 1) & 1);
+      if (!okw) stream_timeout(p, ctrl);
+      okw = __all_sync(0xffffffffu, okw) && !stream_aborted(ctrl);
+      named_bar(1, 128);
+      if (threadIdx.x == 64) ctrl->flag = okw ? 2 : 0;
+      named_bar(1, 128);
+      if (*reinterpret_cast<volatile int*>(&ctrl->flag) != 2) break;
+      tc_fence_after();
+      const size_t n = static_cast<size_t>(i) * 128 + r;
+      const bool whole = kba == 0 && kbb == KB;
+      float4* wrow = reinterpret_cast<float4*>(p.ws + n * BNT);  // partials, [N x BNT]
+#pragma unroll
+      for (int c = 0; c < BNT; c += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + x * BNT + lane_base + c, v);
+        tmem_ld_wait();
+        if (whole) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (c + e < p.M)
+              Y[(c + e) * static_cast<size_t>(p.N) + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
+        } else {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            if (c + 4 * q4 < p.M)
+              atomicAdd(&wrow[(c >> 2) + q4],
+                        make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                    __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3])));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->accempty[x]);
+      if (!whole) {
+        // publish this CTA's partial: barrier, then one release/acquire counter update
+        named_bar(1, 128);
+        if (threadIdx.x == 64) {
+          const int segs = owner_of(static_cast<long long>(i) * KB + KB - 1, U, G) -
+                           owner_of(static_cast<long long>(i) * KB, U, G) + 1;
+          uint32_t prev;
+          asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                       : "=r"(prev)
+                       : "l"(p.counters + i)
+                       : "memory");
+          ctrl->flag = prev == static_cast<uint32_t>(segs - 1) ? 3 : 2;
+        }
+        named_bar(1, 128);
+        if (*reinterpret_cast<volatile int*>(&ctrl->flag) == 3) {
+#pragma unroll
+          for (int c = 0; c < BNT; c += 4) {
+            if (c < p.M) {
+              const float4 t = __ldcg(&wrow[c >> 2]);
+              const float tv[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (c + e < p.M)
+                  Y[(c + e) * static_cast<size_t>(p.N) + n] = __float2bfloat16_rn(tv[e]);
+              __stcg(&wrow[c >> 2], make_float4(0.f, 0.f, 0.f, 0.f));
+            }
+          }
+          if (threadIdx.x == 64) p.counters[i] = 0u;
+        }
+      }
+      u = i * KB + kbb;
+    }
+    // ---- 4. every CTA checks in as a reader of t; the last one clears it for next call
+    if (adapter) {
+      named_bar(1, 128);
+      if (threadIdx.x == 64) {
+        bool ready = t_read || wait_global_flag(&p.tflags[1], 1u);
+        if (!ready) {
+          stream_timeout(p, ctrl);
+          ctrl->flag = 0;
+        } else {
+          const uint32_t prev = atomicAdd(&p.tflags[2], 1u);
+          ctrl->flag = prev == static_cast<uint32_t>(G - 1) ? 4 : 0;
+        }
+      }
+      named_bar(1, 128);
+      if (*reinterpret_cast<volatile int*>(&ctrl->flag) == 4) {
+        for (int e = threadIdx.x - 64; e < BNT * p.R16; e += 128) p.tacc[e] = 0.0f;
+        __threadfence();
+        named_bar(1, 128);
+        if (threadIdx.x == 64) {
+          p.tflags[2] = 0u;
+          st_release(&p.tflags[1], 0u);
+        }
+      }
+    }
+  } else {
+    // ================================================================ decoders
+    // NDEC warps in kStreamGroups groups; group g decodes blocks g, g + groups, ... so
+    // that several blocks are in flight.  Each warp owns 32 rows of its group's block:
+    // it first builds the value offset of each (row, 8-column chunk) of those rows
+    // (thread per row), then expands them one bitmap byte per lane.
+    constexpr int WPG = NDEC / kStreamGroups;  // warps per group
+    static_assert(WPG * 32 == 128 || WPG * 32 == 64 || WPG * 32 == 256, "rows per warp");
+    constexpr int RPW = 128 / WPG;             // rows per warp
+    const int dw = warp - kStreamFixedWarps;
+    const int g = dw / WPG, wg = dw % WPG;
+    const uint32_t* lut = ctrl->lut;
+    const int nunits = u1 - u0;
+    for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
+      const int s = it % S;
+      if (!mbar_wait(&ctrl->full[s], (it / S) & 1)) {
+        stream_timeout(p, ctrl);
+        break;
+      }
+      const uint8_t* cb = cbuf(s);
+      const uint64_t* bm = reinterpret_cast<const uint64_t*>(cb);
+      const uint8_t* vals = cb + kBitmapBytes;
+      uint32_t* cs = csb(s);
+      uint8_t* ab = abuf(s);
+      // ---- chunk offsets of this warp's rows
+      uint32_t base = 0;
+      for (int rr = lane; rr < RPW * wg; rr += 32) base += __popcll(bm[rr]);
+      base = warp_sum(base);
+#pragma unroll
+      for (int h = 0; h < RPW / 32; ++h) {
+        const int row = RPW * wg + 32 * h + lane;
+        const uint64_t w = bm[row];
+        const uint32_t lo = static_cast<uint32_t>(w), hi = static_cast<uint32_t>(w >> 32);
+        const uint32_t clo = __popc(lo), cnt = clo + __popc(hi);
+        const uint32_t inc = warp_incl_scan(cnt);
+        const uint32_t rs = base + inc - cnt;
+        base += __shfl_sync(0xffffffffu, inc, 31);
+        uint32_t bl = lo - ((lo >> 1) & 0x55555555u);
+        bl = (bl & 0x33333333u) + ((bl >> 2) & 0x33333333u);
+        bl = (bl + (bl >> 4)) & 0x0F0F0F0Fu;
+        uint32_t bh = hi - ((hi >> 1) & 0x55555555u);
+        bh = (bh & 0x33333333u) + ((bh >> 2) & 0x33333333u);
+        bh = (bh + (bh >> 4)) & 0x0F0F0F0Fu;
+        const uint32_t plo = bl * 0x01010100u;
+        const uint32_t phi = bh * 0x01010100u + clo * 0x01010101u;
+        // entry = offset | bitmap byte << 16, two uint4 per row
+        uint4 o0, o1;
+        o0.x = rs + (plo & 0xFFu) + ((lo & 0xFFu) << 16);
+        o0.y = rs + ((plo >> 8) & 0xFFu) + (((lo >> 8) & 0xFFu) << 16);
+        o0.z = rs + ((plo >> 16) & 0xFFu) + (((lo >> 16) & 0xFFu) << 16);
+        o0.w = rs + (plo >> 24) + ((lo >> 24) << 16);
+        o1.x = rs + (phi & 0xFFu) + ((hi & 0xFFu) << 16);
+        o1.y = rs + ((phi >> 8) & 0xFFu) + (((hi >> 8) & 0xFFu) << 16);
+        o1.z = rs + ((phi >> 16) & 0xFFu) + (((hi >> 16) & 0xFFu) << 16);
+        o1.w = rs + (phi >> 24) + ((hi >> 24) << 16);
+        reinterpret_cast<uint4*>(cs)[2 * row] = o0;
+        reinterpret_cast<uint4*>(cs)[2 * row + 1] = o1;
+      }
+      __syncwarp();
+      // ---- expansion: 4 rows x 8 chunks per step
+#pragma unroll 2
+      for (int st = 0; st < RPW / 4; ++st) {
+        const int row = RPW * wg + 4 * st + (lane >> 3);
+        const int c = lane & 7;
+        const uint32_t e = cs[row * 8 + c];
+        const uint4 out = expand_byte<SEL_LUT>(vals, e & 0xFFFFu, e >> 16, lut);
+        *reinterpret_cast<uint4*>(ab + row * 128 + ((c ^ (row & 7)) << 4)) = out;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->dec[s]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+}  // namespace salr
