@@ -26,6 +26,7 @@ SIGNATURES = {
     "salr_decode": (_I, [_P, _P, _P]),
     "salr_linear": (_I, [_P, _I64, _P, _P, _P, _I64, _P, _P]),
     "salr_linear_host": (_I, [_P, _I64, _P, _P, _P, _I64, _P, _P]),
+    "salr_linear_noalloc": (_I, [_P, _I64, _P, _P, _P, _I64, _P, _P]),
     "salr_free": (_I, [_P]),
     "salr_info": (_I, [_P, ctypes.POINTER(_I64), ctypes.POINTER(_I64), ctypes.POINTER(_I64),
                        ctypes.POINTER(_I64)]),

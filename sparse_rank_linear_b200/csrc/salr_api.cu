@@ -594,3 +594,88 @@ int salr_sync_status(salr_handle h, void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// salr_linear_noalloc: the small-M layer with its scratch in a fixed device array.
+//
+// Some callers cannot let a library allocate device memory on their behalf: serving
+// loops that pre-plan every byte of device memory and forbid allocations once running
+// (an allocation can fail under memory pressure or stall the device while it is made),
+// and embedders whose own allocator owns the GPU.  For them the scratch the small-M
+// kernel needs lives in one file-scope array, allocated when the library's device code
+// is loaded and held by every GPU that loads it until the process exits.
+// ------------------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kNoAllocMaxM = 16;     // tokens per call
+constexpr int64_t kNoAllocMaxN = 32768;  // output features
+// layout: [counters: N/128 u32][t flags: 4 u32][t accumulator: 16 x 128 f32][partials: N x 16 f32]
+constexpr size_t kNaCounters = 0;
+constexpr size_t kNaFlags = kNaCounters + (kNoAllocMaxN / 128) * sizeof(uint32_t);
+constexpr size_t kNaTacc = kNaFlags + 256;
+constexpr size_t kNaWs = kNaTacc + 16 * 128 * sizeof(float);
+constexpr size_t kNaBytes = kNaWs + static_cast<size_t>(kNoAllocMaxN) * 16 * sizeof(float);
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
+
+std::mutex g_na_mu;
+unsigned char* g_na_ptr[64] = {nullptr};
+
+// Device address of the scratch array for the current device (looked up once per device).
+int noalloc_scratch(int dev, unsigned char** out) {
+  if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_na_mu);
+  if (!g_na_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return SALR_ERR_CUDA;
+    g_na_ptr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_na_ptr[dev];
+  return SALR_OK;
+}
+
+}  // namespace
+
+extern "C" int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, const void* A_cat,
+                                   const void* B_cat, int64_t R, void* Y, void* stream) {
+  int rc = check_linear_args(X, M, h, A_cat, B_cat, R, Y);
+  if (rc != SALR_OK) return rc;
+  if (M > kNoAllocMaxM || h->N > kNoAllocMaxN) return SALR_ERR_UNSUPPORTED;
+  int dev = 0;
+  SALR_TRY(cudaGetDevice(&dev));
+  if (dev != h->device) return SALR_ERR_INVALID;
+  unsigned char* scr = nullptr;
+  rc = noalloc_scratch(dev, &scr);
+  if (rc != SALR_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // zero what this call reads before writing: counters, flags, t and its partial sums
+  SALR_TRY(cudaMemsetAsync(scr, 0, kNaWs + static_cast<size_t>(h->N) * 16 * sizeof(float), st));
+  StreamParams sp{};
+  sp.blob = h->blob;
+  sp.offsets = h->offsets;
+  sp.Y = static_cast<uint16_t*>(Y);
+  sp.ws = reinterpret_cast<float*>(scr + kNaWs);
+  sp.counters = reinterpret_cast<uint32_t*>(scr + kNaCounters);
+  sp.tacc = reinterpret_cast<float*>(scr + kNaTacc);
+  sp.tflags = reinterpret_cast<uint32_t*>(scr + kNaFlags);
+  sp.status = h->status;
+  sp.N = static_cast<int>(h->N);
+  sp.K = static_cast<int>(h->K);
+  sp.M = static_cast<int>(M);
+  sp.R = static_cast<int>(R);
+  sp.R16 = static_cast<int>((R + 15) / 16 * 16);
+  sp.kblocks = static_cast<int>(h->K / 64);
+  sp.RT = static_cast<int>(h->N / 128);
+  sp.units = sp.RT * sp.kblocks;
+  sp.cbuf = static_cast<int>((h->max16 * 16 + 32 + 1023) / 1024 * 1024);
+  CUtensorMap tx, ta, tb;
+  std::memset(&ta, 0, sizeof(ta));
+  std::memset(&tb, 0, sizeof(tb));
+  if (!make_map(&tx, X, h->K, M, 64, 16)) return SALR_ERR_CUDA;
+  if (R > 0) {
+    if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
+    if (!make_map(&tb, B_cat, h->N, R, 64, sp.R16)) return SALR_ERR_CUDA;
+  }
+  return launch_stream<16, false>(sp, tx, ta, tb, device_sms(h->device), st);
+}
