@@ -136,16 +136,16 @@ SALR_API int salr_linear_host(const void* X_host, int64_t M, salr_handle h, cons
  * part of the method.  It computes the same layer as salr_linear (same arguments, same
  * arithmetic and tolerance) for M <= 16 and N <= 32768, and never allocates device
  * memory: the scratch it needs (partial sums, arrival counters, the fp32 t = X A_cat
- * accumulator and its flags, about 2 MiB) is one fixed array in the library's device
+ * accumulator and its flags, about 3.3 MiB) is one fixed array in the library's device
  * code, present on every GPU that loads the library until the process exits.  Meant for
  * callers whose device memory is planned up front and who may not allocate during
  * inference (a failing or stalling cudaMalloc is not acceptable there).  The handle and
  * all inputs and outputs are still the caller's.
  *
- * Returns SALR_ERR_UNSUPPORTED for M > 16 or N > 32768.  The first call on a device
+ * Returns SALR_ERR_UNSUPPORTED for M > 16 or N > 32768 (or a GPU with more than 160 SMs).  The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress) and should come before
- * any stream capture.  Every call first zeroes the part of the array it uses and leaves
- * it zeroed when it succeeds.  All calls on one device share the one array, so calls
+ * any stream capture.  Every call first zeroes the counters and accumulators it reads
+ * (the partial-sum slots are always written before they are read).  All calls on one device share the one array, so calls
  * whose executions overlap on the GPU (different streams, or different threads) race
  * and give wrong results: order them on one stream.
  */

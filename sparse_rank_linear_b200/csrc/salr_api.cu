@@ -29,9 +29,10 @@ struct Workspace {
   size_t n_counters = 0;
 };
 
-// Scratch of the persistent small-M kernel: partial sums [64 x N], per-row-tile
-// arrival counters, the fp32 t = X A_cat accumulator [64 x 128] and its three flags.
-// All of it is left zeroed by every successful call.
+// Scratch of the persistent small-M kernel: partial-sum slots ((SMs + N/128) x 128 x 64
+// fp32, overwritten by every call), per-row-tile arrival counters, the fp32 t = X A_cat
+// accumulator [64 x 128] and its three flags (these three are left zeroed by every
+// successful call).
 struct StreamScratch {
   float* ws = nullptr;
   uint32_t* counters = nullptr;
@@ -223,10 +224,14 @@ int launch_linear(const LinParams& p, const CUtensorMap& tx, const CUtensorMap& 
 // shared through global memory, so every CTA must be resident).
 constexpr int kStreamDecoders = 16;
 
+size_t stream_slot_bytes(const salr_weight_s* h) {
+  return static_cast<size_t>(device_sms(h->device) + h->N / 128) * 128 * 64 * sizeof(float);
+}
+
 int ensure_stream_scratch(salr_weight_s* h, cudaStream_t st) {
   if (h->sscr.ws) return SALR_OK;
   void *a = nullptr, *b = nullptr, *c = nullptr, *d = nullptr;
-  const size_t wsb = static_cast<size_t>(64) * h->N * sizeof(float);
+  const size_t wsb = stream_slot_bytes(h);
   const size_t cb = static_cast<size_t>(h->N / 128) * sizeof(uint32_t);
   const size_t tb = 64 * 128 * sizeof(float);
   cudaError_t e;
@@ -255,12 +260,15 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   using L = StreamLayout<BNT>;
   constexpr int kThreads = 32 * (kStreamFixedWarps + kStreamDecoders);
   p.bcbuf = L::bcat_bytes(p.R16);
-  const int fixed = L::smem_bytes(p.cbuf, p.bcbuf, 0);
-  int stages = (kSmemLimit - fixed) / L::stage_bytes(p.cbuf);
-  if (stages > kStreamMaxStages) stages = kStreamMaxStages;
-  if (stages < 2) return SALR_ERR_UNSUPPORTED;
-  p.stages = stages;
-  const int smem = L::smem_bytes(p.cbuf, p.bcbuf, stages);
+  // decoded-tile ring: one entry per decoder group plus one; the rest of shared memory
+  // becomes compact-block entries, which set how many blocks are in flight from HBM
+  p.sa = kStreamGroups + 1;
+  const int fixed = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, 0, kStreamGroups);
+  int sc = (kSmemLimit - fixed) / p.cbuf;
+  if (sc > kStreamMaxC) sc = kStreamMaxC;
+  if (sc < kStreamGroups + 1) return SALR_ERR_UNSUPPORTED;
+  p.sc = sc;
+  const int smem = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, p.sc, kStreamGroups);
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -583,7 +591,6 @@ int salr_sync_status(salr_handle h, void* stream) {
   if (h->work.counters)
     SALR_TRY(cudaMemset(h->work.counters, 0, h->work.n_counters * sizeof(uint32_t)));
   if (h->sscr.ws) {
-    SALR_TRY(cudaMemset(h->sscr.ws, 0, static_cast<size_t>(64) * h->N * sizeof(float)));
     SALR_TRY(cudaMemset(h->sscr.counters, 0, static_cast<size_t>(h->N / 128) * sizeof(uint32_t)));
     SALR_TRY(cudaMemset(h->sscr.tacc, 0, 64 * 128 * sizeof(float)));
     SALR_TRY(cudaMemset(h->sscr.tflags, 0, 4 * sizeof(uint32_t)));
@@ -609,12 +616,15 @@ namespace {
 
 constexpr int64_t kNoAllocMaxM = 16;     // tokens per call
 constexpr int64_t kNoAllocMaxN = 32768;  // output features
-// layout: [counters: N/128 u32][t flags: 4 u32][t accumulator: 16 x 128 f32][partials: N x 16 f32]
+constexpr int kNoAllocMaxSMs = 160;      // CTAs of the persistent kernel
+// layout: [counters: N/128 u32][t flags: 4 u32][t accumulator: 16 x 128 f32]
+//         [partial slots: (SMs + N/128) x 128 x 16 f32]
 constexpr size_t kNaCounters = 0;
 constexpr size_t kNaFlags = kNaCounters + (kNoAllocMaxN / 128) * sizeof(uint32_t);
 constexpr size_t kNaTacc = kNaFlags + 256;
 constexpr size_t kNaWs = kNaTacc + 16 * 128 * sizeof(float);
-constexpr size_t kNaBytes = kNaWs + static_cast<size_t>(kNoAllocMaxN) * 16 * sizeof(float);
+constexpr size_t kNaBytes =
+    kNaWs + static_cast<size_t>(kNoAllocMaxSMs + kNoAllocMaxN / 128) * 128 * 16 * sizeof(float);
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
 
@@ -642,6 +652,7 @@ extern "C" int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, cons
   int rc = check_linear_args(X, M, h, A_cat, B_cat, R, Y);
   if (rc != SALR_OK) return rc;
   if (M > kNoAllocMaxM || h->N > kNoAllocMaxN) return SALR_ERR_UNSUPPORTED;
+  if (device_sms(h->device) > kNoAllocMaxSMs) return SALR_ERR_UNSUPPORTED;
   int dev = 0;
   SALR_TRY(cudaGetDevice(&dev));
   if (dev != h->device) return SALR_ERR_INVALID;
@@ -649,8 +660,9 @@ extern "C" int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, cons
   rc = noalloc_scratch(dev, &scr);
   if (rc != SALR_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // zero what this call reads before writing: counters, flags, t and its partial sums
-  SALR_TRY(cudaMemsetAsync(scr, 0, kNaWs + static_cast<size_t>(h->N) * 16 * sizeof(float), st));
+  // zero what must start at zero: arrival counters, t flags and the t accumulator (the
+  // partial-sum slots are always written before they are read)
+  SALR_TRY(cudaMemsetAsync(scr, 0, kNaWs, st));
   StreamParams sp{};
   sp.blob = h->blob;
   sp.offsets = h->offsets;

@@ -6,8 +6,8 @@
 // * Work split: the weight's 128 x 64 blocks, in storage order, are cut into one
 //   contiguous range per CTA (one CTA per SM, every SM the same number of blocks).  A
 //   range covers one or more row-tile segments; a segment that does not cover a whole
-//   row tile adds its fp32 partial into a workspace, and the last segment of the tile to
-//   arrive (an arrival counter, no waiting) writes the bf16 output.
+//   row tile stores its fp32 partial in a slot of its own, and the last segment of the
+//   tile to arrive (an arrival counter, no waiting) sums the slots into the bf16 output.
 // * Stage 1 decode (SALR technical summary, Methodology 4): decoder warps work in
 //   groups, each group on a different block so that several blocks are in flight.  A
 //   warp first turns the bitmap words of its 32 rows into the offset of every (row,
@@ -23,8 +23,8 @@
 //   bf16 once and adds B_cat^T t^T to its accumulator with one more MMA.  This needs all
 //   CTAs resident at once, which the host guarantees with a cooperative launch.
 //
-// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 epilogue (and the
-// adapter's t share), 6.. decoders.
+// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-9 epilogue in two groups
+// (group 0 also the adapter's t share), 10.. decoders.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -33,16 +33,17 @@
 
 namespace salr {
 
-constexpr int kStreamFixedWarps = 6;
+constexpr int kStreamFixedWarps = 10;  // producer, MMA, 2 x 4 epilogue warps
 constexpr int kStreamGroups = 4;  // decoder groups, each decodes a different block
 constexpr int kStreamMaxUnitsPerCta = 4096;
-constexpr int kStreamMaxStages = 8;
+constexpr int kStreamMaxA = 8;   // decoded-tile ring
+constexpr int kStreamMaxC = 16;  // compact-block ring
 
 struct StreamParams {
   const uint8_t* blob;
   const uint32_t* offsets;
   uint16_t* Y;
-  float* ws;           // [BNT x N] fp32 partial sums of split row tiles, zero between calls
+  float* ws;           // fp32 partials of split row tiles: (grid + RT) slots of [128 x BNT]
   uint32_t* counters;  // [RT] arrivals per row tile, zero between calls
   float* tacc;         // [BNT x R16] fp32 accumulator of t = X A_cat, zero between calls
   uint32_t* tflags;    // [0] t parts arrived, [1] t complete, [2] t readers done
@@ -54,7 +55,8 @@ struct StreamParams {
   int tshare;   // CTAs 0 .. tshare-1 compute a share of t (tshare = min(grid, kblocks))
   int cbuf;     // per-stage bytes for one compact block (bitmap + values), multiple of 1024
   int bcbuf;    // bytes of the B_cat^T tile / t-share buffer (0 without adapter), x1024
-  int stages;
+  int sa;       // entries of the decoded-tile ring (tile + X tile each)
+  int sc;       // entries of the compact-block ring
 };
 
 template <int BNT>
@@ -62,6 +64,7 @@ struct StreamLayout {
   static constexpr int kAbuf = 16384;
   static constexpr int kXbuf = BNT * 128;
   static constexpr int kCs = 4096;                     // 128 rows x 8 chunks: offset | byte << 16
+  static constexpr int kAent = kAbuf + kXbuf;          // one decoded-tile ring entry
   static constexpr int kTbuf = BNT * 256;              // t as [BNT x 128] bf16, two chunks
   // B_cat^T tile [128 x R16] and, at kernel start, the t-share stage (A_cat block + X)
   __host__ __device__ static int bcat_bytes(int R16) {
@@ -69,22 +72,29 @@ struct StreamLayout {
     const int a = 256 * R16, b = 16384 + kXbuf;
     return ((a > b ? a : b) + 1023) / 1024 * 1024;
   }
-  __host__ __device__ static int stage_bytes(int cbuf) { return kAbuf + kXbuf + cbuf + kCs; }
-  __host__ __device__ static int fixed_off(int cbuf, int stages) { return stages * stage_bytes(cbuf); }
-  __host__ __device__ static int smem_bytes(int cbuf, int bcbuf, int stages) {
-    return fixed_off(cbuf, stages) + kTbuf + bcbuf + 4096 /*lut + ctrl*/ + 1024 /*align*/;
+  // layout: [A ring: sa x (tile, X)] [C ring: sc x cbuf] [chunk tables: groups] [t] [B_cat] [ctrl]
+  __host__ __device__ static int c_off(int sa) { return sa * kAent; }
+  __host__ __device__ static int cs_off(int cbuf, int sa, int sc) { return c_off(sa) + sc * cbuf; }
+  __host__ __device__ static int fixed_off(int cbuf, int sa, int sc, int groups) {
+    return cs_off(cbuf, sa, sc) + groups * kCs;
+  }
+  __host__ __device__ static int smem_bytes(int cbuf, int bcbuf, int sa, int sc, int groups) {
+    return fixed_off(cbuf, sa, sc, groups) + kTbuf + bcbuf + 1024 /*ctrl*/ + 4096 /*lut*/ +
+           1024 /*align*/;
   }
 };
 
 struct StreamCtrl {
-  uint64_t full[kStreamMaxStages], dec[kStreamMaxStages], empty[kStreamMaxStages];
+  uint64_t cfull[kStreamMaxC], cempty[kStreamMaxC];
+  uint64_t dec[kStreamMaxA], xfull[kStreamMaxA], aempty[kStreamMaxA];
   uint64_t accfull[2], accempty[2];
   uint64_t bcfull, bcempty, tready, tsfull, tsfree, tsdone, fin;
   uint32_t tmem;
   int abort;
-  int flag;
-  uint32_t lut[32];
+  int flag[2];
 };
+
+static_assert(sizeof(StreamCtrl) <= 1024, "control block");
 
 __device__ __forceinline__ void stream_timeout(const StreamParams& p, StreamCtrl* c) {
   atomicOr(p.status, DEV_ERR_TIMEOUT);
@@ -167,12 +177,11 @@ __device__ __forceinline__ uint4 expand_byte(const uint8_t* vals, uint32_t p, ui
   const uint32_t H0 = funnel16(V0, V1, sh1), H1 = funnel16(V1, V2, sh1);
   uint32_t pat01, pat23, pr0, pr1;
   if constexpr (SEL_LUT) {
-    const uint32_t lo0 = lut[2 * (b & 15u)], hi0 = lut[2 * (b & 15u) + 1];
-    const uint32_t lo1 = lut[2 * (b >> 4)], hi1 = lut[2 * (b >> 4) + 1];
-    pat01 = (lo0 & 0xFFFFu) | (hi0 << 16);
-    pat23 = (lo1 & 0xFFFFu) | (hi1 << 16);
-    pr0 = lo0 >> 16;
-    pr1 = lo1 >> 16;
+    const uint4 e = reinterpret_cast<const uint4*>(lut)[b];
+    pat01 = e.x;
+    pat23 = e.y;
+    pr0 = e.z;
+    pr1 = e.z >> 16;
   } else {
     const uint32_t bs = (b & 3u) | ((b & 0xCu) << 6) | ((b & 0x30u) << 12) | ((b & 0xC0u) << 18);
     const uint32_t idx = bs * 0x22u + 0x10101010u;
@@ -199,17 +208,17 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int S = p.stages;
-  const int SB = L::stage_bytes(p.cbuf);
-  auto abuf = [&](int s) { return smem + s * SB; };
-  auto xbuf = [&](int s) { return smem + s * SB + L::kAbuf; };
-  auto cbuf = [&](int s) { return smem + s * SB + L::kAbuf + L::kXbuf; };
-  auto csb = [&](int s) {
-    return reinterpret_cast<uint32_t*>(smem + s * SB + L::kAbuf + L::kXbuf + p.cbuf);
+  const int SA = p.sa, SC = p.sc;
+  auto abuf = [&](int s) { return smem + s * L::kAent; };
+  auto xbuf = [&](int s) { return smem + s * L::kAent + L::kAbuf; };
+  auto cbuf = [&](int s) { return smem + L::c_off(SA) + s * p.cbuf; };
+  auto csb = [&](int g) {
+    return reinterpret_cast<uint32_t*>(smem + L::cs_off(p.cbuf, SA, SC) + g * L::kCs);
   };
-  uint8_t* tbuf = smem + L::fixed_off(p.cbuf, S);
+  uint8_t* tbuf = smem + L::fixed_off(p.cbuf, SA, SC, kStreamGroups);
   uint8_t* bcbuf = tbuf + L::kTbuf;  // B_cat^T tile; at kernel start, the t-share stage
   StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(bcbuf + p.bcbuf);
+  uint32_t* lutp = reinterpret_cast<uint32_t*>(bcbuf + p.bcbuf + 1024);  // 256 x 16 B
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool adapter = p.R > 0;
@@ -229,10 +238,14 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
   }
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&ctrl->full[s], 1);
+    for (int s = 0; s < SC; ++s) {
+      mbar_init(&ctrl->cfull[s], 1);
+      mbar_init(&ctrl->cempty[s], NDEC / kStreamGroups);
+    }
+    for (int s = 0; s < SA; ++s) {
       mbar_init(&ctrl->dec[s], NDEC / kStreamGroups);
-      mbar_init(&ctrl->empty[s], 1);
+      mbar_init(&ctrl->xfull[s], 1);
+      mbar_init(&ctrl->aempty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&ctrl->accfull[x], 1);
@@ -246,13 +259,17 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     mbar_init(&ctrl->tsdone, 1);
     mbar_init(&ctrl->fin, 1);
     ctrl->abort = 0;
-    ctrl->flag = 0;
+    ctrl->flag[0] = ctrl->flag[1] = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x < 16) {
-    const uint32_t t = threadIdx.x;
-    ctrl->lut[2 * t] = pat2(t & 3u) | ((0x3210u + 0x2222u * __popc(t & 3u)) << 16);
-    ctrl->lut[2 * t + 1] = pat2(t >> 2);
+  if (SEL_LUT && threadIdx.x < 256) {
+    const uint32_t b = threadIdx.x;
+    uint4 e;
+    e.x = pat2(b & 3u) | (pat2((b >> 2) & 3u) << 16);
+    e.y = pat2((b >> 4) & 3u) | (pat2(b >> 6) << 16);
+    e.z = (0x3210u + 0x2222u * __popc(b & 3u)) | ((0x3210u + 0x2222u * __popc(b & 0x30u)) << 16);
+    e.w = 0u;
+    reinterpret_cast<uint4*>(lutp)[b] = e;
   }
   if (warp == 1) tmem_alloc(&ctrl->tmem, kCols);
   tc_fence_before();
@@ -312,15 +329,14 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         if (lane == 0) {
           if (ts_next < nts && mbar_try_wait(smem_u32(&ctrl->tsfree), (ts_next - 1) & 1))
             issue_ts(ts_next++);
-          const int s = it % S;
-          if (!mbar_wait(&ctrl->empty[s], ((it / S) & 1) ^ 1) || stream_aborted(ctrl)) {
+          const int s = it % SC;
+          if (!mbar_wait(&ctrl->cempty[s], ((it / SC) & 1) ^ 1) || stream_aborted(ctrl)) {
             stream_timeout(p, ctrl);
             fail = 1;
           } else {
             const uint32_t cb = (o1 - o0) * 16u;
-            mbar_arrive_expect_tx(&ctrl->full[s], cb + xbytes);
-            bulk_g2s(cbuf(s), p.blob + static_cast<size_t>(o0) * 16, cb, &ctrl->full[s]);
-            tma_load_2d(xbuf(s), &tmX, kb * 64, 0, &ctrl->full[s]);
+            mbar_arrive_expect_tx(&ctrl->cfull[s], cb);
+            bulk_g2s(cbuf(s), p.blob + static_cast<size_t>(o0) * 16, cb, &ctrl->cfull[s]);
           }
         }
         if (__shfl_sync(0xffffffffu, fail, 0)) {
@@ -350,8 +366,8 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       if (!stop && !finish_ts()) stream_timeout(p, ctrl);
       if (stream_aborted(ctrl)) {
         // let copies this thread started land before the CTA may exit
-        for (int s = 0; s < S; ++s)
-          if (it > s) mbar_wait(&ctrl->full[(it - 1 - s) % S], ((it - 1 - s) / S) & 1);
+        for (int s = 0; s < SC; ++s)
+          if (it > s) mbar_wait(&ctrl->cfull[(it - 1 - s) % SC], ((it - 1 - s) / SC) & 1);
         if (bc_pending) mbar_wait(&ctrl->bcfull, (nad - 1) & 1);
         if (ts_next > 0) mbar_wait(&ctrl->tsfull, (ts_next - 1) & 1);
       }
@@ -373,6 +389,16 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         mma_commit(&ctrl->tsfree);
         if (++ts_done == nts) mma_commit(&ctrl->tsdone);
       };
+      // the t share's data arrives well before the first decoded block: multiply it first
+      // so that t is complete early
+      if (nts > 0) {
+        if (!mbar_wait(&ctrl->tsfull, 0)) {
+          stream_timeout(p, ctrl);
+          ok = false;
+        } else {
+          mma_ts();
+        }
+      }
       int it = 0, seg = 0, nad = 0;
       for (int u = u0; u < u1 && ok && !stream_aborted(ctrl); ++seg) {
         const int i = u / KB, kba = u % KB;
@@ -386,9 +412,9 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         tc_fence_after();
         const uint32_t acc = tmem + x * BNT;
         for (int kb = kba; kb < kbb; ++kb, ++it) {
-          const int s = it % S;
+          const int s = it % SA;
           if (ts_done < nts && mbar_try_wait(smem_u32(&ctrl->tsfull), ts_done & 1)) mma_ts();
-          if (!mbar_wait(&ctrl->dec[s], (it / S) & 1)) {
+          if (!mbar_wait(&ctrl->dec[s], (it / SA) & 1) || !mbar_wait(&ctrl->xfull[s], (it / SA) & 1)) {
             stream_timeout(p, ctrl);
             ok = false;
             break;
@@ -399,7 +425,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
           for (int k = 0; k < 4; ++k)
             mma_bf16_ss(acc, smem_desc_sw128(a0 + 32 * k, 16, 1024),
                         smem_desc_sw128(x0 + 32 * k, 16, 1024), idesc, (kb != kba) || k != 0);
-          mma_commit(&ctrl->empty[s]);
+          mma_commit(&ctrl->aempty[s]);
         }
         if (!ok) break;
         if (adapter && kba == 0) {
@@ -436,162 +462,187 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       mma_commit(&ctrl->fin);
       if (!mbar_wait(&ctrl->fin, 0)) stream_timeout(p, ctrl);
     }
-  } else if (warp < 6) {
-    // ================================================================ epilogue (warps 2-5)
-    const int q = warp & 3;
+  } else if (warp < kStreamFixedWarps) {
+    // ================================================================ epilogue
+    // Two groups of four warps (2-5 and 6-9); group x drains accumulator x, i.e. the
+    // CTA's segments of that parity, so that two segment epilogues can overlap.  Group 0
+    // also handles this CTA's part of the shared t.
+    const int eg = (warp - 2) >> 2;               // epilogue group
+    const int bar_id = 1 + eg;                    // named barrier of the group
+    const bool lead = threadIdx.x == 64 + 128 * eg;
+    const int q = warp & 3;                       // TMEM lane quarter
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     const int r = 32 * q + lane;  // weight row within the tile; rank index for t
     __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(p.Y);
-    bool ok = true;
-    // ---- 1. this CTA's share of t = X A_cat: drain t^T from TMEM into the fp32 buffer
-    if (nts > 0) {
-      ok = mbar_wait(&ctrl->tsdone, 0);
-      if (!ok) stream_timeout(p, ctrl);
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok) {
-        tc_fence_after();
-        for (int c = 0; c < BNT; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(tmem_ts + lane_base + c, v);
-          tmem_ld_wait();
-          if (r < p.R) {
+    volatile int* gflag = &ctrl->flag[eg];
+    bool t_read = false;
+    if (eg == 0) {
+      bool ok = true;
+      // ---- 1. this CTA's share of t = X A_cat: drain t^T from TMEM into the fp32 buffer
+      if (nts > 0) {
+        ok = mbar_wait(&ctrl->tsdone, 0);
+        if (!ok) stream_timeout(p, ctrl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          for (int c = 0; c < BNT; c += 16) {
+            uint32_t v[16];
+            tmem_ld16(tmem_ts + lane_base + c, v);
+            tmem_ld_wait();
+            if (r < p.R) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (c + e < p.M) atomicAdd(&p.tacc[(c + e) * p.R16 + r], __uint_as_float(v[e]));
+              for (int e = 0; e < 16; ++e)
+                if (c + e < p.M) atomicAdd(&p.tacc[(c + e) * p.R16 + r], __uint_as_float(v[e]));
+            }
           }
         }
       }
-    }
-    if (adapter) {
-      __threadfence();
-      named_bar(1, 128);
-      if (threadIdx.x == 64 && nts > 0) {
-        const uint32_t prev = atomicAdd(&p.tflags[0], 1u);
-        if (prev == static_cast<uint32_t>(p.tshare - 1)) {
+      if (adapter) {
+        named_bar(bar_id, 128);
+        if (lead && nts > 0) {
+          uint32_t prev;
+          asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                       : "=r"(prev)
+                       : "l"(p.tflags)
+                       : "memory");
+          if (prev == static_cast<uint32_t>(p.tshare - 1)) {
+            p.tflags[0] = 0u;
+            st_release(&p.tflags[1], 1u);
+          }
+        }
+      }
+      // ---- 2. if this CTA starts some row tile it applies the adapter: wait for the
+      //         complete t and round it to bf16 into shared memory
+      bool has_adapter_seg = false;
+      for (int u = u0; u < u1; u = (u / KB + 1) * KB)
+        if (u % KB == 0) has_adapter_seg = true;
+      if (adapter && has_adapter_seg) {
+        if (lead) *gflag = wait_global_flag(&p.tflags[1], 1u) ? 1 : 0;
+        named_bar(bar_id, 128);
+        if (*gflag == 0) {
+          if (lead) stream_timeout(p, ctrl);
+        } else {
           __threadfence();
-          p.tflags[0] = 0u;
-          st_release(&p.tflags[1], 1u);
+          for (int e = r; e < BNT * p.R16; e += 128) {
+            const int m = e / p.R16, j = e % p.R16;
+            float v = 0.0f;
+            if (m < p.M && j < p.R) v = __ldcg(&p.tacc[m * p.R16 + j]);
+            const int chunk = j >> 6, cc = j & 63;
+            uint8_t* dst = tbuf + chunk * (BNT * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
+                           (((cc >> 3) ^ (m & 7)) << 4) + (cc & 7) * 2;
+            *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
+          }
+          fence_proxy_async_smem();
+          t_read = true;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->tready);
       }
     }
-    // ---- 2. if this CTA owns the first block of some row tile, it applies the adapter:
-    //         wait for the complete t, round it to bf16 into shared memory
-    bool has_adapter_seg = false;
-    for (int u = u0; u < u1; u = (u / KB + 1) * KB)
-      if (u % KB == 0) has_adapter_seg = true;
-    bool t_read = false;
-    if (adapter && has_adapter_seg) {
-      if (threadIdx.x == 64) ctrl->flag = wait_global_flag(&p.tflags[1], 1u) ? 1 : 0;
-      named_bar(1, 128);
-      if (*reinterpret_cast<volatile int*>(&ctrl->flag) == 0) {
-        if (threadIdx.x == 64) stream_timeout(p, ctrl);
-      } else {
-        __threadfence();
-        for (int e = threadIdx.x - 64; e < BNT * p.R16; e += 128) {
-          const int m = e / p.R16, j = e % p.R16;
-          float v = 0.0f;
-          if (m < p.M && j < p.R) v = __ldcg(&p.tacc[m * p.R16 + j]);
-          const int chunk = j >> 6, cc = j & 63;
-          uint8_t* dst = tbuf + chunk * (BNT * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
-                         (((cc >> 3) ^ (m & 7)) << 4) + (cc & 7) * 2;
-          *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
-        }
-        fence_proxy_async_smem();
-        t_read = true;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->tready);
-    }
-    // ---- 3. per segment: drain the accumulator, write Y or a partial sum
+    // ---- 3. segments of this group's parity: drain the accumulator, then write Y or a
+    //         partial.  A partial goes to its own slot, numbered owner CTA + tile index
+    //         (unique under the even contiguous split), so no atomics are needed; the
+    //         last segment of the tile to arrive sums the slots into Y.
     int seg = 0;
     for (int u = u0; u < u1; ++seg) {
       const int i = u / KB, kba = u % KB;
       const int kbb = min(KB, kba + (u1 - u));
       const int x = seg & 1;
-      bool okw = mbar_wait(&ctrl->accfull[x], (seg >> 1) & 1);
-      if (!okw) stream_timeout(p, ctrl);
-      okw = __all_sync(0xffffffffu, okw) && !stream_aborted(ctrl);
-      named_bar(1, 128);
-      if (threadIdx.x == 64) ctrl->flag = okw ? 2 : 0;
-      named_bar(1, 128);
-      if (*reinterpret_cast<volatile int*>(&ctrl->flag) != 2) break;
-      tc_fence_after();
-      const size_t n = static_cast<size_t>(i) * 128 + r;
-      const bool whole = kba == 0 && kbb == KB;
-      float4* wrow = reinterpret_cast<float4*>(p.ws + n * BNT);  // partials, [N x BNT]
+      if (x == eg) {
+        bool okw = mbar_wait(&ctrl->accfull[x], (seg >> 1) & 1);
+        if (!okw) stream_timeout(p, ctrl);
+        okw = __all_sync(0xffffffffu, okw) && !stream_aborted(ctrl);
+        named_bar(bar_id, 128);
+        if (lead) *gflag = okw ? 2 : 0;
+        named_bar(bar_id, 128);
+        if (*gflag != 2) break;
+        tc_fence_after();
+        const size_t n = static_cast<size_t>(i) * 128 + r;
+        const bool whole = kba == 0 && kbb == KB;
+        float4* mine = reinterpret_cast<float4*>(p.ws) +
+                       (static_cast<size_t>(cta + i) * 128 + r) * (BNT / 4);
 #pragma unroll
-      for (int c = 0; c < BNT; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + x * BNT + lane_base + c, v);
-        tmem_ld_wait();
-        if (whole) {
+        for (int c = 0; c < BNT; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(tmem + x * BNT + lane_base + c, v);
+          tmem_ld_wait();
+          if (whole) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (c + e < p.M)
-              Y[(c + e) * static_cast<size_t>(p.N) + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
-        } else {
+            for (int e = 0; e < 16; ++e)
+              if (c + e < p.M)
+                Y[(c + e) * static_cast<size_t>(p.N) + n] =
+                    __float2bfloat16_rn(__uint_as_float(v[e]));
+          } else {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            if (c + 4 * q4 < p.M)
-              atomicAdd(&wrow[(c >> 2) + q4],
-                        make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
-                                    __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3])));
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->accempty[x]);
-      if (!whole) {
-        // publish this CTA's partial: barrier, then one release/acquire counter update
-        named_bar(1, 128);
-        if (threadIdx.x == 64) {
-          const int segs = owner_of(static_cast<long long>(i) * KB + KB - 1, U, G) -
-                           owner_of(static_cast<long long>(i) * KB, U, G) + 1;
-          uint32_t prev;
-          asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                       : "=r"(prev)
-                       : "l"(p.counters + i)
-                       : "memory");
-          ctrl->flag = prev == static_cast<uint32_t>(segs - 1) ? 3 : 2;
-        }
-        named_bar(1, 128);
-        if (*reinterpret_cast<volatile int*>(&ctrl->flag) == 3) {
-#pragma unroll
-          for (int c = 0; c < BNT; c += 4) {
-            if (c < p.M) {
-              const float4 t = __ldcg(&wrow[c >> 2]);
-              const float tv[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (c + e < p.M)
-                  Y[(c + e) * static_cast<size_t>(p.N) + n] = __float2bfloat16_rn(tv[e]);
-              __stcg(&wrow[c >> 2], make_float4(0.f, 0.f, 0.f, 0.f));
-            }
+            for (int q4 = 0; q4 < 4; ++q4)
+              if (c + 4 * q4 < p.M)
+                __stcg(&mine[(c >> 2) + q4],
+                       make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                   __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3])));
           }
-          if (threadIdx.x == 64) p.counters[i] = 0u;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->accempty[x]);
+        if (!whole) {
+          named_bar(bar_id, 128);
+          const int c_first = owner_of(static_cast<long long>(i) * KB, U, G);
+          const int segs = owner_of(static_cast<long long>(i) * KB + KB - 1, U, G) - c_first + 1;
+          if (lead) {
+            uint32_t prev;
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                         : "=r"(prev)
+                         : "l"(p.counters + i)
+                         : "memory");
+            *gflag = prev == static_cast<uint32_t>(segs - 1) ? 3 : 2;
+          }
+          named_bar(bar_id, 128);
+          if (*gflag == 3) {
+            const float4* slot0 = reinterpret_cast<const float4*>(p.ws) +
+                                  (static_cast<size_t>(c_first + i) * 128 + r) * (BNT / 4);
+#pragma unroll
+            for (int c = 0; c < BNT; c += 4) {
+              if (c < p.M) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int k = 0; k < segs; ++k) {
+                  const float4 t = __ldcg(slot0 + static_cast<size_t>(k) * 128 * (BNT / 4) + (c >> 2));
+                  acc.x += t.x;
+                  acc.y += t.y;
+                  acc.z += t.z;
+                  acc.w += t.w;
+                }
+                const float tv[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (c + e < p.M)
+                    Y[(c + e) * static_cast<size_t>(p.N) + n] = __float2bfloat16_rn(tv[e]);
+              }
+            }
+            if (lead) p.counters[i] = 0u;
+          }
         }
       }
       u = i * KB + kbb;
     }
     // ---- 4. every CTA checks in as a reader of t; the last one clears it for next call
-    if (adapter) {
-      named_bar(1, 128);
-      if (threadIdx.x == 64) {
+    if (eg == 0 && adapter) {
+      named_bar(bar_id, 128);
+      if (lead) {
         bool ready = t_read || wait_global_flag(&p.tflags[1], 1u);
         if (!ready) {
           stream_timeout(p, ctrl);
-          ctrl->flag = 0;
+          *gflag = 0;
         } else {
           const uint32_t prev = atomicAdd(&p.tflags[2], 1u);
-          ctrl->flag = prev == static_cast<uint32_t>(G - 1) ? 4 : 0;
+          *gflag = prev == static_cast<uint32_t>(G - 1) ? 4 : 0;
         }
       }
-      named_bar(1, 128);
-      if (*reinterpret_cast<volatile int*>(&ctrl->flag) == 4) {
-        for (int e = threadIdx.x - 64; e < BNT * p.R16; e += 128) p.tacc[e] = 0.0f;
+      named_bar(bar_id, 128);
+      if (*gflag == 4) {
+        for (int e = r; e < BNT * p.R16; e += 128) p.tacc[e] = 0.0f;
         __threadfence();
-        named_bar(1, 128);
-        if (threadIdx.x == 64) {
+        named_bar(bar_id, 128);
+        if (lead) {
           p.tflags[2] = 0u;
           st_release(&p.tflags[1], 0u);
         }
@@ -608,19 +659,21 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     constexpr int RPW = 128 / WPG;             // rows per warp
     const int dw = warp - kStreamFixedWarps;
     const int g = dw / WPG, wg = dw % WPG;
-    const uint32_t* lut = ctrl->lut;
+    const uint32_t* lut = lutp;
     const int nunits = u1 - u0;
+    const bool leader = wg == 0 && lane == 0;  // issues the group's X-tile copies
+    int last_x = -1;
     for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
-      const int s = it % S;
-      if (!mbar_wait(&ctrl->full[s], (it / S) & 1)) {
+      const int sc = it % SC, sa = it % SA;
+      if (!mbar_wait(&ctrl->cfull[sc], (it / SC) & 1)) {
         stream_timeout(p, ctrl);
         break;
       }
-      const uint8_t* cb = cbuf(s);
+      const uint8_t* cb = cbuf(sc);
       const uint64_t* bm = reinterpret_cast<const uint64_t*>(cb);
       const uint8_t* vals = cb + kBitmapBytes;
-      uint32_t* cs = csb(s);
-      uint8_t* ab = abuf(s);
+      uint32_t* cs = csb(g);
+      uint8_t* ab = abuf(sa);
       // ---- chunk offsets of this warp's rows
       uint32_t base = 0;
       for (int rr = lane; rr < RPW * wg; rr += 32) base += __popcll(bm[rr]);
@@ -656,6 +709,16 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         reinterpret_cast<uint4*>(cs)[2 * row + 1] = o1;
       }
       __syncwarp();
+      // ---- the decoded tile's ring entry must be free; the group leader fetches X
+      if (!mbar_wait(&ctrl->aempty[sa], ((it / SA) & 1) ^ 1)) {
+        stream_timeout(p, ctrl);
+        break;
+      }
+      if (leader) {
+        mbar_arrive_expect_tx(&ctrl->xfull[sa], BNT * 128);
+        tma_load_2d(xbuf(sa), &tmX, ((u0 + it) % KB) * 64, 0, &ctrl->xfull[sa]);
+        last_x = it;
+      }
       // ---- expansion: 4 rows x 8 chunks per step
 #pragma unroll 2
       for (int st = 0; st < RPW / 4; ++st) {
@@ -667,8 +730,13 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->dec[s]);
+      if (lane == 0) {
+        mbar_arrive(&ctrl->dec[sa]);
+        mbar_arrive(&ctrl->cempty[sc]);
+      }
     }
+    if (leader && last_x >= 0 && stream_aborted(ctrl))
+      mbar_wait(&ctrl->xfull[last_x % SA], (last_x / SA) & 1);  // own copy lands first
   }
 
   tc_fence_before();
