@@ -105,14 +105,20 @@ SALR_API int salr_decode(salr_handle h, void* W_out, void* stream);
  *
  * Arithmetic: products of bf16 inputs accumulate in fp32 on the tensor cores.  The
  * adapter's inner product t = X A_cat is accumulated in fp32 and rounded once to bf16
- * before it multiplies B_cat.  The order of the fp32 sums is not fixed (split K), so
- * results are not bitwise reproducible between calls with different M, but always
- * satisfy ||Y - Y*||_F <= 4e-3 ||Y*||_F and |Y - Y*| <= 1e-2 * sum|products| against the
+ * before it multiplies B_cat.  The order of the fp32 sums is not fixed (split K, and
+ * for M <= 64 partial sums of a row tile are added in L2 in arrival order), so results
+ * are not bitwise reproducible from call to call, but always satisfy ||Y - Y*||_F <= 4e-3 ||Y*||_F and |Y - Y*| <= 1e-2 * sum|products| against the
  * exact result Y*.
  *
  * The handle holds the split-K workspace used by this call; it is grown on demand
  * (a cudaMalloc) and is not safe to share between calls running concurrently on
  * different streams.
+ *
+ * For M <= 64 the call may start while the previous kernel on `stream` is still
+ * running (programmatic dependent launch): before that kernel has completed it reads
+ * only the handle's encoded weight; X, A_cat, B_cat, the scratch and Y are touched
+ * afterwards.  Whatever writes the encoded weight (salr_encode) must therefore have
+ * completed, or be ordered on the stream before the previous kernel.
  */
 SALR_API int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat,
                 const void* B_cat, int64_t R, void* Y, void* stream);
@@ -135,19 +141,22 @@ SALR_API int salr_linear_host(const void* X_host, int64_t M, salr_handle h, cons
  * No counterpart in the SALR paper: this is an interface variant of this library, not
  * part of the method.  It computes the same layer as salr_linear (same arguments, same
  * arithmetic and tolerance) for M <= 16 and N <= 32768, and never allocates device
- * memory: the scratch it needs (partial sums, arrival counters, the fp32 t = X A_cat
- * accumulator and its flags, about 3.3 MiB) is one fixed array in the library's device
- * code, present on every GPU that loads the library until the process exits.  Meant for
+ * memory: the scratch it needs (fp32 partial sums and their arrival counts, the two
+ * fp32 t = X A_cat accumulators and their counts, about 2 MiB) is one fixed array in the
+ * library's device code, present on every GPU that loads the library until the process
+ * exits.  Meant for
  * callers whose device memory is planned up front and who may not allocate during
  * inference (a failing or stalling cudaMalloc is not acceptable there).  The handle and
  * all inputs and outputs are still the caller's.
  *
- * Returns SALR_ERR_UNSUPPORTED for M > 16 or N > 32768 (or a GPU with more than 160 SMs).  The first call on a device
- * looks up the array's device address (cudaGetSymbolAddress) and should come before
- * any stream capture.  Every call first zeroes the counters and accumulators it reads
- * (the partial-sum slots are always written before they are read).  All calls on one device share the one array, so calls
- * whose executions overlap on the GPU (different streams, or different threads) race
- * and give wrong results: order them on one stream.
+ * Returns SALR_ERR_UNSUPPORTED for M > 16 or N > 32768 (or a GPU with more than 160
+ * SMs).  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress), clears the array on `stream` and should come before any
+ * stream capture.  Each call then leaves the array ready for the next one; after a call
+ * that gave up (salr_sync_status reports it) the array is cleared again.  All calls
+ * on one device share the one array, so calls whose executions overlap on the GPU
+ * (different streams, or different threads) race and give wrong results: order them on
+ * one stream.
  */
 SALR_API int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, const void* A_cat,
                                  const void* B_cat, int64_t R, void* Y, void* stream);

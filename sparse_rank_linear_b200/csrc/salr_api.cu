@@ -29,16 +29,18 @@ struct Workspace {
   size_t n_counters = 0;
 };
 
-// Scratch of the persistent small-M kernel: partial-sum slots ((SMs + N/128) x 128 x 64
-// fp32, overwritten by every call), per-row-tile arrival counters, the fp32 t = X A_cat
-// accumulator [64 x 128] and its three flags (these three are left zeroed by every
-// successful call).
+// Scratch of the persistent small-M kernel: fp32 sums of split row tiles [N x 64] and
+// their arrival counts [N/128] (left zeroed by every call), and two fp32 t = X A_cat
+// accumulators [64 x 128] with their arrival counts, used by alternate calls; each call
+// clears the buffer the next call will use.  `epoch` counts the calls.
 struct StreamScratch {
-  float* ws = nullptr;
+  float* acc = nullptr;
   uint32_t* counters = nullptr;
-  float* tacc = nullptr;
-  uint32_t* tflags = nullptr;
+  float* tacc = nullptr;       // 2 x kTBuf floats
+  uint32_t* tflags = nullptr;  // 2 counts
+  uint32_t epoch = 0;
 };
+constexpr int kTBuf = 64 * 128;
 
 }  // namespace
 
@@ -135,7 +137,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
 }
 
 void release(salr_weight_s* h) {
-  cudaFree(h->sscr.ws);
+  cudaFree(h->sscr.acc);
   cudaFree(h->sscr.counters);
   cudaFree(h->sscr.tacc);
   cudaFree(h->sscr.tflags);
@@ -220,38 +222,54 @@ int launch_linear(const LinParams& p, const CUtensorMap& tx, const CUtensorMap& 
 }
 
 
-// Persistent small-M path: one CTA per SM (cooperative launch: the adapter's t is
-// shared through global memory, so every CTA must be resident).
+// Persistent small-M path: one CTA per SM, launched so that it may overlap the preceding
+// kernel of the stream.
 constexpr int kStreamDecoders = 16;
 
-size_t stream_slot_bytes(const salr_weight_s* h) {
-  return static_cast<size_t>(device_sms(h->device) + h->N / 128) * 128 * 64 * sizeof(float);
-}
-
 int ensure_stream_scratch(salr_weight_s* h, cudaStream_t st) {
-  if (h->sscr.ws) return SALR_OK;
+  if (h->sscr.acc) return SALR_OK;
   void *a = nullptr, *b = nullptr, *c = nullptr, *d = nullptr;
-  const size_t wsb = stream_slot_bytes(h);
+  const size_t ab = static_cast<size_t>(h->N) * 64 * sizeof(float);
   const size_t cb = static_cast<size_t>(h->N / 128) * sizeof(uint32_t);
-  const size_t tb = 64 * 128 * sizeof(float);
+  const size_t tb = 2 * kTBuf * sizeof(float);
   cudaError_t e;
-  if ((e = dev_alloc(&a, wsb)) != cudaSuccess || (e = dev_alloc(&b, cb)) != cudaSuccess ||
-      (e = dev_alloc(&c, tb)) != cudaSuccess || (e = dev_alloc(&d, 4 * sizeof(uint32_t))) != cudaSuccess) {
+  if ((e = dev_alloc(&a, ab)) != cudaSuccess || (e = dev_alloc(&b, cb)) != cudaSuccess ||
+      (e = dev_alloc(&c, tb)) != cudaSuccess || (e = dev_alloc(&d, 2 * sizeof(uint32_t))) != cudaSuccess) {
     cudaFree(a);
     cudaFree(b);
     cudaFree(c);
     cudaFree(d);
     return cuda_status(e);
   }
-  h->sscr.ws = static_cast<float*>(a);
+  h->sscr.acc = static_cast<float*>(a);
   h->sscr.counters = static_cast<uint32_t*>(b);
   h->sscr.tacc = static_cast<float*>(c);
   h->sscr.tflags = static_cast<uint32_t*>(d);
-  SALR_TRY(cudaMemsetAsync(a, 0, wsb, st));
+  h->sscr.epoch = 0;
+  SALR_TRY(cudaMemsetAsync(a, 0, ab, st));
   SALR_TRY(cudaMemsetAsync(b, 0, cb, st));
   SALR_TRY(cudaMemsetAsync(c, 0, tb, st));
-  SALR_TRY(cudaMemsetAsync(d, 0, 4 * sizeof(uint32_t), st));
+  SALR_TRY(cudaMemsetAsync(d, 0, 2 * sizeof(uint32_t), st));
   return SALR_OK;
+}
+
+// Point the kernel at its scratch: this call's t buffer (by the parity of the call count
+// that follows `last`) and the other one, which the call clears for the next.  The caller
+// records the new count only once the launch has succeeded, so that a call that never
+// ran does not flip the parity.
+uint32_t bind_call(StreamParams& sp, float* acc, uint32_t* counters, float* tacc, uint32_t* tflags,
+                   int tbuf, uint32_t last) {
+  const uint32_t epoch = last + 1;
+  const int b = static_cast<int>(epoch & 1u);
+  sp.acc = acc;
+  sp.counters = counters;
+  sp.tacc = tacc + b * tbuf;
+  sp.tacc_next = tacc + (1 - b) * tbuf;
+  sp.tflag = tflags + b;
+  sp.tflag_next = tflags + (1 - b);
+  sp.tzero = tbuf;
+  sp.epoch = epoch;
+  return epoch;
 }
 
 template <int BNT, bool SEL_LUT>
@@ -286,17 +304,23 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  // One CTA per SM (the shared-memory footprint admits no second one) and the t-share
-  // work sits in the lowest-numbered CTAs, which wait on nothing before finishing it; so
-  // the only cross-CTA wait (for the complete t) cannot block those CTAs.  A cooperative
-  // launch would guarantee co-residency outright but costs several microseconds per
-  // call; SALR_COOPERATIVE=1 requests it.
+  // One CTA per SM (the shared-memory footprint admits no second one); cross-CTA waits
+  // go to lower-indexed CTAs or to the t-share CTAs, which wait on nothing before
+  // finishing their share.  The launch may overlap the preceding kernel of the stream
+  // (programmatic stream serialization): the kernel waits for it before touching
+  // anything but the weight blob.  SALR_COOPERATIVE=1 asks for a cooperative launch
+  // instead, which guarantees co-residency outright.
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
   const char* coop = getenv("SALR_COOPERATIVE");
+  if (coop && coop[0] == '1') {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = (coop && coop[0] == '1') ? 1 : 0;
+  cfg.numAttrs = 1;
   SALR_TRY(cudaLaunchKernelEx(&cfg, salr_stream_kernel<BNT, kStreamDecoders, SEL_LUT>, p, tx, ta,
                               tb));
   return SALR_OK;
@@ -316,6 +340,8 @@ int check_linear_args(const void* X, int64_t M, salr_handle h, const void* A, co
 }
 
 }  // namespace
+
+int noalloc_reset(int dev);  // defined with salr_linear_noalloc below
 
 extern "C" {
 
@@ -446,10 +472,8 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     sp.blob = h->blob;
     sp.offsets = h->offsets;
     sp.Y = static_cast<uint16_t*>(Y);
-    sp.ws = h->sscr.ws;
-    sp.counters = h->sscr.counters;
-    sp.tacc = h->sscr.tacc;
-    sp.tflags = h->sscr.tflags;
+    const uint32_t epoch = bind_call(sp, h->sscr.acc, h->sscr.counters, h->sscr.tacc,
+                                     h->sscr.tflags, kTBuf, h->sscr.epoch);
     sp.status = h->status;
     sp.N = static_cast<int>(h->N);
     sp.K = static_cast<int>(h->K);
@@ -474,13 +498,20 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     const char* lutv = getenv("SALR_DECODE_LUT");
     const bool use_lut = lutv && lutv[0] == '1';
     switch (bnt) {
-      case 16: return use_lut ? launch_stream<16, true>(sp, tx, ta, tb, sms, st)
-                              : launch_stream<16, false>(sp, tx, ta, tb, sms, st);
-      case 32: return use_lut ? launch_stream<32, true>(sp, tx, ta, tb, sms, st)
-                              : launch_stream<32, false>(sp, tx, ta, tb, sms, st);
-      default: return use_lut ? launch_stream<64, true>(sp, tx, ta, tb, sms, st)
-                              : launch_stream<64, false>(sp, tx, ta, tb, sms, st);
+      case 16:
+        rc = use_lut ? launch_stream<16, true>(sp, tx, ta, tb, sms, st)
+                     : launch_stream<16, false>(sp, tx, ta, tb, sms, st);
+        break;
+      case 32:
+        rc = use_lut ? launch_stream<32, true>(sp, tx, ta, tb, sms, st)
+                     : launch_stream<32, false>(sp, tx, ta, tb, sms, st);
+        break;
+      default:
+        rc = use_lut ? launch_stream<64, true>(sp, tx, ta, tb, sms, st)
+                     : launch_stream<64, false>(sp, tx, ta, tb, sms, st);
     }
+    if (rc == SALR_OK) h->sscr.epoch = epoch;
+    return rc;
   }
   const Schedule sc = choose_schedule(M, h->N, h->K, device_sms(h->device));
   LinParams p{};
@@ -590,11 +621,14 @@ int salr_sync_status(salr_handle h, void* stream) {
   if (h->work.ws) SALR_TRY(cudaMemset(h->work.ws, 0, h->work.ws_elems * sizeof(float)));
   if (h->work.counters)
     SALR_TRY(cudaMemset(h->work.counters, 0, h->work.n_counters * sizeof(uint32_t)));
-  if (h->sscr.ws) {
+  if (h->sscr.acc) {
+    SALR_TRY(cudaMemset(h->sscr.acc, 0, static_cast<size_t>(h->N) * 64 * sizeof(float)));
     SALR_TRY(cudaMemset(h->sscr.counters, 0, static_cast<size_t>(h->N / 128) * sizeof(uint32_t)));
-    SALR_TRY(cudaMemset(h->sscr.tacc, 0, 64 * 128 * sizeof(float)));
-    SALR_TRY(cudaMemset(h->sscr.tflags, 0, 4 * sizeof(uint32_t)));
+    SALR_TRY(cudaMemset(h->sscr.tacc, 0, 2 * kTBuf * sizeof(float)));
+    SALR_TRY(cudaMemset(h->sscr.tflags, 0, 2 * sizeof(uint32_t)));
   }
+  const int nrc = noalloc_reset(h->device);
+  if (nrc != SALR_OK) return nrc;
   if (status & DEV_ERR_TIMEOUT) return SALR_ERR_TIMEOUT;
   if (status & DEV_ERR_NAN) return SALR_ERR_INVALID;
   return SALR_ERR_UNSUPPORTED;
@@ -617,33 +651,60 @@ namespace {
 constexpr int64_t kNoAllocMaxM = 16;     // tokens per call
 constexpr int64_t kNoAllocMaxN = 32768;  // output features
 constexpr int kNoAllocMaxSMs = 160;      // CTAs of the persistent kernel
-// layout: [counters: N/128 u32][t flags: 4 u32][t accumulator: 16 x 128 f32]
-//         [partial slots: (SMs + N/128) x 128 x 16 f32]
-constexpr size_t kNaCounters = 0;
-constexpr size_t kNaFlags = kNaCounters + (kNoAllocMaxN / 128) * sizeof(uint32_t);
-constexpr size_t kNaTacc = kNaFlags + 256;
-constexpr size_t kNaWs = kNaTacc + 16 * 128 * sizeof(float);
-constexpr size_t kNaBytes =
-    kNaWs + static_cast<size_t>(kNoAllocMaxSMs + kNoAllocMaxN / 128) * 128 * 16 * sizeof(float);
+// layout: [t counts: 2 u32][t accumulators: 2 x 16 x 128 f32]
+//         [split-tile arrival counts: N/128 u32][split-tile sums: N x 16 f32]
+constexpr int kNaTBuf = 16 * 128;
+constexpr size_t kNaFlags = 0;
+constexpr size_t kNaTacc = 256;
+constexpr size_t kNaCounters = kNaTacc + 2 * kNaTBuf * sizeof(float);
+constexpr size_t kNaAcc = kNaCounters + (kNoAllocMaxN / 128) * sizeof(uint32_t);
+constexpr size_t kNaBytes = kNaAcc + static_cast<size_t>(kNoAllocMaxN) * 16 * sizeof(float);
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
 
 std::mutex g_na_mu;
 unsigned char* g_na_ptr[64] = {nullptr};
+uint32_t g_na_epoch[64] = {0};
 
-// Device address of the scratch array for the current device (looked up once per device).
-int noalloc_scratch(int dev, unsigned char** out) {
+// Device address of the scratch array for the current device (looked up, and cleared on
+// the caller's stream, once per device) and the tag of this call.
+int noalloc_scratch(int dev, cudaStream_t st, unsigned char** out, uint32_t* epoch) {
   if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> g(g_na_mu);
   if (!g_na_ptr[dev]) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) return SALR_ERR_CUDA;
+    SALR_TRY(cudaMemsetAsync(p, 0, kNaBytes, st));
     g_na_ptr[dev] = static_cast<unsigned char*>(p);
   }
   *out = g_na_ptr[dev];
+  *epoch = g_na_epoch[dev];
   return SALR_OK;
 }
+
+void noalloc_commit_epoch(int dev, uint32_t epoch) {
+  std::lock_guard<std::mutex> g(g_na_mu);
+  g_na_epoch[dev] = epoch;
+}
+
+}  // namespace
+
+// After a call that gave up, clear the shared array of the device (if it is in use) so
+// that the next call starts clean.
+int noalloc_reset(int dev) {
+  if (dev < 0 || dev >= 64) return SALR_OK;
+  std::lock_guard<std::mutex> g(g_na_mu);
+  if (!g_na_ptr[dev]) return SALR_OK;
+  int cur = 0;
+  SALR_TRY(cudaGetDevice(&cur));
+  if (cur != dev) SALR_TRY(cudaSetDevice(dev));
+  const cudaError_t e = cudaMemset(g_na_ptr[dev], 0, kNaBytes);
+  if (cur != dev) cudaSetDevice(cur);
+  return cuda_status(e);
+}
+
+namespace {
 
 }  // namespace
 
@@ -657,20 +718,18 @@ extern "C" int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, cons
   SALR_TRY(cudaGetDevice(&dev));
   if (dev != h->device) return SALR_ERR_INVALID;
   unsigned char* scr = nullptr;
-  rc = noalloc_scratch(dev, &scr);
-  if (rc != SALR_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // zero what must start at zero: arrival counters, t flags and the t accumulator (the
-  // partial-sum slots are always written before they are read)
-  SALR_TRY(cudaMemsetAsync(scr, 0, kNaWs, st));
+  uint32_t epoch = 0;
+  rc = noalloc_scratch(dev, st, &scr, &epoch);
+  if (rc != SALR_OK) return rc;
   StreamParams sp{};
   sp.blob = h->blob;
   sp.offsets = h->offsets;
   sp.Y = static_cast<uint16_t*>(Y);
-  sp.ws = reinterpret_cast<float*>(scr + kNaWs);
-  sp.counters = reinterpret_cast<uint32_t*>(scr + kNaCounters);
-  sp.tacc = reinterpret_cast<float*>(scr + kNaTacc);
-  sp.tflags = reinterpret_cast<uint32_t*>(scr + kNaFlags);
+  epoch = bind_call(sp, reinterpret_cast<float*>(scr + kNaAcc),
+                    reinterpret_cast<uint32_t*>(scr + kNaCounters),
+                    reinterpret_cast<float*>(scr + kNaTacc),
+                    reinterpret_cast<uint32_t*>(scr + kNaFlags), kNaTBuf, epoch);
   sp.status = h->status;
   sp.N = static_cast<int>(h->N);
   sp.K = static_cast<int>(h->K);
@@ -689,5 +748,7 @@ extern "C" int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, cons
     if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
     if (!make_map(&tb, B_cat, h->N, R, 64, sp.R16)) return SALR_ERR_CUDA;
   }
-  return launch_stream<16, false>(sp, tx, ta, tb, device_sms(h->device), st);
+  rc = launch_stream<16, false>(sp, tx, ta, tb, device_sms(h->device), st);
+  if (rc == SALR_OK) noalloc_commit_epoch(dev, epoch);
+  return rc;
 }

@@ -5,9 +5,11 @@
 //
 // * Work split: the weight's 128 x 64 blocks, in storage order, are cut into one
 //   contiguous range per CTA (one CTA per SM, every SM the same number of blocks).  A
-//   range covers one or more row-tile segments; a segment that does not cover a whole
-//   row tile stores its fp32 partial in a slot of its own, and the last segment of the
-//   tile to arrive (an arrival counter, no waiting) sums the slots into the bf16 output.
+//   range covers one or more row-tile segments.  A segment that does not cover a whole
+//   row tile adds its fp32 partial into the tile's fp32 accumulator with vector
+//   reductions performed in L2, fences, and counts itself in; the last segment of the
+//   tile to arrive (no waiting) reads the sum, writes the bf16 output and clears the
+//   accumulator and its count for the next call.
 // * Stage 1 decode (SALR technical summary, Methodology 4): decoder warps work in
 //   groups, each group on a different block so that several blocks are in flight.  A
 //   warp first turns the bitmap words of its 32 rows into the offset of every (row,
@@ -17,11 +19,18 @@
 //   16-entry nibble lookup table.
 // * Stage 2: tcgen05 bf16 MMAs into a double-buffered TMEM accumulator, pipelined
 //   against the decode through shared-memory stages filled by TMA.
-// * Concatenated adapter (Methodology 3): t = X A_cat is computed once per call.  Each
-//   CTA multiplies a share of the K dimension on the tensor cores and adds its part into
-//   an fp32 buffer; when all parts have arrived every row tile reads t back, rounds it to
-//   bf16 once and adds B_cat^T t^T to its accumulator with one more MMA.  This needs all
-//   CTAs resident at once, which the host guarantees with a cooperative launch.
+// * Concatenated adapter (Methodology 3): t = X A_cat is computed once per call.  The
+//   lowest CTAs multiply a share of the K dimension each on the tensor cores and add
+//   their parts into an fp32 buffer; when all parts have arrived every row tile reads t
+//   back, rounds it to bf16 once and adds B_cat^T t^T to its accumulator with one more
+//   MMA.  The buffer is double-buffered by call parity: each call clears the other one
+//   for the next call, so nothing waits at the end of a call.
+// * Consecutive calls overlap (programmatic dependent launch): a CTA fetches its first
+//   compact blocks before waiting for the previous kernel of the stream, and touches X,
+//   the adapters, the scratch and Y only after that wait.
+//
+// The only cross-CTA wait is for t, on the t-share CTAs, which finish their share without
+// waiting on anything.  Every wait is bounded.
 //
 // Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-9 epilogue in two groups
 // (group 0 also the adapter's t share), 10.. decoders.
@@ -43,10 +52,14 @@ struct StreamParams {
   const uint8_t* blob;
   const uint32_t* offsets;
   uint16_t* Y;
-  float* ws;           // fp32 partials of split row tiles: (grid + RT) slots of [128 x BNT]
-  uint32_t* counters;  // [RT] arrivals per row tile, zero between calls
-  float* tacc;         // [BNT x R16] fp32 accumulator of t = X A_cat, zero between calls
-  uint32_t* tflags;    // [0] t parts arrived, [1] t complete, [2] t readers done
+  float* acc;            // [RT x 128 x BNT] fp32 sums of split row tiles, zero between calls
+  uint32_t* counters;    // [RT] segments of each split tile arrived, zero between calls
+  float* tacc;           // [BNT x R16] fp32 accumulator of t = X A_cat (this call's buffer)
+  float* tacc_next;      // the other buffer, cleared by this call for the next one
+  uint32_t* tflag;       // t parts arrived in this call's buffer
+  uint32_t* tflag_next;  // the other buffer's count, cleared by this call
+  int tzero;             // floats per t buffer
+  uint32_t epoch;        // call count; its parity picks the t buffer
   int* status;
   int N, K, M, R, R16;
   int kblocks;  // K / 64
@@ -145,25 +158,44 @@ __device__ __forceinline__ uint32_t funnel16(uint32_t lo, uint32_t hi, uint32_t 
   return __funnelshift_r(lo, hi, sh);
 }
 
-// Expand one bitmap byte `b` whose values start at halfword p of the block's value
-// array (shared memory, 16-byte aligned, readable 24 bytes past its end).  The window
-// is 8 values from the 8-byte boundary at or below p, plus 4 more only for lanes whose
-// high nibble reaches past them.  SEL_LUT picks the byte-permute selectors from the
-// nibble table in shared memory, otherwise they are built in registers:
+// Expansion of one bitmap byte `b` whose values start at halfword p of the block's value
+// array (shared memory, 16-byte aligned, readable 24 bytes past its end), in two parts so
+// that a decoder can issue the shared-memory loads of several bytes before any of their
+// arithmetic.  The window is the 12 values from the 8-byte boundary at or below p: the
+// low nibble's values start at halfword o = p mod 4 of it and the high nibble's at
+// x = o + popc(low nibble) <= 7.  Window bytes that lie past the block's values only ever
+// meet columns whose mask bit is clear, which the byte permutes zero.  SEL_LUT takes the
+// byte-permute selectors from the nibble table in shared memory, otherwise they are built
+// in registers:
 //   PAT(v), v the 2-bit mask of two columns, is 0x4444 / 0x4410 / 0x1044 / 0x3210 (both
 //   zero, first value low, first value high, both values), looked up for all four
 //   column pairs at once by one byte permute of a constant table;
 //   PAIR(s) = 0x3210 + 0x2222 s brings values s, s+1 of a window to the bottom.
 template <bool SEL_LUT>
-__device__ __forceinline__ uint4 expand_byte(const uint8_t* vals, uint32_t p, uint32_t b,
-                                             const uint32_t* lut) {
+struct ExpandIn {
+  uint2 a0, a1, a2;  // the window
+  uint4 sel;         // nibble-table entry (SEL_LUT only)
+};
+
+template <bool SEL_LUT>
+__device__ __forceinline__ ExpandIn<SEL_LUT> expand_load(const uint8_t* vals, uint32_t p,
+                                                         uint32_t b, const uint32_t* lut) {
+  ExpandIn<SEL_LUT> in;
   const uint8_t* wp = vals + ((p & ~3u) << 1);
-  const uint2 a0 = lds64(wp), a1 = lds64(wp + 8);
+  in.a0 = lds64(wp);
+  in.a1 = lds64(wp + 8);
+  in.a2 = lds64(wp + 16);
+  if constexpr (SEL_LUT) in.sel = reinterpret_cast<const uint4*>(lut)[b];
+  return in;
+}
+
+template <bool SEL_LUT>
+__device__ __forceinline__ uint4 expand_compute(const ExpandIn<SEL_LUT>& in, uint32_t p,
+                                                uint32_t b) {
+  const uint32_t W0 = in.a0.x, W1 = in.a0.y, W2 = in.a1.x, W3 = in.a1.y, W4 = in.a2.x,
+                 W5 = in.a2.y;
   const uint32_t o = p & 3u;
   const uint32_t x = o + __popc(b & 15u);  // first value of the high nibble
-  uint2 a2 = make_uint2(0u, 0u);
-  if (x >= 5u) a2 = lds64(wp + 16);
-  const uint32_t W0 = a0.x, W1 = a0.y, W2 = a1.x, W3 = a1.y, W4 = a2.x, W5 = a2.y;
   // low nibble: window at halfword o
   const bool o2 = (o & 2u) != 0;
   const uint32_t sh0 = (o & 1u) << 4;
@@ -177,11 +209,10 @@ __device__ __forceinline__ uint4 expand_byte(const uint8_t* vals, uint32_t p, ui
   const uint32_t H0 = funnel16(V0, V1, sh1), H1 = funnel16(V1, V2, sh1);
   uint32_t pat01, pat23, pr0, pr1;
   if constexpr (SEL_LUT) {
-    const uint4 e = reinterpret_cast<const uint4*>(lut)[b];
-    pat01 = e.x;
-    pat23 = e.y;
-    pr0 = e.z;
-    pr1 = e.z >> 16;
+    pat01 = in.sel.x;
+    pat23 = in.sel.y;
+    pr0 = in.sel.z;
+    pr1 = in.sel.z >> 16;
   } else {
     const uint32_t bs = (b & 3u) | ((b & 0xCu) << 6) | ((b & 0x30u) << 12) | ((b & 0xC0u) << 18);
     const uint32_t idx = bs * 0x22u + 0x10101010u;
@@ -220,6 +251,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
   StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(bcbuf + p.bcbuf);
   uint32_t* lutp = reinterpret_cast<uint32_t*>(bcbuf + p.bcbuf + 1024);  // 256 x 16 B
 
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool adapter = p.R > 0;
   const int G = gridDim.x, cta = blockIdx.x;
@@ -286,6 +318,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     // been consumed and the B_cat tile of a segment only after its last block.
     const uint32_t xbytes = BNT * 128;
     int ts_next = 0;  // next t-share round to issue (lane 0)
+    bool dep = false;  // lane 0 has waited for the preceding kernel
     auto issue_ts = [&](int r) {
       const int kb = cta + r * p.tshare;
       mbar_arrive_expect_tx(&ctrl->tsfull, (p.R > 64 ? 16384u : 8192u) + xbytes);
@@ -294,6 +327,15 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       tma_load_2d(bcbuf + 16384, &tmX, kb * 64, 0, &ctrl->tsfull);
     };
     // blocking: issue every remaining round, then wait until the last one is consumed
+    // X, the adapters and everything after are touched only after the preceding kernel
+    // of the stream has completed; the compact blocks before that need no wait
+    auto dep_wait = [&]() {
+      if (!dep) {
+        griddep_wait();
+        dep = true;
+        if (nts > 0) issue_ts(ts_next++);
+      }
+    };
     auto finish_ts = [&]() -> bool {
       while (ts_next < nts) {
         if (!mbar_wait(&ctrl->tsfree, (ts_next - 1) & 1)) return false;
@@ -307,7 +349,6 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
       }
-      if (nts > 0) issue_ts(ts_next++);
     }
     int it = 0, nad = 0, obase = u0;
     bool stop = false, bc_pending = false;
@@ -327,7 +368,8 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         const uint32_t o1 = (k + 1 < 32) ? o1n : offx;
         int fail = 0;
         if (lane == 0) {
-          if (ts_next < nts && mbar_try_wait(smem_u32(&ctrl->tsfree), (ts_next - 1) & 1))
+          if (it >= SC) dep_wait();
+          if (ts_next < nts && ts_next > 0 && mbar_test_wait(smem_u32(&ctrl->tsfree), (ts_next - 1) & 1))
             issue_ts(ts_next++);
           const int s = it % SC;
           if (!mbar_wait(&ctrl->cempty[s], ((it / SC) & 1) ^ 1) || stream_aborted(ctrl)) {
@@ -337,6 +379,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
             const uint32_t cb = (o1 - o0) * 16u;
             mbar_arrive_expect_tx(&ctrl->cfull[s], cb);
             bulk_g2s(cbuf(s), p.blob + static_cast<size_t>(o0) * 16, cb, &ctrl->cfull[s]);
+            if (it == SC - 1) dep_wait();
           }
         }
         if (__shfl_sync(0xffffffffu, fail, 0)) {
@@ -347,6 +390,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       if (!stop && adapter && kba == 0) {
         int fail = 0;
         if (lane == 0) {
+          dep_wait();
           if (!finish_ts() || !mbar_wait(&ctrl->bcempty, (nad & 1) ^ 1)) {
             stream_timeout(p, ctrl);
             fail = 1;
@@ -363,6 +407,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       u = i * KB + kbb;
     }
     if (lane == 0) {
+      dep_wait();
       if (!stop && !finish_ts()) stream_timeout(p, ctrl);
       if (stream_aborted(ctrl)) {
         // let copies this thread started land before the CTA may exit
@@ -413,7 +458,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         const uint32_t acc = tmem + x * BNT;
         for (int kb = kba; kb < kbb; ++kb, ++it) {
           const int s = it % SA;
-          if (ts_done < nts && mbar_try_wait(smem_u32(&ctrl->tsfull), ts_done & 1)) mma_ts();
+          if (ts_done < nts && mbar_test_wait(smem_u32(&ctrl->tsfull), ts_done & 1)) mma_ts();
           if (!mbar_wait(&ctrl->dec[s], (it / SA) & 1) || !mbar_wait(&ctrl->xfull[s], (it / SA) & 1)) {
             stream_timeout(p, ctrl);
             ok = false;
@@ -475,7 +520,13 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     const int r = 32 * q + lane;  // weight row within the tile; rank index for t
     __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(p.Y);
     volatile int* gflag = &ctrl->flag[eg];
-    bool t_read = false;
+    griddep_wait();
+    if (eg == 1 && cta == G - 1) {
+      // ---- 0. clear the other t buffer and its arrival count for the next call
+      float4* z = reinterpret_cast<float4*>(p.tacc_next);
+      for (int e = r; e < p.tzero / 4; e += 128) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (lead) *p.tflag_next = 0u;
+    }
     if (eg == 0) {
       bool ok = true;
       // ---- 1. this CTA's share of t = X A_cat: drain t^T from TMEM into the fp32 buffer
@@ -496,33 +547,24 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
             }
           }
         }
-      }
-      if (adapter) {
+        // publish: the group's adds happen before the arrival (release, cumulative over
+        // the barrier)
         named_bar(bar_id, 128);
-        if (lead && nts > 0) {
-          uint32_t prev;
-          asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                       : "=r"(prev)
-                       : "l"(p.tflags)
-                       : "memory");
-          if (prev == static_cast<uint32_t>(p.tshare - 1)) {
-            p.tflags[0] = 0u;
-            st_release(&p.tflags[1], 1u);
-          }
+        if (lead) {
+          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.tflag) : "memory");
         }
       }
-      // ---- 2. if this CTA starts some row tile it applies the adapter: wait for the
-      //         complete t and round it to bf16 into shared memory
+      // ---- 2. if this CTA starts some row tile it applies the adapter: wait for every
+      //         share of t and round it to bf16 into shared memory
       bool has_adapter_seg = false;
       for (int u = u0; u < u1; u = (u / KB + 1) * KB)
         if (u % KB == 0) has_adapter_seg = true;
       if (adapter && has_adapter_seg) {
-        if (lead) *gflag = wait_global_flag(&p.tflags[1], 1u) ? 1 : 0;
+        if (lead) *gflag = wait_global_flag(p.tflag, static_cast<uint32_t>(p.tshare)) ? 1 : 0;
         named_bar(bar_id, 128);
         if (*gflag == 0) {
           if (lead) stream_timeout(p, ctrl);
         } else {
-          __threadfence();
           for (int e = r; e < BNT * p.R16; e += 128) {
             const int m = e / p.R16, j = e % p.R16;
             float v = 0.0f;
@@ -533,16 +575,14 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
             *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
           }
           fence_proxy_async_smem();
-          t_read = true;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->tready);
       }
     }
-    // ---- 3. segments of this group's parity: drain the accumulator, then write Y or a
-    //         partial.  A partial goes to its own slot, numbered owner CTA + tile index
-    //         (unique under the even contiguous split), so no atomics are needed; the
-    //         last segment of the tile to arrive sums the slots into Y.
+    // ---- 3. segments of this group's parity: drain the accumulator, then write Y or, for
+    //         a split tile, add the partial into the tile's fp32 sum in L2; the last of
+    //         the tile's segments to count itself in writes Y and clears the sum
     int seg = 0;
     for (int u = u0; u < u1; ++seg) {
       const int i = u / KB, kba = u % KB;
@@ -559,8 +599,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         tc_fence_after();
         const size_t n = static_cast<size_t>(i) * 128 + r;
         const bool whole = kba == 0 && kbb == KB;
-        float4* mine = reinterpret_cast<float4*>(p.ws) +
-                       (static_cast<size_t>(cta + i) * 128 + r) * (BNT / 4);
+        float* sum = p.acc + n * BNT;
 #pragma unroll
         for (int c = 0; c < BNT; c += 16) {
           uint32_t v[16];
@@ -574,48 +613,49 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
                     __float2bfloat16_rn(__uint_as_float(v[e]));
           } else {
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-              if (c + 4 * q4 < p.M)
-                __stcg(&mine[(c >> 2) + q4],
-                       make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
-                                   __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3])));
+            for (int e = 0; e < 16; e += 4)
+              if (c + e < p.M)
+                red_add_v4f32(sum + c + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                              __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->accempty[x]);
         if (!whole) {
+          // every thread's additions are performed before the tile's count moves
+          __threadfence();
           named_bar(bar_id, 128);
-          const int c_first = owner_of(static_cast<long long>(i) * KB, U, G);
-          const int segs = owner_of(static_cast<long long>(i) * KB + KB - 1, U, G) - c_first + 1;
           if (lead) {
-            uint32_t prev;
-            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                         : "=r"(prev)
-                         : "l"(p.counters + i)
-                         : "memory");
+            const int c_first = owner_of(static_cast<long long>(i) * KB, U, G);
+            const int segs =
+                owner_of(static_cast<long long>(i) * KB + KB - 1, U, G) - c_first + 1;
+            const uint32_t prev = atomicAdd(p.counters + i, 1u);
             *gflag = prev == static_cast<uint32_t>(segs - 1) ? 3 : 2;
           }
           named_bar(bar_id, 128);
           if (*gflag == 3) {
-            const float4* slot0 = reinterpret_cast<const float4*>(p.ws) +
-                                  (static_cast<size_t>(c_first + i) * 128 + r) * (BNT / 4);
+            __threadfence();
 #pragma unroll
-            for (int c = 0; c < BNT; c += 4) {
-              if (c < p.M) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int k = 0; k < segs; ++k) {
-                  const float4 t = __ldcg(slot0 + static_cast<size_t>(k) * 128 * (BNT / 4) + (c >> 2));
-                  acc.x += t.x;
-                  acc.y += t.y;
-                  acc.z += t.z;
-                  acc.w += t.w;
+            for (int c0 = 0; c0 < BNT; c0 += 16) {
+              if (c0 < p.M) {
+                float4 t4[4];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                  if (c0 + 4 * q4 < p.M)
+                    t4[q4] = __ldcg(reinterpret_cast<const float4*>(sum + c0 + 4 * q4));
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                  const int c = c0 + 4 * q4;
+                  if (c < p.M) {
+                    const float tv[4] = {t4[q4].x, t4[q4].y, t4[q4].z, t4[q4].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                      if (c + e < p.M)
+                        Y[(c + e) * static_cast<size_t>(p.N) + n] = __float2bfloat16_rn(tv[e]);
+                    __stcg(reinterpret_cast<float4*>(sum + c), make_float4(0.f, 0.f, 0.f, 0.f));
+                  }
                 }
-                const float tv[4] = {acc.x, acc.y, acc.z, acc.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  if (c + e < p.M)
-                    Y[(c + e) * static_cast<size_t>(p.N) + n] = __float2bfloat16_rn(tv[e]);
               }
             }
             if (lead) p.counters[i] = 0u;
@@ -623,30 +663,6 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         }
       }
       u = i * KB + kbb;
-    }
-    // ---- 4. every CTA checks in as a reader of t; the last one clears it for next call
-    if (eg == 0 && adapter) {
-      named_bar(bar_id, 128);
-      if (lead) {
-        bool ready = t_read || wait_global_flag(&p.tflags[1], 1u);
-        if (!ready) {
-          stream_timeout(p, ctrl);
-          *gflag = 0;
-        } else {
-          const uint32_t prev = atomicAdd(&p.tflags[2], 1u);
-          *gflag = prev == static_cast<uint32_t>(G - 1) ? 4 : 0;
-        }
-      }
-      named_bar(bar_id, 128);
-      if (*gflag == 4) {
-        for (int e = r; e < BNT * p.R16; e += 128) p.tacc[e] = 0.0f;
-        __threadfence();
-        named_bar(bar_id, 128);
-        if (lead) {
-          p.tflags[2] = 0u;
-          st_release(&p.tflags[1], 0u);
-        }
-      }
     }
   } else {
     // ================================================================ decoders
@@ -663,6 +679,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     const int nunits = u1 - u0;
     const bool leader = wg == 0 && lane == 0;  // issues the group's X-tile copies
     int last_x = -1;
+    griddep_wait();
     for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
       const int sc = it % SC, sa = it % SA;
       if (!mbar_wait(&ctrl->cfull[sc], (it / SC) & 1)) {
@@ -719,14 +736,24 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         tma_load_2d(xbuf(sa), &tmX, ((u0 + it) % KB) * 64, 0, &ctrl->xfull[sa]);
         last_x = it;
       }
-      // ---- expansion: 4 rows x 8 chunks per step
-#pragma unroll 2
-      for (int st = 0; st < RPW / 4; ++st) {
-        const int row = RPW * wg + 4 * st + (lane >> 3);
-        const int c = lane & 7;
-        const uint32_t e = cs[row * 8 + c];
-        const uint4 out = expand_byte<SEL_LUT>(vals, e & 0xFFFFu, e >> 16, lut);
-        *reinterpret_cast<uint4*>(ab + row * 128 + ((c ^ (row & 7)) << 4)) = out;
+      // ---- expansion: 4 rows x 8 chunks per step, four steps per batch; every
+      //      shared-memory load of a batch is issued before its arithmetic and stores
+      static_assert((RPW / 4) % 4 == 0, "steps per batch");
+      const int c = lane & 7;
+#pragma unroll 1
+      for (int st0 = 0; st0 < RPW / 4; st0 += 4) {
+        uint32_t e[4];
+        ExpandIn<SEL_LUT> in[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) e[j] = cs[(RPW * wg + 4 * (st0 + j) + (lane >> 3)) * 8 + c];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) in[j] = expand_load<SEL_LUT>(vals, e[j] & 0xFFFFu, e[j] >> 16, lut);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int row = RPW * wg + 4 * (st0 + j) + (lane >> 3);
+          const uint4 out = expand_compute<SEL_LUT>(in[j], e[j] & 0xFFFFu, e[j] >> 16);
+          *reinterpret_cast<uint4*>(ab + row * 128 + ((c ^ (row & 7)) << 4)) = out;
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();

@@ -52,6 +52,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same condition (try_wait may suspend the thread for a while,
+// test_wait returns at once).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false if the
 // wait ran past kWaitLimitCycles; the caller then records DEV_ERR_TIMEOUT and unwinds.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
@@ -62,6 +75,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 255u) == 0 && clock64() - t0 > kWaitLimitCycles) return false;
   }
+}
+
+// Programmatic dependent launch.  launch_dependents lets the next kernel of the stream
+// (launched with programmatic stream serialization) start its CTAs as this grid's CTAs
+// exit; wait blocks until every preceding grid has completed and its memory operations
+// are visible, and must come before any access to data an earlier kernel may write.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Add four fp32 values into 16-byte aligned global memory; the addition is performed in
+// L2 (no return value, relaxed, gpu scope).
+__device__ __forceinline__ void red_add_v4f32(float* p, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
