@@ -229,6 +229,77 @@ __device__ __forceinline__ uint4 expand_compute(const ExpandIn<SEL_LUT>& in, uin
   return out;
 }
 
+// Chunk table of one decoder warp's RPW rows (rows RPW*wg ..) of a block: entry (row,
+// 8-column chunk) = offset of the chunk's first kept value in the block's value array |
+// the chunk's bitmap byte << 16.  Thread per row: the rows before the warp's own are
+// counted first, then a warp scan of the rows' counts gives each row's start, and a
+// bytewise popcount prefix the chunk offsets within the row.
+template <int RPW>
+__device__ __forceinline__ void build_chunk_table(const uint64_t* bm, uint32_t* cs, int wg, int lane) {
+  uint32_t base = 0;
+  for (int rr = lane; rr < RPW * wg; rr += 32) base += __popcll(bm[rr]);
+  base = warp_sum(base);
+#pragma unroll
+  for (int h = 0; h < (RPW + 31) / 32; ++h) {
+    const int rl = 32 * h + lane;  // row within the warp's rows (lanes past RPW idle)
+    const bool act = rl < RPW;
+    const int row = RPW * wg + rl;
+    const uint64_t w = act ? bm[row] : 0ull;
+    const uint32_t lo = static_cast<uint32_t>(w), hi = static_cast<uint32_t>(w >> 32);
+    const uint32_t clo = __popc(lo), cnt = clo + __popc(hi);
+    const uint32_t inc = warp_incl_scan(cnt);
+    const uint32_t rs = base + inc - cnt;
+    base += __shfl_sync(0xffffffffu, inc, 31);
+    uint32_t bl = lo - ((lo >> 1) & 0x55555555u);
+    bl = (bl & 0x33333333u) + ((bl >> 2) & 0x33333333u);
+    bl = (bl + (bl >> 4)) & 0x0F0F0F0Fu;
+    uint32_t bh = hi - ((hi >> 1) & 0x55555555u);
+    bh = (bh & 0x33333333u) + ((bh >> 2) & 0x33333333u);
+    bh = (bh + (bh >> 4)) & 0x0F0F0F0Fu;
+    const uint32_t plo = bl * 0x01010100u;
+    const uint32_t phi = bh * 0x01010100u + clo * 0x01010101u;
+    // entry = offset | bitmap byte << 16, two uint4 per row
+    uint4 o0, o1;
+    o0.x = rs + (plo & 0xFFu) + ((lo & 0xFFu) << 16);
+    o0.y = rs + ((plo >> 8) & 0xFFu) + (((lo >> 8) & 0xFFu) << 16);
+    o0.z = rs + ((plo >> 16) & 0xFFu) + (((lo >> 16) & 0xFFu) << 16);
+    o0.w = rs + (plo >> 24) + ((lo >> 24) << 16);
+    o1.x = rs + (phi & 0xFFu) + ((hi & 0xFFu) << 16);
+    o1.y = rs + ((phi >> 8) & 0xFFu) + (((hi >> 8) & 0xFFu) << 16);
+    o1.z = rs + ((phi >> 16) & 0xFFu) + (((hi >> 16) & 0xFFu) << 16);
+    o1.w = rs + (phi >> 24) + ((hi >> 24) << 16);
+    if (act) {
+      reinterpret_cast<uint4*>(cs)[2 * row] = o0;
+      reinterpret_cast<uint4*>(cs)[2 * row + 1] = o1;
+    }
+  }
+}
+
+// Expansion of one decoder warp's RPW rows into the decoded tile (K-major, 128-byte
+// swizzle): 4 rows x 8 chunks per step, four steps per batch; every shared-memory load of
+// a batch is issued before its arithmetic and stores.
+template <int RPW, bool SEL_LUT>
+__device__ __forceinline__ void expand_rows(const uint8_t* vals, const uint32_t* cs, uint8_t* ab,
+                                            int wg, int lane, const uint32_t* lut) {
+  static_assert((RPW / 4) % 4 == 0, "steps per batch");
+  const int c = lane & 7;
+#pragma unroll 1
+  for (int st0 = 0; st0 < RPW / 4; st0 += 4) {
+    uint32_t e[4];
+    ExpandIn<SEL_LUT> in[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) e[j] = cs[(RPW * wg + 4 * (st0 + j) + (lane >> 3)) * 8 + c];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) in[j] = expand_load<SEL_LUT>(vals, e[j] & 0xFFFFu, e[j] >> 16, lut);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int row = RPW * wg + 4 * (st0 + j) + (lane >> 3);
+      const uint4 out = expand_compute<SEL_LUT>(in[j], e[j] & 0xFFFFu, e[j] >> 16);
+      *reinterpret_cast<uint4*>(ab + row * 128 + ((c ^ (row & 7)) << 4)) = out;
+    }
+  }
+}
+
 template <int BNT, int NDEC, bool SEL_LUT>
 __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     salr_stream_kernel(const __grid_constant__ StreamParams p,
@@ -444,33 +515,47 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
           mma_ts();
         }
       }
-      int it = 0, seg = 0, nad = 0;
+      // The block loop runs on one thread that shares its SM sub-partition with ALU-bound
+      // decoder warps, so it is kept short: descriptors differ from slot 0's only in the
+      // start-address field (address >> 4, which never carries past its 14 bits in shared
+      // memory), and the slot index and its phase parity advance without division.
+      const uint64_t adesc0 = smem_desc_sw128(smem_u32(abuf(0)), 16, 1024);
+      const uint64_t xdesc0 = smem_desc_sw128(smem_u32(xbuf(0)), 16, 1024);
+      constexpr uint32_t kSlotStep = L::kAent >> 4;
+      uint32_t dec0 = smem_u32(&ctrl->dec[0]), xf0 = smem_u32(&ctrl->xfull[0]);
+      int s = 0;
+      uint32_t ph = 0;
+      int seg = 0, nad = 0;
       for (int u = u0; u < u1 && ok && !stream_aborted(ctrl); ++seg) {
         const int i = u / KB, kba = u % KB;
         const int kbb = min(KB, kba + (u1 - u));
         const int x = seg & 1;
-        (void)i;
         if (!mbar_wait(&ctrl->accempty[x], ((seg >> 1) & 1) ^ 1)) {
           stream_timeout(p, ctrl);
           break;
         }
         tc_fence_after();
         const uint32_t acc = tmem + x * BNT;
-        for (int kb = kba; kb < kbb; ++kb, ++it) {
-          const int s = it % SA;
+        for (int kb = kba; kb < kbb; ++kb) {
           if (ts_done < nts && mbar_test_wait(smem_u32(&ctrl->tsfull), ts_done & 1)) mma_ts();
-          if (!mbar_wait(&ctrl->dec[s], (it / SA) & 1) || !mbar_wait(&ctrl->xfull[s], (it / SA) & 1)) {
-            stream_timeout(p, ctrl);
-            ok = false;
-            break;
+          if (!mbar_try_wait(dec0 + 8 * s, ph) || !mbar_try_wait(xf0 + 8 * s, ph)) {
+            if (!mbar_wait(&ctrl->dec[s], ph) || !mbar_wait(&ctrl->xfull[s], ph)) {
+              stream_timeout(p, ctrl);
+              ok = false;
+              break;
+            }
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(abuf(s)), x0 = smem_u32(xbuf(s));
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(acc, smem_desc_sw128(a0 + 32 * k, 16, 1024),
-                        smem_desc_sw128(x0 + 32 * k, 16, 1024), idesc, (kb != kba) || k != 0);
+          const uint64_t da = adesc0 + s * kSlotStep, dx = xdesc0 + s * kSlotStep;
+          mma_bf16_ss(acc, da, dx, idesc, kb != kba);
+          mma_bf16_ss(acc, da + 2, dx + 2, idesc, 1u);
+          mma_bf16_ss(acc, da + 4, dx + 4, idesc, 1u);
+          mma_bf16_ss(acc, da + 6, dx + 6, idesc, 1u);
           mma_commit(&ctrl->aempty[s]);
+          if (++s == SA) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
         if (!ok) break;
         if (adapter && kba == 0) {
@@ -671,7 +756,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     // it first builds the value offset of each (row, 8-column chunk) of those rows
     // (thread per row), then expands them one bitmap byte per lane.
     constexpr int WPG = NDEC / kStreamGroups;  // warps per group
-    static_assert(WPG * 32 == 128 || WPG * 32 == 64 || WPG * 32 == 256, "rows per warp");
+    static_assert(WPG == 2 || WPG == 4 || WPG == 8, "rows per warp");
     constexpr int RPW = 128 / WPG;             // rows per warp
     const int dw = warp - kStreamFixedWarps;
     const int g = dw / WPG, wg = dw % WPG;
@@ -691,40 +776,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       const uint8_t* vals = cb + kBitmapBytes;
       uint32_t* cs = csb(g);
       uint8_t* ab = abuf(sa);
-      // ---- chunk offsets of this warp's rows
-      uint32_t base = 0;
-      for (int rr = lane; rr < RPW * wg; rr += 32) base += __popcll(bm[rr]);
-      base = warp_sum(base);
-#pragma unroll
-      for (int h = 0; h < RPW / 32; ++h) {
-        const int row = RPW * wg + 32 * h + lane;
-        const uint64_t w = bm[row];
-        const uint32_t lo = static_cast<uint32_t>(w), hi = static_cast<uint32_t>(w >> 32);
-        const uint32_t clo = __popc(lo), cnt = clo + __popc(hi);
-        const uint32_t inc = warp_incl_scan(cnt);
-        const uint32_t rs = base + inc - cnt;
-        base += __shfl_sync(0xffffffffu, inc, 31);
-        uint32_t bl = lo - ((lo >> 1) & 0x55555555u);
-        bl = (bl & 0x33333333u) + ((bl >> 2) & 0x33333333u);
-        bl = (bl + (bl >> 4)) & 0x0F0F0F0Fu;
-        uint32_t bh = hi - ((hi >> 1) & 0x55555555u);
-        bh = (bh & 0x33333333u) + ((bh >> 2) & 0x33333333u);
-        bh = (bh + (bh >> 4)) & 0x0F0F0F0Fu;
-        const uint32_t plo = bl * 0x01010100u;
-        const uint32_t phi = bh * 0x01010100u + clo * 0x01010101u;
-        // entry = offset | bitmap byte << 16, two uint4 per row
-        uint4 o0, o1;
-        o0.x = rs + (plo & 0xFFu) + ((lo & 0xFFu) << 16);
-        o0.y = rs + ((plo >> 8) & 0xFFu) + (((lo >> 8) & 0xFFu) << 16);
-        o0.z = rs + ((plo >> 16) & 0xFFu) + (((lo >> 16) & 0xFFu) << 16);
-        o0.w = rs + (plo >> 24) + ((lo >> 24) << 16);
-        o1.x = rs + (phi & 0xFFu) + ((hi & 0xFFu) << 16);
-        o1.y = rs + ((phi >> 8) & 0xFFu) + (((hi >> 8) & 0xFFu) << 16);
-        o1.z = rs + ((phi >> 16) & 0xFFu) + (((hi >> 16) & 0xFFu) << 16);
-        o1.w = rs + (phi >> 24) + ((hi >> 24) << 16);
-        reinterpret_cast<uint4*>(cs)[2 * row] = o0;
-        reinterpret_cast<uint4*>(cs)[2 * row + 1] = o1;
-      }
+      build_chunk_table<RPW>(bm, cs, wg, lane);
       __syncwarp();
       // ---- the decoded tile's ring entry must be free; the group leader fetches X
       if (!mbar_wait(&ctrl->aempty[sa], ((it / SA) & 1) ^ 1)) {
@@ -736,25 +788,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         tma_load_2d(xbuf(sa), &tmX, ((u0 + it) % KB) * 64, 0, &ctrl->xfull[sa]);
         last_x = it;
       }
-      // ---- expansion: 4 rows x 8 chunks per step, four steps per batch; every
-      //      shared-memory load of a batch is issued before its arithmetic and stores
-      static_assert((RPW / 4) % 4 == 0, "steps per batch");
-      const int c = lane & 7;
-#pragma unroll 1
-      for (int st0 = 0; st0 < RPW / 4; st0 += 4) {
-        uint32_t e[4];
-        ExpandIn<SEL_LUT> in[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) e[j] = cs[(RPW * wg + 4 * (st0 + j) + (lane >> 3)) * 8 + c];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) in[j] = expand_load<SEL_LUT>(vals, e[j] & 0xFFFFu, e[j] >> 16, lut);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int row = RPW * wg + 4 * (st0 + j) + (lane >> 3);
-          const uint4 out = expand_compute<SEL_LUT>(in[j], e[j] & 0xFFFFu, e[j] >> 16);
-          *reinterpret_cast<uint4*>(ab + row * 128 + ((c ^ (row & 7)) << 4)) = out;
-        }
-      }
+      expand_rows<RPW, SEL_LUT>(vals, cs, ab, wg, lane, lut);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
