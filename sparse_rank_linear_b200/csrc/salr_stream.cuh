@@ -505,16 +505,8 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         mma_commit(&ctrl->tsfree);
         if (++ts_done == nts) mma_commit(&ctrl->tsdone);
       };
-      // the t share's data arrives well before the first decoded block: multiply it first
-      // so that t is complete early
-      if (nts > 0) {
-        if (!mbar_wait(&ctrl->tsfull, 0)) {
-          stream_timeout(p, ctrl);
-          ok = false;
-        } else {
-          mma_ts();
-        }
-      }
+      // the t share is multiplied as soon as its data has landed (polled between blocks),
+      // never ahead of decoded blocks: it is fetched only after the dependency wait
       // The block loop runs on one thread that shares its SM sub-partition with ALU-bound
       // decoder warps, so it is kept short: descriptors differ from slot 0's only in the
       // start-address field (address >> 4, which never carries past its 14 bits in shared
