@@ -272,7 +272,7 @@ uint32_t bind_call(StreamParams& sp, float* acc, uint32_t* counters, float* tacc
   return epoch;
 }
 
-template <int BNT, bool SEL_LUT>
+template <int BNT>
 int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
                   const CUtensorMap& tb, int sms, cudaStream_t st) {
   using L = StreamLayout<BNT>;
@@ -292,7 +292,7 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
   if (!attr_set[dev]) {
-    SALR_TRY(cudaFuncSetAttribute(salr_stream_kernel<BNT, kStreamDecoders, SEL_LUT>,
+    SALR_TRY(cudaFuncSetAttribute(salr_stream_kernel<BNT, kStreamDecoders>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
     attr_set[dev] = true;
   }
@@ -321,7 +321,7 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  SALR_TRY(cudaLaunchKernelEx(&cfg, salr_stream_kernel<BNT, kStreamDecoders, SEL_LUT>, p, tx, ta,
+  SALR_TRY(cudaLaunchKernelEx(&cfg, salr_stream_kernel<BNT, kStreamDecoders>, p, tx, ta,
                               tb));
   return SALR_OK;
 }
@@ -493,22 +493,10 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
       if (!make_map(&tb, B_cat, h->N, R, 64, sp.R16)) return SALR_ERR_CUDA;
     }
     const int sms = device_sms(h->device);
-    // selector source of the decoder (shared-memory table or registers); registers by
-    // default, SALR_DECODE_LUT=1 selects the table (kept for measurements)
-    const char* lutv = getenv("SALR_DECODE_LUT");
-    const bool use_lut = lutv && lutv[0] == '1';
     switch (bnt) {
-      case 16:
-        rc = use_lut ? launch_stream<16, true>(sp, tx, ta, tb, sms, st)
-                     : launch_stream<16, false>(sp, tx, ta, tb, sms, st);
-        break;
-      case 32:
-        rc = use_lut ? launch_stream<32, true>(sp, tx, ta, tb, sms, st)
-                     : launch_stream<32, false>(sp, tx, ta, tb, sms, st);
-        break;
-      default:
-        rc = use_lut ? launch_stream<64, true>(sp, tx, ta, tb, sms, st)
-                     : launch_stream<64, false>(sp, tx, ta, tb, sms, st);
+      case 16: rc = launch_stream<16>(sp, tx, ta, tb, sms, st); break;
+      case 32: rc = launch_stream<32>(sp, tx, ta, tb, sms, st); break;
+      default: rc = launch_stream<64>(sp, tx, ta, tb, sms, st);
     }
     if (rc == SALR_OK) h->sscr.epoch = epoch;
     return rc;
@@ -748,7 +736,7 @@ extern "C" int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, cons
     if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
     if (!make_map(&tb, B_cat, h->N, R, 64, sp.R16)) return SALR_ERR_CUDA;
   }
-  rc = launch_stream<16, false>(sp, tx, ta, tb, device_sms(h->device), st);
+  rc = launch_stream<16>(sp, tx, ta, tb, device_sms(h->device), st);
   if (rc == SALR_OK) noalloc_commit_epoch(dev, epoch);
   return rc;
 }

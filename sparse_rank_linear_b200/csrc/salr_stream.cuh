@@ -14,9 +14,9 @@
 //   groups, each group on a different block so that several blocks are in flight.  A
 //   warp first turns the bitmap words of its 32 rows into the offset of every (row,
 //   8-column chunk) in the compact value array, then expands one bitmap byte per lane:
-//   an aligned 12-value window is loaded from shared memory, shifted to the chunk's first
-//   value and spread over the eight columns by byte permutes whose selectors come from a
-//   16-entry nibble lookup table.
+//   each nibble reads three 32-bit words from the 4-byte boundary at or below its first
+//   value, shifts them by a halfword when that value is odd, and spreads them over its
+//   four columns with byte permutes whose selectors come from a 16-entry table.
 // * Stage 2: tcgen05 bf16 MMAs into a double-buffered TMEM accumulator, pipelined
 //   against the decode through shared-memory stages filled by TMA.
 // * Concatenated adapter (Methodology 3): t = X A_cat is computed once per call.  The
@@ -92,7 +92,7 @@ struct StreamLayout {
     return cs_off(cbuf, sa, sc) + groups * kCs;
   }
   __host__ __device__ static int smem_bytes(int cbuf, int bcbuf, int sa, int sc, int groups) {
-    return fixed_off(cbuf, sa, sc, groups) + kTbuf + bcbuf + 1024 /*ctrl*/ + 4096 /*lut*/ +
+    return fixed_off(cbuf, sa, sc, groups) + kTbuf + bcbuf + 1024 /*ctrl*/ + 128 /*nibbles*/ +
            1024 /*align*/;
   }
 };
@@ -145,87 +145,61 @@ __device__ __forceinline__ int owner_of(long long u, long long U, int G) {
   return c;
 }
 
-// Selectors for the nibble lookup table.  For a 4-bit mask t over 4 output columns and
-// a window E0 = (h0, h1), E1 = (h2, h3) holding the nibble's kept values in order:
-//   out0 = prmt(E0, 0, lo) places h0/h1 in columns 0/1 (or zero),
-//   pair = prmt(E0, E1, lo >> 16) brings the next two unused values to the bottom,
-//   out1 = prmt(pair, 0, hi) places them in columns 2/3 (or zero).
+// Expansion of a bitmap byte into 8 bf16 columns.  A nibble n (4 columns) whose kept
+// values, in order, sit in the window (W0, W1) from its first one expands as
+//   word 0 (columns 0, 1) = prmt(W0, 0, PAT(n & 3))
+//   word 1 (columns 2, 3) = prmt(prmt(W0, W1, PAIR(popc(n & 3))), 0, PAT(n >> 2))
+// where PAT(v), v the 2-bit mask of two columns, is 0x4444 / 0x4410 / 0x1044 / 0x3210
+// (both zero, first value low, first value high, both values; selector 4 reads the zero
+// operand) and PAIR(s) = 0x3210 + 0x2222 s brings values s, s + 1 to the bottom.  The
+// selectors of the 16 nibbles sit in a 128-byte table in shared memory (conflict-free
+// reads): entry n = {PAT(n & 3) | PAT(n >> 2) << 16, PAIR(popc(n & 3))}.
 __device__ __forceinline__ uint32_t pat2(uint32_t v) {
   return v == 0 ? 0x4444u : v == 1 ? 0x4410u : v == 2 ? 0x1044u : 0x3210u;
 }
-
-__device__ __forceinline__ uint32_t funnel16(uint32_t lo, uint32_t hi, uint32_t sh) {
-  return __funnelshift_r(lo, hi, sh);
+__device__ __forceinline__ uint2 nibble_entry(uint32_t n) {
+  return make_uint2(pat2(n & 3u) | (pat2(n >> 2) << 16), 0x3210u + 0x2222u * __popc(n & 3u));
 }
 
-// Expansion of one bitmap byte `b` whose values start at halfword p of the block's value
-// array (shared memory, 16-byte aligned, readable 24 bytes past its end), in two parts so
-// that a decoder can issue the shared-memory loads of several bytes before any of their
-// arithmetic.  The window is the 12 values from the 8-byte boundary at or below p: the
-// low nibble's values start at halfword o = p mod 4 of it and the high nibble's at
-// x = o + popc(low nibble) <= 7.  Window bytes that lie past the block's values only ever
-// meet columns whose mask bit is clear, which the byte permutes zero.  SEL_LUT takes the
-// byte-permute selectors from the nibble table in shared memory, otherwise they are built
-// in registers:
-//   PAT(v), v the 2-bit mask of two columns, is 0x4444 / 0x4410 / 0x1044 / 0x3210 (both
-//   zero, first value low, first value high, both values), looked up for all four
-//   column pairs at once by one byte permute of a constant table;
-//   PAIR(s) = 0x3210 + 0x2222 s brings values s, s+1 of a window to the bottom.
-template <bool SEL_LUT>
+// Shared-memory operands of one byte's expansion: each nibble's window is the three
+// 32-bit words from the 4-byte boundary at or below its first value (the low nibble's at
+// halfword p, the high nibble's at q = p + popc(low nibble)); words past the block's values
+// (the value array is readable 24 bytes past its end) only meet columns whose mask bit is
+// clear, which the permutes zero.
 struct ExpandIn {
-  uint2 a0, a1, a2;  // the window
-  uint4 sel;         // nibble-table entry (SEL_LUT only)
+  uint32_t a0, a1, a2, c0, c1, c2;  // low / high nibble windows
+  uint2 el, eh;                     // nibble-table entries
+  uint32_t p, q;
 };
 
-template <bool SEL_LUT>
-__device__ __forceinline__ ExpandIn<SEL_LUT> expand_load(const uint8_t* vals, uint32_t p,
-                                                         uint32_t b, const uint32_t* lut) {
-  ExpandIn<SEL_LUT> in;
-  const uint8_t* wp = vals + ((p & ~3u) << 1);
-  in.a0 = lds64(wp);
-  in.a1 = lds64(wp + 8);
-  in.a2 = lds64(wp + 16);
-  if constexpr (SEL_LUT) in.sel = reinterpret_cast<const uint4*>(lut)[b];
+__device__ __forceinline__ ExpandIn expand_load(const uint8_t* vals, uint32_t p, uint32_t b,
+                                                const uint2* nt) {
+  ExpandIn in;
+  in.p = p;
+  in.q = p + __popc(b & 15u);
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(vals + ((p & ~1u) << 1));
+  const uint32_t* v = reinterpret_cast<const uint32_t*>(vals + ((in.q & ~1u) << 1));
+  in.a0 = w[0];
+  in.a1 = w[1];
+  in.a2 = w[2];
+  in.c0 = v[0];
+  in.c1 = v[1];
+  in.c2 = v[2];
+  in.el = nt[b & 15u];
+  in.eh = nt[b >> 4];
   return in;
 }
 
-template <bool SEL_LUT>
-__device__ __forceinline__ uint4 expand_compute(const ExpandIn<SEL_LUT>& in, uint32_t p,
-                                                uint32_t b) {
-  const uint32_t W0 = in.a0.x, W1 = in.a0.y, W2 = in.a1.x, W3 = in.a1.y, W4 = in.a2.x,
-                 W5 = in.a2.y;
-  const uint32_t o = p & 3u;
-  const uint32_t x = o + __popc(b & 15u);  // first value of the high nibble
-  // low nibble: window at halfword o
-  const bool o2 = (o & 2u) != 0;
-  const uint32_t sh0 = (o & 1u) << 4;
-  const uint32_t U0 = o2 ? W1 : W0, U1 = o2 ? W2 : W1, U2 = o2 ? W3 : W2;
-  const uint32_t L0 = funnel16(U0, U1, sh0), L1 = funnel16(U1, U2, sh0);
-  // high nibble: window at halfword x
-  const bool x4 = (x & 4u) != 0, x2 = (x & 2u) != 0;
-  const uint32_t sh1 = (x & 1u) << 4;
-  const uint32_t T0 = x4 ? W2 : W0, T1 = x4 ? W3 : W1, T2 = x4 ? W4 : W2, T3 = x4 ? W5 : W3;
-  const uint32_t V0 = x2 ? T1 : T0, V1 = x2 ? T2 : T1, V2 = x2 ? T3 : T2;
-  const uint32_t H0 = funnel16(V0, V1, sh1), H1 = funnel16(V1, V2, sh1);
-  uint32_t pat01, pat23, pr0, pr1;
-  if constexpr (SEL_LUT) {
-    pat01 = in.sel.x;
-    pat23 = in.sel.y;
-    pr0 = in.sel.z;
-    pr1 = in.sel.z >> 16;
-  } else {
-    const uint32_t bs = (b & 3u) | ((b & 0xCu) << 6) | ((b & 0x30u) << 12) | ((b & 0xC0u) << 18);
-    const uint32_t idx = bs * 0x22u + 0x10101010u;
-    pat01 = __byte_perm(0x44104444u, 0x32101044u, idx);
-    pat23 = __byte_perm(0x44104444u, 0x32101044u, idx >> 16);
-    pr0 = 0x3210u + 0x2222u * __popc(b & 3u);
-    pr1 = 0x3210u + 0x2222u * __popc(b & 0x30u);
-  }
+__device__ __forceinline__ uint4 expand_compute(const ExpandIn& in) {
+  // windows start at the nibbles' first values: shift by one halfword when that is odd
+  const uint32_t sh0 = (in.p & 1u) << 4, sh1 = (in.q & 1u) << 4;
+  const uint32_t L0 = __funnelshift_r(in.a0, in.a1, sh0), L1 = __funnelshift_r(in.a1, in.a2, sh0);
+  const uint32_t H0 = __funnelshift_r(in.c0, in.c1, sh1), H1 = __funnelshift_r(in.c1, in.c2, sh1);
   uint4 out;
-  out.x = __byte_perm(L0, 0u, pat01);
-  out.y = __byte_perm(__byte_perm(L0, L1, pr0), 0u, pat01 >> 16);
-  out.z = __byte_perm(H0, 0u, pat23);
-  out.w = __byte_perm(__byte_perm(H0, H1, pr1), 0u, pat23 >> 16);
+  out.x = __byte_perm(L0, 0u, in.el.x);
+  out.y = __byte_perm(__byte_perm(L0, L1, in.el.y), 0u, in.el.x >> 16);
+  out.z = __byte_perm(H0, 0u, in.eh.x);
+  out.w = __byte_perm(__byte_perm(H0, H1, in.eh.y), 0u, in.eh.x >> 16);
   return out;
 }
 
@@ -276,31 +250,21 @@ __device__ __forceinline__ void build_chunk_table(const uint64_t* bm, uint32_t* 
 }
 
 // Expansion of one decoder warp's RPW rows into the decoded tile (K-major, 128-byte
-// swizzle): 4 rows x 8 chunks per step, four steps per batch; every shared-memory load of
-// a batch is issued before its arithmetic and stores.
-template <int RPW, bool SEL_LUT>
+// swizzle): 4 rows x 8 chunks per step, one bitmap byte per lane.
+template <int RPW>
 __device__ __forceinline__ void expand_rows(const uint8_t* vals, const uint32_t* cs, uint8_t* ab,
-                                            int wg, int lane, const uint32_t* lut) {
-  static_assert((RPW / 4) % 4 == 0, "steps per batch");
+                                            int wg, int lane, const uint2* nt) {
   const int c = lane & 7;
-#pragma unroll 1
-  for (int st0 = 0; st0 < RPW / 4; st0 += 4) {
-    uint32_t e[4];
-    ExpandIn<SEL_LUT> in[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) e[j] = cs[(RPW * wg + 4 * (st0 + j) + (lane >> 3)) * 8 + c];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) in[j] = expand_load<SEL_LUT>(vals, e[j] & 0xFFFFu, e[j] >> 16, lut);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int row = RPW * wg + 4 * (st0 + j) + (lane >> 3);
-      const uint4 out = expand_compute<SEL_LUT>(in[j], e[j] & 0xFFFFu, e[j] >> 16);
-      *reinterpret_cast<uint4*>(ab + row * 128 + ((c ^ (row & 7)) << 4)) = out;
-    }
+#pragma unroll 2
+  for (int st = 0; st < RPW / 4; ++st) {
+    const int row = RPW * wg + 4 * st + (lane >> 3);
+    const uint32_t e = cs[row * 8 + c];
+    const ExpandIn in = expand_load(vals, e & 0xFFFFu, e >> 16, nt);
+    *reinterpret_cast<uint4*>(ab + row * 128 + ((c ^ (row & 7)) << 4)) = expand_compute(in);
   }
 }
 
-template <int BNT, int NDEC, bool SEL_LUT>
+template <int BNT, int NDEC>
 __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     salr_stream_kernel(const __grid_constant__ StreamParams p,
                        const __grid_constant__ CUtensorMap tmX,
@@ -320,7 +284,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
   uint8_t* tbuf = smem + L::fixed_off(p.cbuf, SA, SC, kStreamGroups);
   uint8_t* bcbuf = tbuf + L::kTbuf;  // B_cat^T tile; at kernel start, the t-share stage
   StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(bcbuf + p.bcbuf);
-  uint32_t* lutp = reinterpret_cast<uint32_t*>(bcbuf + p.bcbuf + 1024);  // 256 x 16 B
+  uint2* ntab = reinterpret_cast<uint2*>(bcbuf + p.bcbuf + 1024);  // 16 x 8 B nibble table
 
   griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -365,15 +329,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     ctrl->flag[0] = ctrl->flag[1] = 0;
     fence_mbar_init();
   }
-  if (SEL_LUT && threadIdx.x < 256) {
-    const uint32_t b = threadIdx.x;
-    uint4 e;
-    e.x = pat2(b & 3u) | (pat2((b >> 2) & 3u) << 16);
-    e.y = pat2((b >> 4) & 3u) | (pat2(b >> 6) << 16);
-    e.z = (0x3210u + 0x2222u * __popc(b & 3u)) | ((0x3210u + 0x2222u * __popc(b & 0x30u)) << 16);
-    e.w = 0u;
-    reinterpret_cast<uint4*>(lutp)[b] = e;
-  }
+  if (threadIdx.x < 16) ntab[threadIdx.x] = nibble_entry(threadIdx.x);
   if (warp == 1) tmem_alloc(&ctrl->tmem, kCols);
   tc_fence_before();
   __syncthreads();
@@ -752,7 +708,6 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     constexpr int RPW = 128 / WPG;             // rows per warp
     const int dw = warp - kStreamFixedWarps;
     const int g = dw / WPG, wg = dw % WPG;
-    const uint32_t* lut = lutp;
     const int nunits = u1 - u0;
     const bool leader = wg == 0 && lane == 0;  // issues the group's X-tile copies
     int last_x = -1;
@@ -780,7 +735,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         tma_load_2d(xbuf(sa), &tmX, ((u0 + it) % KB) * 64, 0, &ctrl->xfull[sa]);
         last_x = it;
       }
-      expand_rows<RPW, SEL_LUT>(vals, cs, ab, wg, lane, lut);
+      expand_rows<RPW>(vals, cs, ab, wg, lane, ntab);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
