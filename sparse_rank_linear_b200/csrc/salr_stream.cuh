@@ -486,12 +486,30 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         const uint32_t acc = tmem + x * BNT;
         for (int kb = kba; kb < kbb; ++kb) {
           if (ts_done < nts && mbar_test_wait(smem_u32(&ctrl->tsfull), ts_done & 1)) mma_ts();
-          if (!mbar_try_wait(dec0 + 8 * s, ph) || !mbar_try_wait(xf0 + 8 * s, ph)) {
-            if (!mbar_wait(&ctrl->dec[s], ph) || !mbar_wait(&ctrl->xfull[s], ph)) {
+          if (ts_done < nts) {
+            // while the block is still being decoded, take the t share once it has landed
+            const long long t0 = clock64();
+            while (!mbar_test_wait(dec0 + 8 * s, ph)) {
+              if (ts_done < nts && mbar_test_wait(smem_u32(&ctrl->tsfull), ts_done & 1)) mma_ts();
+              if (clock64() - t0 > kWaitLimitCycles || stream_aborted(ctrl)) {
+                ok = false;
+                break;
+              }
+              __nanosleep(32);
+            }
+            if (!ok) {
               stream_timeout(p, ctrl);
-              ok = false;
               break;
             }
+          } else if (!mbar_try_wait(dec0 + 8 * s, ph) && !mbar_wait(&ctrl->dec[s], ph)) {
+            stream_timeout(p, ctrl);
+            ok = false;
+            break;
+          }
+          if (!mbar_try_wait(xf0 + 8 * s, ph) && !mbar_wait(&ctrl->xfull[s], ph)) {
+            stream_timeout(p, ctrl);
+            ok = false;
+            break;
           }
           tc_fence_after();
           const uint64_t da = adesc0 + s * kSlotStep, dx = xdesc0 + s * kSlotStep;
