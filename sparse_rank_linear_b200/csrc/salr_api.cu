@@ -30,7 +30,7 @@ struct Workspace {
 };
 
 // Scratch of the persistent small-M kernel: fp32 sums of split row tiles [N x 64] and
-// their arrival counts [N/128] (left zeroed by every call), and two fp32 t = X A_cat
+// their arrival counts [N/128 x 4 quarters] (left zeroed by every call), and two fp32 t = X A_cat
 // accumulators [64 x 128] with their arrival counts, used by alternate calls; each call
 // clears the buffer the next call will use.  `epoch` counts the calls.
 struct StreamScratch {
@@ -230,7 +230,7 @@ int ensure_stream_scratch(salr_weight_s* h, cudaStream_t st) {
   if (h->sscr.acc) return SALR_OK;
   void *a = nullptr, *b = nullptr, *c = nullptr, *d = nullptr;
   const size_t ab = static_cast<size_t>(h->N) * 64 * sizeof(float);
-  const size_t cb = static_cast<size_t>(h->N / 128) * sizeof(uint32_t);
+  const size_t cb = static_cast<size_t>(h->N / 128) * 4 * sizeof(uint32_t);
   const size_t tb = 2 * kTBuf * sizeof(float);
   cudaError_t e;
   if ((e = dev_alloc(&a, ab)) != cudaSuccess || (e = dev_alloc(&b, cb)) != cudaSuccess ||
@@ -611,7 +611,7 @@ int salr_sync_status(salr_handle h, void* stream) {
     SALR_TRY(cudaMemset(h->work.counters, 0, h->work.n_counters * sizeof(uint32_t)));
   if (h->sscr.acc) {
     SALR_TRY(cudaMemset(h->sscr.acc, 0, static_cast<size_t>(h->N) * 64 * sizeof(float)));
-    SALR_TRY(cudaMemset(h->sscr.counters, 0, static_cast<size_t>(h->N / 128) * sizeof(uint32_t)));
+    SALR_TRY(cudaMemset(h->sscr.counters, 0, static_cast<size_t>(h->N / 128) * 4 * sizeof(uint32_t)));
     SALR_TRY(cudaMemset(h->sscr.tacc, 0, 2 * kTBuf * sizeof(float)));
     SALR_TRY(cudaMemset(h->sscr.tflags, 0, 2 * sizeof(uint32_t)));
   }
@@ -640,12 +640,12 @@ constexpr int64_t kNoAllocMaxM = 16;     // tokens per call
 constexpr int64_t kNoAllocMaxN = 32768;  // output features
 constexpr int kNoAllocMaxSMs = 160;      // CTAs of the persistent kernel
 // layout: [t counts: 2 u32][t accumulators: 2 x 16 x 128 f32]
-//         [split-tile arrival counts: N/128 u32][split-tile sums: N x 16 f32]
+//         [split-tile arrival counts: N/128 x 4 u32][split-tile sums: N x 16 f32]
 constexpr int kNaTBuf = 16 * 128;
 constexpr size_t kNaFlags = 0;
 constexpr size_t kNaTacc = 256;
 constexpr size_t kNaCounters = kNaTacc + 2 * kNaTBuf * sizeof(float);
-constexpr size_t kNaAcc = kNaCounters + (kNoAllocMaxN / 128) * sizeof(uint32_t);
+constexpr size_t kNaAcc = kNaCounters + (kNoAllocMaxN / 128) * 4 * sizeof(uint32_t);
 constexpr size_t kNaBytes = kNaAcc + static_cast<size_t>(kNoAllocMaxN) * 16 * sizeof(float);
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];

@@ -7,9 +7,9 @@
 //   contiguous range per CTA (one CTA per SM, every SM the same number of blocks).  A
 //   range covers one or more row-tile segments.  A segment that does not cover a whole
 //   row tile adds its fp32 partial into the tile's fp32 accumulator with vector
-//   reductions performed in L2, fences, and counts itself in; the last segment of the
-//   tile to arrive (no waiting) reads the sum, writes the bf16 output and clears the
-//   accumulator and its count for the next call.
+//   reductions performed in L2, fences, and counts itself in per 32-row quarter; the last
+//   warp to arrive for a quarter (no waiting) reads its sum, writes the bf16 output and
+//   clears the accumulator and the count for the next call.
 // * Stage 1 decode (SALR technical summary, Methodology 4): decoder warps work in
 //   groups, each group on a different block so that several blocks are in flight.  A
 //   warp first turns the bitmap words of its 32 rows into the offset of every (row,
@@ -53,7 +53,7 @@ struct StreamParams {
   const uint32_t* offsets;
   uint16_t* Y;
   float* acc;            // [RT x 128 x BNT] fp32 sums of split row tiles, zero between calls
-  uint32_t* counters;    // [RT] segments of each split tile arrived, zero between calls
+  uint32_t* counters;    // [RT x 4] segments arrived per split tile and 32-row quarter, zero between calls
   float* tacc;           // [BNT x R16] fp32 accumulator of t = X A_cat (this call's buffer)
   float* tacc_next;      // the other buffer, cleared by this call for the next one
   uint32_t* tflag;       // t parts arrived in this call's buffer
@@ -674,19 +674,19 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->accempty[x]);
         if (!whole) {
-          // every thread's additions are performed before the tile's count moves
+          // Each warp counts its 32 rows of the tile in on its own: its additions are
+          // performed first (fence), and the warp that arrives last for these rows reads
+          // their sum, writes Y and clears the sum and the count for the next call.
           __threadfence();
-          named_bar(bar_id, 128);
-          if (lead) {
+          __syncwarp();
+          uint32_t last = 0;
+          if (lane == 0) {
             const int c_first = owner_of(static_cast<long long>(i) * KB, U, G);
             const int segs =
                 owner_of(static_cast<long long>(i) * KB + KB - 1, U, G) - c_first + 1;
-            const uint32_t prev = atomicAdd(p.counters + i, 1u);
-            *gflag = prev == static_cast<uint32_t>(segs - 1) ? 3 : 2;
+            last = atomicAdd(p.counters + 4 * i + q, 1u) == static_cast<uint32_t>(segs - 1);
           }
-          named_bar(bar_id, 128);
-          if (*gflag == 3) {
-            __threadfence();
+          if (__shfl_sync(0xffffffffu, last, 0)) {
 #pragma unroll
             for (int c0 = 0; c0 < BNT; c0 += 16) {
               if (c0 < p.M) {
@@ -709,7 +709,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
                 }
               }
             }
-            if (lead) p.counters[i] = 0u;
+            if (lane == 0) p.counters[4 * i + q] = 0u;
           }
         }
       }
