@@ -36,7 +36,7 @@ METRIC = "SALR linear tokens/s + achieved fraction of HBM/tensor roofline on 1 B
 WORKLOAD = "q_proj"
 M_TOKENS = 16
 L2_BYTES = 126 * 1024 * 1024
-KERNEL_SOURCES = ["sm100.cuh", "salr_codec.cuh", "salr_linear.cuh", "salr_stream.cuh", "salr_api.cu"]
+KERNEL_SOURCES = ["sm100.cuh", "salr_codec.cuh", "salr_prefill.cuh", "salr_stream.cuh", "salr_api.cu"]
 
 
 def algorithmic_bytes(N, K, R, M, keep):

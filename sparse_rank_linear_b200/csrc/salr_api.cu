@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -13,7 +14,7 @@
 
 #include "../../include/salr.h"
 #include "salr_codec.cuh"
-#include "salr_linear.cuh"
+#include "salr_prefill.cuh"
 #include "salr_stream.cuh"
 
 using namespace salr;
@@ -21,12 +22,24 @@ using namespace salr;
 namespace {
 
 constexpr uint64_t kMagic = 0x53414c5257454754ull;  // "SALRWEGT"
+constexpr int kSmemLimit = 232448;  // B200 opt-in dynamic shared memory per CTA
 
+// Split-K scratch of the prefill kernel: fp32 tile sums and arrival counts (grown on
+// demand, left zeroed by every call).
 struct Workspace {
   float* ws = nullptr;
   size_t ws_elems = 0;
   uint32_t* counters = nullptr;
   size_t n_counters = 0;
+};
+
+// Prefill adapter scratch: t = X A_cat as bf16 [M x 128], its fp32 split sums [128 x M]
+// and their arrival counts (grown on demand; sums and counts left zeroed by every call).
+struct TScratch {
+  uint16_t* T = nullptr;
+  float* T32 = nullptr;
+  uint32_t* counters = nullptr;
+  int64_t rows = 0;  // token capacity (multiple of 256)
 };
 
 // Scratch of the persistent small-M kernel: fp32 sums of split row tiles [N x 64] and
@@ -56,6 +69,7 @@ struct salr_weight_s {
   int* status;  // device status word (DEV_ERR_* bits)
   uint32_t max16;  // largest encoded block, 16-byte units
   Workspace work;
+  TScratch tscr;
   StreamScratch sscr;
   uint8_t* x_stage;  // salr_linear_host staging
   size_t x_cap;
@@ -146,6 +160,9 @@ void release(salr_weight_s* h) {
   cudaFree(h->status);
   cudaFree(h->work.ws);
   cudaFree(h->work.counters);
+  cudaFree(h->tscr.T);
+  cudaFree(h->tscr.T32);
+  cudaFree(h->tscr.counters);
   cudaFree(h->x_stage);
   cudaFree(h->y_stage);
   h->magic = 0;
@@ -183,44 +200,92 @@ int ensure_workspace(salr_weight_s* h, size_t elems, size_t ctrs, cudaStream_t s
   return SALR_OK;
 }
 
-struct Schedule {
-  int bnt, tt, splits;
-};
-
-Schedule choose_schedule(int64_t M, int64_t N, int64_t K, int sms) {
-  Schedule s;
-  s.bnt = M <= 16 ? 16 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
-  s.tt = static_cast<int>((M + s.bnt - 1) / s.bnt);
-  const int64_t tiles = (N / 128) * s.tt;
-  const int kblocks = static_cast<int>(K / 64);
-  int splits = 1;
-  if (tiles < sms) {
-    splits = static_cast<int>(sms / tiles);
-    if (splits > kblocks) splits = kblocks;
-    if (splits < 1) splits = 1;
+int ensure_tscratch(salr_weight_s* h, int64_t M, cudaStream_t st) {
+  const int64_t rows = (M + 255) / 256 * 256;
+  if (rows <= h->tscr.rows) return SALR_OK;
+  if (h->tscr.T) {
+    SALR_TRY(cudaStreamSynchronize(st));
+    cudaFree(h->tscr.T);
+    cudaFree(h->tscr.T32);
+    cudaFree(h->tscr.counters);
+    h->tscr = TScratch{};
   }
-  s.splits = splits;
-  return s;
+  void *a = nullptr, *b = nullptr, *c = nullptr;
+  const size_t tb = static_cast<size_t>(rows) * 128 * sizeof(uint16_t);
+  const size_t t32b = static_cast<size_t>(rows) * 128 * sizeof(float);
+  const size_t cb = static_cast<size_t>(rows / 128) * 4 * sizeof(uint32_t);
+  cudaError_t e;
+  if ((e = dev_alloc(&a, tb)) != cudaSuccess || (e = dev_alloc(&b, t32b)) != cudaSuccess ||
+      (e = dev_alloc(&c, cb)) != cudaSuccess) {
+    cudaFree(a);
+    cudaFree(b);
+    cudaFree(c);
+    return cuda_status(e);
+  }
+  h->tscr.T = static_cast<uint16_t*>(a);
+  h->tscr.T32 = static_cast<float*>(b);
+  h->tscr.counters = static_cast<uint32_t*>(c);
+  h->tscr.rows = rows;
+  SALR_TRY(cudaMemsetAsync(a, 0, tb, st));
+  SALR_TRY(cudaMemsetAsync(b, 0, t32b, st));
+  SALR_TRY(cudaMemsetAsync(c, 0, cb, st));
+  return SALR_OK;
 }
 
 template <int BNT>
-int launch_linear(const LinParams& p, const CUtensorMap& tx, const CUtensorMap& ta,
-                  const CUtensorMap& tb, int grid, cudaStream_t st) {
-  constexpr int smem = LinLayout<BNT>::kSmemBytes;
+int launch_t(const TParams& p, const CUtensorMap& tx, const CUtensorMap& ta, int grid,
+             cudaStream_t st) {
+  constexpr int smem = TLayout<BNT>::kSmemBytes;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
   if (!attr_set[dev]) {
-    SALR_TRY(cudaFuncSetAttribute(salr_linear_kernel<BNT>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    SALR_TRY(cudaFuncSetAttribute(salr_t_kernel<BNT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem));
     attr_set[dev] = true;
   }
-  salr_linear_kernel<BNT><<<grid, kLinThreads, smem, st>>>(p, tx, ta, tb);
+  salr_t_kernel<BNT><<<grid, kTThreads, smem, st>>>(p, tx, ta);
   SALR_TRY(cudaGetLastError());
   return SALR_OK;
 }
 
+template <int BNT>
+int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb,
+                   const CUtensorMap& tt, int grid, cudaStream_t st) {
+  using L = PrefillLayout<BNT>;
+  // One decoded-tile slot per decoder group plus one; as many X tiles as leave room for
+  // one compact-block slot per decoder group; the rest of shared memory for compact
+  // blocks.  The compact-block slots come in a multiple of the group count, so that slot
+  // s only ever holds blocks of group s mod 4: a group then never waits on a slot whose
+  // previous fill it has not consumed itself, and a parity wait can never pass on a phase
+  // two fills old.
+  p.sa = kPreGroups + 1;
+  int sx = kPreMaxX, sc = 0;
+  for (; sx >= 2; --sx) {
+    sc = (kSmemLimit - L::smem_bytes(p.sa, sx, 0, p.cbuf)) / p.cbuf;
+    if (sc >= kPreGroups) break;
+  }
+  if (sx < 2 || sc < kPreGroups) return SALR_ERR_UNSUPPORTED;
+  if (sc > kPreMaxC) sc = kPreMaxC;
+  sc -= sc % kPreGroups;
+  p.sx = sx;
+  p.sc = sc;
+  if (L::table_off(p.sa, p.sx, p.sc, p.cbuf) < L::kAdapterBytes) return SALR_ERR_UNSUPPORTED;
+  const int smem = L::smem_bytes(p.sa, p.sx, p.sc, p.cbuf);
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
+  if (!attr_set[dev]) {
+    SALR_TRY(cudaFuncSetAttribute(salr_prefill_kernel<BNT>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
+    attr_set[dev] = true;
+  }
+  salr_prefill_kernel<BNT><<<grid, kPreThreads, smem, st>>>(p, tx, tb, tt);
+  SALR_TRY(cudaGetLastError());
+  return SALR_OK;
+}
 
 // Persistent small-M path: one CTA per SM, launched so that it may overlap the preceding
 // kernel of the stream.
@@ -282,9 +347,13 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   // becomes compact-block entries, which set how many blocks are in flight from HBM
   p.sa = kStreamGroups + 1;
   const int fixed = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, 0, kStreamGroups);
+  // The compact-block slots come in a multiple of the group count, so that slot s only
+  // ever holds blocks of group s mod 4: a group never waits on a slot whose previous fill
+  // it has not consumed itself, and a parity wait can never pass on a phase two fills old.
   int sc = (kSmemLimit - fixed) / p.cbuf;
   if (sc > kStreamMaxC) sc = kStreamMaxC;
-  if (sc < kStreamGroups + 1) return SALR_ERR_UNSUPPORTED;
+  sc -= sc % kStreamGroups;
+  if (sc < kStreamGroups) return SALR_ERR_UNSUPPORTED;
   p.sc = sc;
   const int smem = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, p.sc, kStreamGroups);
   static bool attr_set[64] = {false};
@@ -361,7 +430,7 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
                 salr_handle* out) {
   if (!W || !out) return SALR_ERR_INVALID;
   if (!(sparsity >= 0.0f && sparsity < 1.0f)) return SALR_ERR_INVALID;
-  if (N < 128 || K < 64 || N % 128 || K % 64 || K > 64 * kMaxKBlocks) return SALR_ERR_UNSUPPORTED;
+  if (N < 128 || K < 64 || N % 128 || K % 64 || K > 64 * kPreMaxKBlocks) return SALR_ERR_UNSUPPORTED;
   if (N > (1ll << 22)) return SALR_ERR_UNSUPPORTED;
   if (!aligned16(W)) return SALR_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -501,42 +570,64 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     if (rc == SALR_OK) h->sscr.epoch = epoch;
     return rc;
   }
-  const Schedule sc = choose_schedule(M, h->N, h->K, device_sms(h->device));
-  LinParams p{};
-  p.blob = h->blob;
-  p.offsets = h->offsets;
-  p.Y = static_cast<uint16_t*>(Y);
-  p.status = h->status;
-  p.N = static_cast<int>(h->N);
-  p.K = static_cast<int>(h->K);
-  p.M = static_cast<int>(M);
-  p.R = static_cast<int>(R);
-  p.R16 = static_cast<int>((R + 15) / 16 * 16);
-  p.kblocks = static_cast<int>(h->K / 64);
-  p.TT = sc.tt;
-  p.splits = sc.splits;
-  if (sc.splits > 1) {
-    rc = ensure_workspace(h, static_cast<size_t>(sc.tt) * sc.bnt * h->N,
-                          static_cast<size_t>(h->N / 128) * sc.tt, st);
-    if (rc != SALR_OK) return rc;
-    p.ws = h->work.ws;
-    p.counters = h->work.counters;
-  }
-  CUtensorMap tx, ta, tb;
+  // prefill shapes: t = X A_cat once (own kernel), then the fused decode + GEMM
+  const int bnt = M <= 128 ? 128 : 256;
+  const int sms = device_sms(h->device);
+  const int TT = static_cast<int>((M + bnt - 1) / bnt);
+  const int RT = static_cast<int>(h->N / 128);
+  const int KB = static_cast<int>(h->K / 64);
+  if (KB > kPreMaxKBlocks) return SALR_ERR_UNSUPPORTED;
+  const int R16 = static_cast<int>((R + 15) / 16 * 16);
+  const int64_t Mp = (M + 3) / 4 * 4;  // row stride of the fp32 sums (16-byte rows)
+  CUtensorMap tx, ta, tb, tt;
   std::memset(&ta, 0, sizeof(ta));
   std::memset(&tb, 0, sizeof(tb));
-  if (!make_map(&tx, X, h->K, M, 64, sc.bnt)) return SALR_ERR_CUDA;
+  std::memset(&tt, 0, sizeof(tt));
+  if (!make_map(&tx, X, h->K, M, 64, bnt)) return SALR_ERR_CUDA;
   if (R > 0) {
+    rc = ensure_tscratch(h, M, st);
+    if (rc != SALR_OK) return rc;
     if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
-    if (!make_map(&tb, B_cat, h->N, R, 64, p.R16)) return SALR_ERR_CUDA;
+    if (!make_map(&tb, B_cat, h->N, R, 64, R16)) return SALR_ERR_CUDA;
+    if (!make_map(&tt, h->tscr.T, 128, M, 64, bnt)) return SALR_ERR_CUDA;
+    TParams tp{};
+    tp.T = h->tscr.T;
+    tp.T32 = h->tscr.T32;
+    tp.counters = h->tscr.counters;
+    tp.status = h->status;
+    tp.M = static_cast<int>(M);
+    tp.Mp = static_cast<int>(Mp);
+    tp.R16 = R16;
+    tp.kblocks = KB;
+    tp.TT = TT;
+    tp.splits = TT < sms ? std::min(KB, sms / TT) : 1;
+    rc = bnt == 128 ? launch_t<128>(tp, tx, ta, TT * tp.splits, st)
+                    : launch_t<256>(tp, tx, ta, TT * tp.splits, st);
+    if (rc != SALR_OK) return rc;
   }
-  const int grid = static_cast<int>((h->N / 128) * sc.tt * sc.splits);
-  switch (sc.bnt) {
-    case 16: return launch_linear<16>(p, tx, ta, tb, grid, st);
-    case 64: return launch_linear<64>(p, tx, ta, tb, grid, st);
-    case 128: return launch_linear<128>(p, tx, ta, tb, grid, st);
-    default: return launch_linear<256>(p, tx, ta, tb, grid, st);
+  PrefillParams pp{};
+  pp.blob = h->blob;
+  pp.offsets = h->offsets;
+  pp.Y = static_cast<uint16_t*>(Y);
+  pp.status = h->status;
+  pp.N = static_cast<int>(h->N);
+  pp.K = static_cast<int>(h->K);
+  pp.M = static_cast<int>(M);
+  pp.Mp = static_cast<int>(Mp);
+  pp.R16 = R > 0 ? R16 : 0;
+  pp.kblocks = KB;
+  pp.TT = TT;
+  pp.splits = RT * TT < sms ? std::min(KB, sms / (RT * TT)) : 1;
+  pp.cbuf = static_cast<int>((h->max16 * 16 + 32 + 1023) / 1024 * 1024);
+  if (pp.splits > 1) {
+    rc = ensure_workspace(h, static_cast<size_t>(h->N) * Mp, static_cast<size_t>(RT) * TT * 4, st);
+    if (rc != SALR_OK) return rc;
+    pp.acc = h->work.ws;
+    pp.counters = h->work.counters;
   }
+  const int grid = RT * TT * pp.splits;
+  return bnt == 128 ? launch_prefill<128>(pp, tx, tb, tt, grid, st)
+                    : launch_prefill<256>(pp, tx, tb, tt, grid, st);
 }
 
 int salr_linear_host(const void* X_host, int64_t M, salr_handle h, const void* A_cat,
@@ -609,6 +700,10 @@ int salr_sync_status(salr_handle h, void* stream) {
   if (h->work.ws) SALR_TRY(cudaMemset(h->work.ws, 0, h->work.ws_elems * sizeof(float)));
   if (h->work.counters)
     SALR_TRY(cudaMemset(h->work.counters, 0, h->work.n_counters * sizeof(uint32_t)));
+  if (h->tscr.T32) {
+    SALR_TRY(cudaMemset(h->tscr.T32, 0, static_cast<size_t>(h->tscr.rows) * 128 * sizeof(float)));
+    SALR_TRY(cudaMemset(h->tscr.counters, 0, static_cast<size_t>(h->tscr.rows / 128) * 4 * sizeof(uint32_t)));
+  }
   if (h->sscr.acc) {
     SALR_TRY(cudaMemset(h->sscr.acc, 0, static_cast<size_t>(h->N) * 64 * sizeof(float)));
     SALR_TRY(cudaMemset(h->sscr.counters, 0, static_cast<size_t>(h->N / 128) * 4 * sizeof(uint32_t)));
