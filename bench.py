@@ -3,10 +3,15 @@
 
 One step is one salr_linear call on the decode q_proj workload (W 4096 x 4096 bf16, 50%
 per-row magnitude pruned and bitmap-encoded, adapters 64 + 16 stacked to R = 80,
-X 16 x 4096).  Prints one JSON line (see --help).  Timing: W warm-up steps, then K steps
-queued behind a short GPU sleep so that host launch overhead does not leave gaps, each
-bracketed by CUDA events on the launching stream; the weight/adapter set rotates over
-enough copies that the working set exceeds L2 (no step finds its weights in L2).
+X 16 x 4096).  --workload/--tokens time another configuration of salr_synth.WORKLOADS the
+same way (the default is the headline line).  Prints one JSON line (see --help).
+
+Timing: W warm-up steps, then K steps queued back to back behind a short GPU sleep (so
+that host launch overhead leaves no gaps), with CUDA events on the launching stream at the
+two ends of the region; consecutive calls may overlap (programmatic dependent launch), as
+consecutive layers would.  A second pass puts an event pair around every call and reports
+their percentiles.  The weight/adapter set rotates over enough copies that the working set
+exceeds twice the L2 (no step finds its weights in L2).
 
 --impl reference times the fp64 CPU oracle on the same workload instead (one full layer
 per step on the host cores).  Under torchrun every rank runs an independent replica
@@ -147,7 +152,9 @@ def blas_threads():
 
 
 def time_oracle(wl, M, steps=None, budget_s=10.0):
-    step = oracle_step_fn(wl, M)
+    """Oracle steps in a bounded time; above 64 tokens each step is a fixed 64-token slice
+    of X (the work per token is the same, so tokens/s carries over)."""
+    step = oracle_step_fn(wl, min(M, 64))
     step()  # warm
     t0 = time.perf_counter()
     n = 0
@@ -165,21 +172,23 @@ def run_reference(args):
     if rank != 0:
         return
     wl = synth.WORKLOADS[WORKLOAD]
-    step = oracle_step_fn(wl, M_TOKENS)
+    step = oracle_step_fn(wl, min(M_TOKENS, 64))
     for _ in range(args.warmup):
         step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         step()
     el = time.perf_counter() - t0
-    value = args.steps * M_TOKENS / el
+    mo = min(M_TOKENS, 64)
+    value = args.steps * mo / el
     cores = blas_threads()
-    sample = f"full {WORKLOAD} layer (M={M_TOKENS}) per step, fp64 numpy oracle"
+    sample = f"full {WORKLOAD} layer (M={mo} of {M_TOKENS} tokens) per step, fp64 numpy oracle"
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD} N=4096 K=4096 R=80 M={M_TOKENS} s=0.5"},
+            "config": {"workload": f"{WORKLOAD} N={wl.N} K={wl.K} R={wl.R} M={M_TOKENS} "
+                                   f"sparsity={wl.sparsity}"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -200,8 +209,11 @@ def traffic_for(kname, workload):
 
 
 def main():
+    global WORKLOAD, M_TOKENS
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=M_TOKENS, help="M, tokens per call")
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["salr", "reference"], default="salr")
@@ -209,6 +221,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    WORKLOAD, M_TOKENS = args.workload, args.tokens
     if args.impl == "reference":
         return run_reference(args)
 
@@ -248,7 +261,8 @@ def main():
     # rotate over enough independent weight + adapter copies to exceed 2x L2
     first = salr.encode(W, wl.sparsity)
     per_copy = first.info()["bytes"] + 2 * R * (K + N)
-    ncopies = max(2, int(np.ceil(2 * L2_BYTES / per_copy)))
+    # (at most 64 copies: the smallest layers cannot outgrow L2 this way; the line says so)
+    ncopies = min(64, max(2, int(np.ceil(2 * L2_BYTES / per_copy))))
     handles = [first] + [salr.encode(W, wl.sparsity) for _ in range(ncopies - 1)]
     A = [dev(a_cat) for _ in range(ncopies)]
     B = [dev(b_cat) for _ in range(ncopies)]
@@ -267,7 +281,8 @@ def main():
         if rc:
             raise RuntimeError(salr.status_string(rc))
 
-    for i in range(args.warmup):
+    # every copy is used once before timing (a handle allocates its scratch on first use)
+    for i in range(max(args.warmup, ncopies)):
         launch(i)
     torch.cuda.synchronize()
     for h in handles[:1]:
@@ -314,7 +329,8 @@ def main():
     # ---------------- end to end: host activations in, host outputs back, per step
     xh = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
-    e2e_steps = args.steps
+    # bounded so that the host copies of a prefill-sized step stay within a few seconds
+    e2e_steps = max(3, min(args.steps, int(4e9 // (2 * M * (K + N)))))
 
     def launch_host(i):
         c = i % ncopies
@@ -358,7 +374,12 @@ def main():
         achieved = aflops / (kern_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
-    kname = "salr_stream_kernel<16,16>" if M <= 16 else "salr_linear_kernel"
+    if M <= 64:
+        kname = f"salr_stream_kernel<{16 if M <= 16 else 32 if M <= 32 else 64},16>"
+        launches_per_call = 1
+    else:
+        kname = f"salr_prefill_kernel<{128 if M <= 128 else 256}>"
+        launches_per_call = 2 if R > 0 else 1  # t = X A_cat kernel, then the layer
     roof["traffic"] = traffic_for(kname, WORKLOAD)
     roof["peak_source"] = peak_src
     roof["kernel"] = kname
@@ -371,15 +392,18 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD} N={N} K={K} R={R} (64+16) M={M} sparsity=0.5",
-                       "model": "SALR linear layer (decode q_proj shape)", "global_batch": M * ws,
+            "config": {"workload": f"{WORKLOAD} N={N} K={K} R={R} "
+                                   f"({'+'.join(str(r) for r in wl.ranks)}) M={M} "
+                                   f"sparsity={wl.sparsity}",
+                       "model": f"SALR linear layer ({WORKLOAD} shape)", "global_batch": M * ws,
                        "parallelism": f"replicas x{ws}",
                        "l2": f"rotating {ncopies} weight+adapter copies "
-                             f"({ncopies * per_copy / 2**20:.0f} MiB > 2x L2)"},
+                             f"({ncopies * per_copy / 2**20:.0f} MiB"
+                             f"{' > 2x L2' if ncopies * per_copy > 2 * L2_BYTES else ', smaller than L2'})"},
             "roofline": roof,
             "e2e": {"value": ws * e2e_steps * M / (e2e_ms * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * launches_per_call,
             "clocks": clocks.summary(),
             "per_launch_event_ms_p10_p50_p90": [float(np.percentile(per_launch_ms, q))
                                                 for q in (10, 50, 90)]}
