@@ -20,6 +20,7 @@ per step on the host cores).  Under torchrun every rank runs an independent repl
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -40,8 +41,17 @@ import salr_synth as synth  # noqa: E402
 METRIC = "SALR linear tokens/s + achieved fraction of HBM/tensor roofline on 1 B200"
 WORKLOAD = "q_proj"
 M_TOKENS = 16
+SPARSITY = None  # None: the workload's own (0.5)
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = ["sm100.cuh", "salr_codec.cuh", "salr_prefill.cuh", "salr_stream.cuh", "salr_api.cu"]
+
+
+def workload():
+    wl = synth.WORKLOADS[WORKLOAD]
+    if SPARSITY is None:
+        return wl
+    # the library takes sparsity as a float32: use that value everywhere
+    return dataclasses.replace(wl, sparsity=float(np.float32(SPARSITY)))
 
 
 def algorithmic_bytes(N, K, R, M, keep):
@@ -171,7 +181,7 @@ def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
         return
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = workload()
     step = oracle_step_fn(wl, min(M_TOKENS, 64))
     for _ in range(args.warmup):
         step()
@@ -188,11 +198,84 @@ def run_reference(args):
             "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{WORKLOAD} N={wl.N} K={wl.K} R={wl.R} M={M_TOKENS} "
-                                   f"sparsity={wl.sparsity}"},
+                                   f"sparsity={wl.sparsity:.6g}"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# Linear layers of one decoder layer of a Llama3-8B-shaped model (out x in) and the
+# model's other tensors, for the compressed-size report (the pages quote the model size
+# of Llama3-8B before and after compression).
+LLAMA3_8B_LINEARS = [("q_proj", 4096, 4096), ("k_proj", 1024, 4096), ("v_proj", 1024, 4096),
+                     ("o_proj", 4096, 4096), ("gate_proj", 14336, 4096),
+                     ("up_proj", 14336, 4096), ("down_proj", 4096, 14336)]
+LLAMA3_8B_LAYERS = 32
+LLAMA3_8B_OTHER_PARAMS = 2 * 128256 * 4096 + (2 * LLAMA3_8B_LAYERS + 1) * 4096  # emb, head, norms
+
+
+def run_encode_report(args):
+    """salr_encode throughput and the encoded size of every linear layer of a
+    Llama3-8B-shaped model (synthetic N(0, 0.02) weights drawn on the device)."""
+    import torch
+
+    from sparse_rank_linear_b200.build import build
+    import sparse_rank_linear_b200 as salr
+
+    build()
+    salr.load_library()
+    s = float(np.float32(0.5 if SPARSITY is None else SPARSITY))
+    peaks, peak_src = measured_peaks()
+    gen = torch.Generator(device="cuda")
+    rows, enc_bytes, dense_bytes = [], 0, 0
+    for name, N, K in LLAMA3_8B_LINEARS:
+        gen.manual_seed(N * 131 + K)
+        W = (torch.randn(N, K, generator=gen, device="cuda") * 0.02).to(torch.bfloat16)
+        salr.encode(W, s).free()  # warm
+        ms, wall = [], []
+        for _ in range(max(3, args.steps)):
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0 = time.perf_counter()
+            e0.record()
+            h = salr.encode(W, s)  # synchronous: returns with the weight encoded
+            e1.record()
+            torch.cuda.synchronize()
+            wall.append(time.perf_counter() - t0)
+            ms.append(e0.elapsed_time(e1))
+            info = h.info()
+            h.free()
+        keep = K - int(np.floor(s * K))
+        nb = (N // 128) * (K // 64)
+        # closed form of the format size, up to the 16-byte padding of each block
+        lo = N * K // 8 + 2 * N * keep + 4 * (nb + 1)
+        assert info["nnz"] == N * keep and lo <= info["bytes"] <= lo + 14 * nb, info
+        t = statistics.median(ms) * 1e-3
+        moved = 2 * N * K + info["bytes"]  # W read once, the format written once
+        rows.append({"layer": name, "N": N, "K": K, "encoded_bytes": info["bytes"],
+                     "dense_bytes": 2 * N * K, "ratio": 2 * N * K / info["bytes"],
+                     "encode_ms": t * 1e3, "encode_wall_ms": statistics.median(wall) * 1e3,
+                     "w_gbs": 2 * N * K / t / 1e9, "hbm_frac": moved / t / 1e9 / peaks["hbm_gbs"]})
+        enc_bytes += info["bytes"]
+        dense_bytes += 2 * N * K
+        del W
+    L = LLAMA3_8B_LAYERS
+    enc_t = sum(r["encode_ms"] for r in rows) * 1e-3
+    other = 2 * LLAMA3_8B_OTHER_PARAMS
+    line = {"metric": "SALR encode throughput (dense W bytes/s) and encoded size, "
+                      "Llama3-8B-shaped linear layers", "value": dense_bytes / enc_t / 1e9,
+            "unit": "GB/s", "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "sparsity": s, "steps": max(3, args.steps),
+            "model": {"linear_dense_bytes": L * dense_bytes, "linear_encoded_bytes": L * enc_bytes,
+                      "linear_ratio": dense_bytes / enc_bytes,
+                      "whole_dense_bytes": L * dense_bytes + other,
+                      "whole_encoded_bytes": L * enc_bytes + other,
+                      "whole_ratio": (L * dense_bytes + other) / (L * enc_bytes + other),
+                      "other_tensors": "embedding, lm_head and norms kept dense bf16",
+                      "encode_seconds": L * enc_t},
+            "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": peak_src, "layers": rows}
     print(json.dumps(line), flush=True)
 
 
@@ -209,21 +292,29 @@ def traffic_for(kname, workload):
 
 
 def main():
-    global WORKLOAD, M_TOKENS
+    global WORKLOAD, M_TOKENS, SPARSITY
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--tokens", type=int, default=M_TOKENS, help="M, tokens per call")
+    ap.add_argument("--sparsity", type=float, default=None,
+                    help="fraction of each row pruned (default: the workload's, 0.5)")
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["salr", "reference"], default="salr")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--encode-report", action="store_true",
+                    help="time salr_encode on Llama3-8B-shaped layers and report sizes")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    WORKLOAD, M_TOKENS = args.workload, args.tokens
+    WORKLOAD, M_TOKENS, SPARSITY = args.workload, args.tokens, args.sparsity
+    if SPARSITY is not None and not 0.0 <= SPARSITY < 1.0:
+        ap.error("--sparsity must lie in [0, 1)")
     if args.impl == "reference":
         return run_reference(args)
+    if args.encode_report:
+        return run_encode_report(args)
 
     import torch
     import torch.distributed as dist
@@ -242,7 +333,7 @@ def main():
         dist.barrier()
     lib = salr.load_library()
 
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = workload()
     N, K, R, M = wl.N, wl.K, wl.R, M_TOKENS
     keep = K - int(np.floor(wl.sparsity * K))
 
@@ -380,7 +471,8 @@ def main():
     else:
         kname = f"salr_prefill_kernel<{128 if M <= 128 else 256}>"
         launches_per_call = 2 if R > 0 else 1  # t = X A_cat kernel, then the layer
-    roof["traffic"] = traffic_for(kname, WORKLOAD)
+    roof["traffic"] = traffic_for(kname, WORKLOAD if wl.sparsity == 0.5
+                                  else f"{WORKLOAD} s={wl.sparsity:.6g}")
     roof["peak_source"] = peak_src
     roof["kernel"] = kname
     roof["kernel_ms"] = kern_ms
@@ -394,7 +486,7 @@ def main():
             "data": "synthetic",
             "config": {"workload": f"{WORKLOAD} N={N} K={K} R={R} "
                                    f"({'+'.join(str(r) for r in wl.ranks)}) M={M} "
-                                   f"sparsity={wl.sparsity}",
+                                   f"sparsity={wl.sparsity:.6g}",
                        "model": f"SALR linear layer ({WORKLOAD} shape)", "global_batch": M * ws,
                        "parallelism": f"replicas x{ws}",
                        "l2": f"rotating {ncopies} weight+adapter copies "

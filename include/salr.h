@@ -174,6 +174,60 @@ SALR_API int salr_info(salr_handle h, int64_t* N, int64_t* K, int64_t* nnz, int6
 SALR_API int salr_format_view(salr_handle h, const void** blob, int64_t* blob_bytes,
                      const void** offsets, int64_t* n_offsets);
 
+/*
+ * Serialised image: the byte form of an encoded weight, for storing the compressed model
+ * (technical summary, Methodology 4: bitmap encoding is what makes the size reduction
+ * real, and Experimental Results: model size halved).  The image is the encoded format
+ * above behind a fixed header; all fields little-endian:
+ *
+ *   bytes [0, 64)   header
+ *                     0  char[8] "SALRBLK1"       32  int64 keep (entries kept per row)
+ *                     8  uint32 version = 1       40  int64 nnz = N * keep
+ *                    12  uint32 header size = 64  48  float32 sparsity
+ *                    16  int64 N                  52  uint32 0
+ *                    24  int64 K                  56  int64 blob bytes (multiple of 16)
+ *   then            offset table, (N/128)(K/64) + 1 uint32, zero bytes up to a multiple
+ *                   of 16
+ *   then            the blob, byte for byte
+ *
+ * The image holds no device addresses and no state of earlier calls: any GPU can load
+ * it.  It carries no checksum; salr_load checks its structure instead (below).
+ */
+
+/* salr_save_size - size in bytes of the image salr_save writes for `h`. */
+SALR_API int salr_save_size(salr_handle h, int64_t* bytes);
+
+/*
+ * salr_save - write the image of `h` to host memory.
+ *
+ * buf       host memory (page-locked or pageable), at least salr_save_size bytes; only
+ *           the first salr_save_size bytes are written.
+ * stream    the copies of the offset table and the blob are queued on it after work
+ *           already queued there (so after the salr_encode that made `h`), and the call
+ *           returns once they are complete.
+ * Returns SALR_ERR_INVALID for an unknown handle, a NULL buf or buf_bytes too small
+ * (nothing is written then).
+ */
+SALR_API int salr_save(salr_handle h, void* buf, int64_t buf_bytes, void* stream);
+
+/*
+ * salr_load - make a new handle on the current device from an image in host memory.
+ *
+ * buf       host memory holding an image; bytes past the image's end are ignored.
+ * out       receives the new handle on SALR_OK (unchanged otherwise).  The handle is the
+ *           one salr_encode gave for the same weight: salr_decode, salr_linear and the
+ *           rest behave the same way on it.
+ *
+ * Checks before anything is used: the header (magic, version, N and K under the shape
+ * rules, keep = K - floor(sparsity * K), nnz = N * keep), the offset table on the host
+ * (starts at 0, each block at least its 1 KB bitmap and at most a dense block, ends at
+ * the blob size), then on the device every block (its bitmap's population matches its
+ * size, no kept value is NaN, padding is zero) and every row (exactly `keep` bits set).
+ * A failed check returns SALR_ERR_INVALID (SALR_ERR_UNSUPPORTED for a shape outside the
+ * rules) and frees everything the call allocated.  Synchronises `stream`.
+ */
+SALR_API int salr_load(const void* buf, int64_t buf_bytes, void* stream, salr_handle* out);
+
 /* salr_sync_status - synchronise `stream`, return the first device-side error recorded
  * for this handle since the last call (SALR_OK if none) and clear it. */
 SALR_API int salr_sync_status(salr_handle h, void* stream);

@@ -32,6 +32,9 @@ SIGNATURES = {
                        ctypes.POINTER(_I64)]),
     "salr_format_view": (_I, [_P, ctypes.POINTER(_P), ctypes.POINTER(_I64), ctypes.POINTER(_P),
                               ctypes.POINTER(_I64)]),
+    "salr_save_size": (_I, [_P, ctypes.POINTER(_I64)]),
+    "salr_save": (_I, [_P, _P, _I64, _P]),
+    "salr_load": (_I, [_P, _I64, _P, ctypes.POINTER(_P)]),
     "salr_sync_status": (_I, [_P, _P]),
     "salr_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -133,6 +136,16 @@ class Weight:
         _check("salr_decode", load_library().salr_decode(self.handle, _ptr(out), _stream_ptr(stream)))
         return out
 
+    def to_bytes(self, stream=None) -> bytes:
+        """salr_save: the serialised image of this weight (layout in include/salr.h)."""
+        lib = load_library()
+        n = _I64()
+        _check("salr_save_size", lib.salr_save_size(self.handle, ctypes.byref(n)))
+        buf = ctypes.create_string_buffer(n.value)
+        _check("salr_save", lib.salr_save(self.handle, ctypes.cast(buf, _P), n.value,
+                                          _stream_ptr(stream)))
+        return buf.raw
+
     def sync_status(self, stream=None) -> int:
         return load_library().salr_sync_status(self.handle, _stream_ptr(stream))
 
@@ -170,6 +183,16 @@ def encode(W, sparsity: float = 0.5, stream=None) -> Weight:
     h = _P()
     _check("salr_encode", load_library().salr_encode(_ptr(W), N, K, float(sparsity),
                                                      _stream_ptr(stream), ctypes.byref(h)))
+    return Weight(h)
+
+
+def load(image: bytes, stream=None) -> Weight:
+    """salr_load: a weight on the current CUDA device from a serialised image."""
+    data = bytes(image)
+    h = _P()
+    _check("salr_load", load_library().salr_load(ctypes.cast(ctypes.c_char_p(data), _P),
+                                                 len(data), _stream_ptr(stream),
+                                                 ctypes.byref(h)))
     return Weight(h)
 
 

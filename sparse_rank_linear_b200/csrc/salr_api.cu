@@ -62,6 +62,7 @@ struct salr_weight_s {
   int device;
   int64_t N, K, keep, nnz;
   float sparsity;
+  uint8_t* mem;  // one device allocation: [status][offsets][blob]
   uint8_t* blob;
   int64_t blob_bytes;
   uint32_t* offsets;
@@ -113,6 +114,25 @@ cudaError_t dev_alloc(void** p, size_t bytes) {
   return cudaMalloc(p, bytes);
 }
 
+// Stream-ordered scratch (freed with cudaFreeAsync on the same stream).
+cudaError_t dev_alloc_async(void** p, size_t bytes, cudaStream_t st) {
+  if (fake_oom()) return cudaErrorMemoryAllocation;
+  return cudaMallocAsync(p, bytes, st);
+}
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+// The handle's device memory, [status word][offset table][blob], in one allocation.
+cudaError_t alloc_handle_memory(salr_weight_s* h, int64_t blob_capacity) {
+  const size_t offs = round256((h->nblocks + 1) * sizeof(uint32_t));
+  const cudaError_t e = dev_alloc(reinterpret_cast<void**>(&h->mem), 256 + offs + blob_capacity);
+  if (e != cudaSuccess) return e;
+  h->status = reinterpret_cast<int*>(h->mem);
+  h->offsets = reinterpret_cast<uint32_t*>(h->mem + 256);
+  h->blob = h->mem + 256 + offs;
+  return cudaSuccess;
+}
+
 int device_sms(int dev) {
   static int cache[64] = {0};
   if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
@@ -155,9 +175,7 @@ void release(salr_weight_s* h) {
   cudaFree(h->sscr.counters);
   cudaFree(h->sscr.tacc);
   cudaFree(h->sscr.tflags);
-  cudaFree(h->blob);
-  cudaFree(h->offsets);
-  cudaFree(h->status);
+  cudaFree(h->mem);
   cudaFree(h->work.ws);
   cudaFree(h->work.counters);
   cudaFree(h->tscr.T);
@@ -259,14 +277,21 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   // blocks.  The compact-block slots come in a multiple of the group count, so that slot
   // s only ever holds blocks of group s mod 4: a group then never waits on a slot whose
   // previous fill it has not consumed itself, and a parity wait can never pass on a phase
-  // two fills old.
-  p.sa = kPreGroups + 1;
-  int sx = kPreMaxX, sc = 0;
-  for (; sx >= 2; --sx) {
-    sc = (kSmemLimit - L::smem_bytes(p.sa, sx, 0, p.cbuf)) / p.cbuf;
-    if (sc >= kPreGroups) break;
+  // two fills old.  Large blocks (little or no pruning) may not leave room for that: then
+  // one decoded-tile slot per group.  That ring is safe for any count of at least the
+  // group count: a group's wait for the consumption of block it - SA follows its own
+  // earlier wait, at block it - 4, which saw block it - 4 - SA >= it - 2 SA consumed (the
+  // MMA consumes in order), so the slot can never be two phases behind.
+  int sa = kPreGroups + 1, sx = kPreMaxX, sc = 0;
+  for (; sa >= kPreGroups; --sa) {
+    for (sx = kPreMaxX; sx >= 2; --sx) {
+      sc = (kSmemLimit - L::smem_bytes(sa, sx, 0, p.cbuf)) / p.cbuf;
+      if (sc >= kPreGroups) break;
+    }
+    if (sx >= 2 && sc >= kPreGroups) break;
   }
-  if (sx < 2 || sc < kPreGroups) return SALR_ERR_UNSUPPORTED;
+  if (sa < kPreGroups || sx < 2 || sc < kPreGroups) return SALR_ERR_UNSUPPORTED;
+  p.sa = sa;
   if (sc > kPreMaxC) sc = kPreMaxC;
   sc -= sc % kPreGroups;
   p.sx = sx;
@@ -412,6 +437,47 @@ int check_linear_args(const void* X, int64_t M, salr_handle h, const void* A, co
 
 int noalloc_reset(int dev);  // defined with salr_linear_noalloc below
 
+namespace {
+
+constexpr char kImageMagic[8] = {'S', 'A', 'L', 'R', 'B', 'L', 'K', '1'};
+constexpr uint32_t kImageVersion = 1;
+constexpr int64_t kImageHeader = 64;
+
+struct ImageHeader {
+  char magic[8];
+  uint32_t version;
+  uint32_t header_bytes;
+  int64_t N, K, keep, nnz;
+  float sparsity;
+  uint32_t zero;
+  int64_t blob_bytes;
+};
+static_assert(sizeof(ImageHeader) == kImageHeader, "image header is 64 bytes");
+
+int64_t image_offsets_bytes(int64_t nblocks) { return ((nblocks + 1) * 4 + 15) / 16 * 16; }
+
+int64_t keep_for(int64_t K, float sparsity) {
+  return K - static_cast<int64_t>(std::floor(static_cast<double>(sparsity) * K));
+}
+
+// the shape rules salr_encode applies, shared by salr_load
+int check_shape(int64_t N, int64_t K) {
+  if (N < 128 || K < 64 || N % 128 || K % 64 || K > 64 * kPreMaxKBlocks) return SALR_ERR_UNSUPPORTED;
+  if (N > (1ll << 22)) return SALR_ERR_UNSUPPORTED;
+  return SALR_OK;
+}
+
+void publish(salr_weight_s* h, salr_handle* out) {
+  h->magic = kMagic;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    live().insert(h);
+  }
+  *out = h;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* salr_status_string(int status) {
@@ -430,13 +496,19 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
                 salr_handle* out) {
   if (!W || !out) return SALR_ERR_INVALID;
   if (!(sparsity >= 0.0f && sparsity < 1.0f)) return SALR_ERR_INVALID;
-  if (N < 128 || K < 64 || N % 128 || K % 64 || K > 64 * kPreMaxKBlocks) return SALR_ERR_UNSUPPORTED;
-  if (N > (1ll << 22)) return SALR_ERR_UNSUPPORTED;
+  const int shape = check_shape(N, K);
+  if (shape != SALR_OK) return shape;
   if (!aligned16(W)) return SALR_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t keep = K - static_cast<int64_t>(std::floor(static_cast<double>(sparsity) * K));
+  const int64_t keep = keep_for(K, sparsity);
   const int64_t nwords = K / 64;
   const int64_t nblocks = (N / 128) * nwords;
+
+  // The blob is written straight into the handle: its capacity is the largest size the
+  // kept count allows (each block pads its values by at most 14 bytes), so the encoder
+  // needs no size round trip to the host before writing it.
+  const int64_t capacity = (kBitmapBytes + 16) * nblocks + 2 * N * keep;
+  if (capacity / 16 >= (1ll << 32)) return SALR_ERR_UNSUPPORTED;  // offsets are uint32 x 16 B
 
   salr_weight_s* h = new (std::nothrow) salr_weight_s();
   if (!h) return SALR_ERR_OOM;
@@ -448,39 +520,50 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
   h->sparsity = sparsity;
   h->nblocks = nblocks;
 
-  uint64_t* bits = nullptr;
-  uint32_t* size16 = nullptr;
-  unsigned long long* nnz_d = nullptr;  // [0] kept entries, [1] largest block (16 B units)
+  // scratch: the row-major bitmap, block sizes, and [kept entries, largest block]
+  uint8_t* scratch = nullptr;
+  const size_t bits_bytes = round256(N * nwords * sizeof(uint64_t));
+  const size_t size_bytes = round256(nblocks * sizeof(uint32_t));
   auto fail = [&](int code) {
+    if (scratch) cudaFreeAsync(scratch, st);
     cudaStreamSynchronize(st);
-    cudaFree(bits);
-    cudaFree(size16);
-    cudaFree(nnz_d);
     release(h);
     return code;
   };
   cudaError_t e;
-  if ((e = dev_alloc(reinterpret_cast<void**>(&h->status), sizeof(int))) != cudaSuccess ||
-      (e = dev_alloc(reinterpret_cast<void**>(&h->offsets), (nblocks + 1) * sizeof(uint32_t))) !=
-          cudaSuccess ||
-      (e = dev_alloc(reinterpret_cast<void**>(&bits), N * nwords * sizeof(uint64_t))) !=
-          cudaSuccess ||
-      (e = dev_alloc(reinterpret_cast<void**>(&size16), nblocks * sizeof(uint32_t))) !=
-          cudaSuccess ||
-      (e = dev_alloc(reinterpret_cast<void**>(&nnz_d), 2 * sizeof(unsigned long long))) !=
-          cudaSuccess)
+  if ((e = alloc_handle_memory(h, capacity)) != cudaSuccess ||
+      (e = dev_alloc_async(reinterpret_cast<void**>(&scratch), bits_bytes + size_bytes + 256,
+                           st)) != cudaSuccess)
     return fail(cuda_status(e));
+  uint64_t* bits = reinterpret_cast<uint64_t*>(scratch);
+  uint32_t* size16 = reinterpret_cast<uint32_t*>(scratch + bits_bytes);
+  unsigned long long* nnz_d = reinterpret_cast<unsigned long long*>(scratch + bits_bytes + size_bytes);
   if ((e = cudaMemsetAsync(h->status, 0, sizeof(int), st)) != cudaSuccess ||
       (e = cudaMemsetAsync(nnz_d, 0, 2 * sizeof(unsigned long long), st)) != cudaSuccess)
     return fail(cuda_status(e));
 
-  encode_mask_kernel<<<static_cast<unsigned>(N), kEncThreads, K * sizeof(uint16_t), st>>>(
+  const int mask_smem = static_cast<int>(K * sizeof(uint16_t));
+  if (mask_smem > 48 * 1024) {
+    static bool attr_set[64] = {false};
+    if (h->device < 0 || h->device >= 64) return fail(SALR_ERR_UNSUPPORTED);
+    if (!attr_set[h->device]) {
+      if ((e = cudaFuncSetAttribute(encode_mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    mask_smem)) != cudaSuccess)
+        return fail(cuda_status(e));
+      attr_set[h->device] = true;
+    }
+  }
+  encode_mask_kernel<<<static_cast<unsigned>(N), kEncThreads, mask_smem, st>>>(
       static_cast<const uint16_t*>(W), static_cast<int>(K), static_cast<int>(keep), bits,
       h->status);
   encode_count_kernel<<<static_cast<unsigned>((nblocks + 7) / 8), 256, 0, st>>>(
       bits, static_cast<int>(nwords), static_cast<int>(nblocks), size16, nnz_d,
       reinterpret_cast<unsigned int*>(nnz_d + 1));
-  encode_scan_kernel<<<1, 1024, 0, st>>>(size16, static_cast<int>(nblocks), h->offsets, h->status);
+  const unsigned long long cap16 = static_cast<unsigned long long>(capacity / 16);
+  encode_scan_kernel<<<1, 1024, 0, st>>>(size16, static_cast<int>(nblocks), cap16, h->offsets,
+                                         h->status);
+  encode_scatter_kernel<<<static_cast<unsigned>(nblocks), kBlockRows, 0, st>>>(
+      static_cast<const uint16_t*>(W), static_cast<int>(K), bits, h->offsets, cap16, h->blob);
   if ((e = cudaGetLastError()) != cudaSuccess) return fail(cuda_status(e));
 
   uint32_t total16 = 0;
@@ -492,29 +575,17 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
           cudaSuccess ||
       (e = cudaMemcpyAsync(nnz, nnz_d, 2 * sizeof(unsigned long long), cudaMemcpyDeviceToHost,
                            st)) != cudaSuccess ||
-      (e = cudaStreamSynchronize(st)) != cudaSuccess)
+      (e = cudaFreeAsync(scratch, st)) != cudaSuccess)
     return fail(cuda_status(e));
+  scratch = nullptr;
+  if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return fail(cuda_status(e));
   if (status & DEV_ERR_NAN) return fail(SALR_ERR_INVALID);
   if (status & DEV_ERR_RANGE) return fail(SALR_ERR_UNSUPPORTED);
 
   h->nnz = static_cast<int64_t>(nnz[0]);
   h->max16 = static_cast<uint32_t>(nnz[1]);
   h->blob_bytes = static_cast<int64_t>(total16) * 16;
-  if ((e = dev_alloc(reinterpret_cast<void**>(&h->blob), h->blob_bytes)) != cudaSuccess)
-    return fail(cuda_status(e));
-  encode_scatter_kernel<<<static_cast<unsigned>(nblocks), kBlockRows, 0, st>>>(
-      static_cast<const uint16_t*>(W), static_cast<int>(K), bits, h->offsets, h->blob);
-  if ((e = cudaGetLastError()) != cudaSuccess || (e = cudaStreamSynchronize(st)) != cudaSuccess)
-    return fail(cuda_status(e));
-  cudaFree(bits);
-  cudaFree(size16);
-  cudaFree(nnz_d);
-  h->magic = kMagic;
-  {
-    std::lock_guard<std::mutex> g(g_mu);
-    live().insert(h);
-  }
-  *out = h;
+  publish(h, out);
   return SALR_OK;
 }
 
@@ -685,6 +756,141 @@ int salr_format_view(salr_handle h, const void** blob, int64_t* blob_bytes, cons
   if (blob_bytes) *blob_bytes = h->blob_bytes;
   if (offsets) *offsets = h->offsets;
   if (n_offsets) *n_offsets = h->nblocks + 1;
+  return SALR_OK;
+}
+
+// ------------------------------------------------------------------------------------
+// Serialised image of a handle: the byte form of the compressed weight.  Layout (all
+// little-endian; include/salr.h documents it for readers of the files):
+//   [0,64)   header: "SALRBLK1", u32 version 1, u32 header bytes 64, i64 N, i64 K,
+//            i64 keep, i64 nnz, f32 sparsity, u32 0, i64 blob bytes
+//   [64,..)  offset table, (nblocks + 1) x u32, zero padded to a multiple of 16 bytes
+//   then     the blob (bitmaps, kept values, zero padding), exactly as on the device
+// ------------------------------------------------------------------------------------
+int salr_save_size(salr_handle h, int64_t* bytes) {
+  if (!valid_handle(h) || !bytes) return SALR_ERR_INVALID;
+  *bytes = kImageHeader + image_offsets_bytes(h->nblocks) + h->blob_bytes;
+  return SALR_OK;
+}
+
+int salr_save(salr_handle h, void* buf, int64_t buf_bytes, void* stream) {
+  int64_t need = 0;
+  if (salr_save_size(h, &need) != SALR_OK || !buf) return SALR_ERR_INVALID;
+  if (buf_bytes < need) return SALR_ERR_INVALID;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* out = static_cast<uint8_t*>(buf);
+  ImageHeader hd;
+  std::memset(&hd, 0, sizeof(hd));
+  std::memcpy(hd.magic, kImageMagic, sizeof(hd.magic));
+  hd.version = kImageVersion;
+  hd.header_bytes = static_cast<uint32_t>(kImageHeader);
+  hd.N = h->N;
+  hd.K = h->K;
+  hd.keep = h->keep;
+  hd.nnz = h->nnz;
+  hd.sparsity = h->sparsity;
+  hd.blob_bytes = h->blob_bytes;
+  std::memcpy(out, &hd, sizeof(hd));
+  const int64_t ob = image_offsets_bytes(h->nblocks);
+  const int64_t used = (h->nblocks + 1) * 4;
+  std::memset(out + kImageHeader + used, 0, ob - used);
+  SALR_TRY(cudaMemcpyAsync(out + kImageHeader, h->offsets, used, cudaMemcpyDeviceToHost, st));
+  SALR_TRY(cudaMemcpyAsync(out + kImageHeader + ob, h->blob, h->blob_bytes,
+                           cudaMemcpyDeviceToHost, st));
+  SALR_TRY(cudaStreamSynchronize(st));
+  return SALR_OK;
+}
+
+int salr_load(const void* buf, int64_t buf_bytes, void* stream, salr_handle* out) {
+  if (!buf || !out || buf_bytes < kImageHeader) return SALR_ERR_INVALID;
+  const uint8_t* in = static_cast<const uint8_t*>(buf);
+  ImageHeader hd;
+  std::memcpy(&hd, in, sizeof(hd));
+  if (std::memcmp(hd.magic, kImageMagic, sizeof(hd.magic)) != 0 || hd.version != kImageVersion ||
+      hd.header_bytes != kImageHeader || hd.zero != 0)
+    return SALR_ERR_INVALID;
+  if (!(hd.sparsity >= 0.0f && hd.sparsity < 1.0f)) return SALR_ERR_INVALID;
+  const int shape = check_shape(hd.N, hd.K);
+  if (shape != SALR_OK) return shape;
+  if (hd.keep != keep_for(hd.K, hd.sparsity) || hd.nnz != hd.N * hd.keep) return SALR_ERR_INVALID;
+  const int64_t nwords = hd.K / 64;
+  const int64_t nblocks = (hd.N / 128) * nwords;
+  const int64_t ob = image_offsets_bytes(nblocks);
+  if (hd.blob_bytes < 0 || hd.blob_bytes % 16 ||
+      hd.blob_bytes > (buf_bytes - kImageHeader - ob))
+    return SALR_ERR_INVALID;
+  // offsets: from 0, each block at least its bitmap and at most a dense block, ending at
+  // the blob's end.  These bounds keep every device read of the checks below in range.
+  const uint8_t* offs_in = in + kImageHeader;
+  constexpr uint32_t kMin16 = kBitmapBytes / 16;
+  constexpr uint32_t kMax16 = (kBitmapBytes + 2 * kBlockRows * kBlockCols) / 16;
+  uint32_t prev = 0, max16 = 0;
+  std::memcpy(&prev, offs_in, 4);
+  if (prev != 0) return SALR_ERR_INVALID;
+  for (int64_t b = 1; b <= nblocks; ++b) {
+    uint32_t cur;
+    std::memcpy(&cur, offs_in + 4 * b, 4);
+    if (cur < prev || cur - prev < kMin16 || cur - prev > kMax16) return SALR_ERR_INVALID;
+    max16 = std::max(max16, cur - prev);
+    prev = cur;
+  }
+  if (static_cast<int64_t>(prev) * 16 != hd.blob_bytes) return SALR_ERR_INVALID;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  salr_weight_s* h = new (std::nothrow) salr_weight_s();
+  if (!h) return SALR_ERR_OOM;
+  std::memset(h, 0, sizeof(*h));
+  cudaGetDevice(&h->device);
+  h->N = hd.N;
+  h->K = hd.K;
+  h->keep = hd.keep;
+  h->sparsity = hd.sparsity;
+  h->nblocks = nblocks;
+  h->max16 = max16;
+  h->blob_bytes = hd.blob_bytes;
+  uint32_t* row_keep = nullptr;
+  unsigned long long* nnz_d = nullptr;
+  auto fail = [&](int code) {
+    cudaStreamSynchronize(st);
+    cudaFree(row_keep);
+    cudaFree(nnz_d);
+    release(h);
+    return code;
+  };
+  cudaError_t e;
+  if ((e = alloc_handle_memory(h, h->blob_bytes)) != cudaSuccess ||
+      (e = dev_alloc(reinterpret_cast<void**>(&row_keep), hd.N * sizeof(uint32_t))) !=
+          cudaSuccess ||
+      (e = dev_alloc(reinterpret_cast<void**>(&nnz_d), sizeof(unsigned long long))) !=
+          cudaSuccess)
+    return fail(cuda_status(e));
+  if ((e = cudaMemsetAsync(h->status, 0, sizeof(int), st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(row_keep, 0, hd.N * sizeof(uint32_t), st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(nnz_d, 0, sizeof(unsigned long long), st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(h->offsets, offs_in, (nblocks + 1) * sizeof(uint32_t),
+                           cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(h->blob, in + kImageHeader + ob, h->blob_bytes,
+                           cudaMemcpyHostToDevice, st)) != cudaSuccess)
+    return fail(cuda_status(e));
+  load_check_blocks_kernel<<<static_cast<unsigned>((nblocks + 7) / 8), 256, 0, st>>>(
+      h->blob, h->offsets, static_cast<int>(nwords), static_cast<int>(nblocks), row_keep, nnz_d,
+      h->status);
+  load_check_rows_kernel<<<static_cast<unsigned>((hd.N + 255) / 256), 256, 0, st>>>(
+      row_keep, static_cast<int>(hd.N), static_cast<uint32_t>(hd.keep), h->status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return fail(cuda_status(e));
+  int status = 0;
+  unsigned long long nnz = 0;
+  if ((e = cudaMemcpyAsync(&status, h->status, sizeof(int), cudaMemcpyDeviceToHost, st)) !=
+          cudaSuccess ||
+      (e = cudaMemcpyAsync(&nnz, nnz_d, sizeof(nnz), cudaMemcpyDeviceToHost, st)) !=
+          cudaSuccess ||
+      (e = cudaStreamSynchronize(st)) != cudaSuccess)
+    return fail(cuda_status(e));
+  if (status != 0 || static_cast<int64_t>(nnz) != hd.nnz) return fail(SALR_ERR_INVALID);
+  h->nnz = hd.nnz;
+  cudaFree(row_keep);
+  cudaFree(nnz_d);
+  publish(h, out);
   return SALR_OK;
 }
 

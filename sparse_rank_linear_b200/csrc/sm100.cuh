@@ -8,7 +8,7 @@
 namespace salr {
 
 // Status bits a kernel may record in the handle's device status word.
-enum : int { DEV_ERR_NAN = 1, DEV_ERR_TIMEOUT = 2, DEV_ERR_RANGE = 4 };
+enum : int { DEV_ERR_NAN = 1, DEV_ERR_TIMEOUT = 2, DEV_ERR_RANGE = 4, DEV_ERR_FORMAT = 8 };
 
 // Upper bound on how long any single wait may spin, in SM clock cycles (~1 s at the
 // B200's 1.9 GHz boost clock).  A correct pipeline never comes near it.

@@ -6,6 +6,7 @@ import re
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 from sparse_rank_linear_b200 import binding
@@ -72,6 +73,9 @@ def test_bad_arguments_rejected_on_host(lib):
         assert lib.salr_info(bad, None, None, None, None) == 1
         assert lib.salr_format_view(bad, None, None, None, None) == 1
         assert lib.salr_sync_status(bad, P(0)) == 1
+        n = ctypes.c_int64()
+        assert lib.salr_save_size(bad, ctypes.byref(n)) == 1
+        assert lib.salr_save(bad, fake, 1 << 20, P(0)) == 1
 
 
 def test_fake_oom_reported(lib):
@@ -94,3 +98,54 @@ def test_missing_library_fails_loudly(tmp_path):
             binding.load_library(str(tmp_path / "absent.so"))
     finally:
         binding._lib = saved
+
+
+def test_load_rejects_bad_images_on_host(lib):
+    # every image below fails a check made on the host before any CUDA call
+    import image_util as iu
+    import salr_synth as synth
+    P = ctypes.c_void_p
+    w = synth.weight(synth.WORKLOADS["tiny"])
+    good = iu.image(w, 0.5)
+    f, offs, blob = iu.split(good)
+    n, k, keep, nnz, s = f[3], f[4], f[5], f[6], f[7]
+
+    def load(img):
+        h = P()
+        buf = ctypes.create_string_buffer(img, len(img))
+        rc = lib.salr_load(ctypes.cast(buf, P), len(img), P(0), ctypes.byref(h))
+        assert h.value is None
+        return rc
+
+    def pk(**kw):
+        a = dict(n=n, k=k, keep=keep, nnz=nnz, sparsity=s, offs=offs, blob=blob)
+        a.update(kw)
+        return iu.pack(**a)
+
+    o = offs.astype(np.int64)
+    bad = {
+        "short": good[:63],
+        "magic": pk(magic=b"SALRBLK2"),
+        "version": pk(version=2),
+        "header size": pk(header_bytes=72),
+        "reserved word": pk(zero=1),
+        "keep": pk(keep=keep + 1, nnz=n * (keep + 1)),
+        "nnz": pk(nnz=nnz - 1),
+        "sparsity nan": pk(sparsity=float("nan")),
+        "sparsity one": pk(sparsity=1.0),
+        "first offset": pk(offs=np.concatenate([[1], o[1:]])),
+        "block under a bitmap": pk(offs=np.concatenate([[0, 63], o[2:]])),
+        "block over a dense block": pk(offs=np.concatenate([[0], o[1:] + 1025])),
+        "offsets fall": pk(offs=np.concatenate([[0, o[2], o[1]], o[3:]])),
+        "end short of the blob": pk(blob=np.concatenate([blob, np.zeros(16, np.uint8)])),
+        "truncated": good[:-1],
+    }
+    for name, img in bad.items():
+        assert load(img) == 1, name
+    # the blob size field must be a multiple of 16 and fit the buffer
+    odd = bytearray(good)
+    odd[56:64] = (len(blob) + 8).to_bytes(8, "little")
+    assert load(bytes(odd)) == 1
+    # shapes outside the rules are unsupported, as for salr_encode
+    assert load(pk(n=100)) == 2
+    assert load(pk(k=96)) == 2

@@ -134,6 +134,25 @@ def test_encode_other_sparsities(s):
     h.free()
 
 
+def test_encode_widest_rows():
+    # K = 32768, the largest the format allows: the row's keys need 64 KB of shared memory
+    wl = synth.Workload("wide", 256, 32768, (8,), (4,))
+    w = synth.weight(wl)
+    m = oracle.magnitude_mask(w, 0.5)
+    wp = oracle.prune(w, m)
+    h = salr.encode(to_dev(w), 0.5)
+    assert (to_bits(h.decode()) == wp).all()
+    o, b = oracle.encode_format(wp, m)
+    gb, go = h.format_tensors()
+    assert (go.cpu().numpy().view(np.uint32) == o).all() and (gb.cpu().numpy() == b).all()
+    x = synth.activations(wl, 4)
+    ad = synth.adapters(wl)
+    Y = salr.linear(to_dev(x), h, to_dev(ad[0][0]), to_dev(ad[0][1]))
+    assert h.sync_status() == 0
+    assert_close(to_bits(Y), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad), "K=32768")
+    h.free()
+
+
 def test_encode_rejects_nan():
     w = synth.weight(synth.Workload("t", 128, 64, (8,), (1,))).copy()
     w[77, 5] = 0x7FC1
@@ -241,6 +260,40 @@ def test_sparsity_zero_is_dense_gemm():
     h.free()
 
 
+@pytest.mark.parametrize("s", [0.0, 0.3, 0.75])
+@pytest.mark.parametrize("M", [16, 300])
+def test_linear_other_sparsities(s, M):
+    # the block sizes follow s (17 KB for a dense block, about 5 KB at s = 0.75): both
+    # kernels size their compact-block ring slots from the handle's largest block
+    wl = synth.Workload("t", 640, 1152, (64, 16), (M,))
+    w, x = synth.weight(wl), synth.activations(wl, M)
+    ad = synth.adapters(wl)
+    acat = np.concatenate([a for a, _ in ad], axis=1)
+    bcat = np.concatenate([b for _, b in ad], axis=0)
+    s32 = float(np.float32(s))
+    h = salr.encode(to_dev(w), s)
+    Y = salr.linear(to_dev(x), h, to_dev(acat), to_dev(bcat))
+    assert h.sync_status() == 0
+    wp = oracle.prune(w, oracle.magnitude_mask(w, s32))
+    assert_close(to_bits(Y), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad),
+                 f"s={s} M={M}")
+    h.free()
+
+
+def test_linear_q_proj_sparsity_0p3_full_compare():
+    wl = synth.WORKLOADS["q_proj"]
+    w, x = weight("q_proj"), synth.activations(wl, 16)
+    ad, A, B = adapters_dev("q_proj")
+    s32 = float(np.float32(0.3))
+    h = salr.encode(to_dev(w), 0.3)
+    assert h.info()["nnz"] == wl.N * oracle.keep_count(wl.K, s32)
+    Y = salr.linear(to_dev(x), h, A, B)
+    assert h.sync_status() == 0
+    wp = oracle.prune(w, oracle.magnitude_mask(w, s32))
+    assert_close(to_bits(Y), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad), "q_proj s=0.3")
+    h.free()
+
+
 def test_linear_host_matches_device_path():
     name, M = "q_proj", 16
     h, _ = encoded(name)
@@ -266,3 +319,110 @@ def test_linear_rejects_unsupported_rank():
     with pytest.raises(salr.SalrError) as e:
         salr.linear(x, h, A, B)
     assert e.value.code == 2
+
+
+# ---------------------------------------------------------------- serialised image
+
+import image_util  # noqa: E402
+
+
+@pytest.mark.parametrize("name,s", [("tiny", 0.5), ("q_proj", 0.5), ("q_proj", 0.3)])
+def test_save_writes_the_documented_image(name, s):
+    w = weight(name)
+    h = salr.encode(to_dev(w), s)
+    img = h.to_bytes()
+    assert img == image_util.image(w, s)
+    h.free()
+
+
+def test_load_of_an_oracle_image_is_the_encoded_weight():
+    # the image is built by the oracle alone: salr_load must rebuild the handle that
+    # salr_encode would give
+    name = "q_proj"
+    wl = synth.WORKLOADS[name]
+    w = weight(name)
+    img = image_util.image(w, 0.5)
+    h = salr.load(img)
+    m = oracle.magnitude_mask(w, 0.5)
+    wp = oracle.prune(w, m)
+    assert (to_bits(h.decode()) == wp).all()
+    offs, blob = oracle.encode_format(wp, m)
+    gblob, goffs = h.format_tensors()
+    assert (goffs.cpu().numpy().view(np.uint32) == offs).all()
+    assert (gblob.cpu().numpy() == blob).all()
+    assert h.info() == {"N": wl.N, "K": wl.K, "nnz": wl.N * wl.K // 2,
+                        "bytes": blob.size + 4 * offs.size}
+    assert h.to_bytes() == img
+    x = synth.activations(wl, 16)
+    ad, A, B = adapters_dev(name)
+    Y = salr.linear(to_dev(x), h, A, B)
+    assert h.sync_status() == 0
+    assert_close(to_bits(Y), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad), "loaded")
+    h.free()
+
+
+@pytest.mark.parametrize("M", [16, 300])
+def test_save_load_round_trip_serves_the_layer(M):
+    wl = synth.Workload("t", 640, 1152, (64, 16), (M,))
+    w, x = synth.weight(wl), synth.activations(wl, M)
+    ad = synth.adapters(wl)
+    acat = np.concatenate([a for a, _ in ad], axis=1)
+    bcat = np.concatenate([b for _, b in ad], axis=0)
+    h0 = salr.encode(to_dev(w), 0.3)
+    img = h0.to_bytes()
+    h0.free()
+    h = salr.load(img)
+    Y = salr.linear(to_dev(x), h, to_dev(acat), to_dev(bcat))
+    assert h.sync_status() == 0
+    wp = oracle.prune(w, oracle.magnitude_mask(w, float(np.float32(0.3))))
+    assert_close(to_bits(Y), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad),
+                 f"round trip M={M}")
+    h.free()
+
+
+def test_load_rejects_images_that_fail_the_device_checks():
+    # offsets stay valid, so every read of the checks stays inside its block
+    w = weight("tiny")
+    good = image_util.image(w, 0.5)
+    f, offs, blob = image_util.split(good)
+    n, k, keep, nnz, s = f[3], f[4], f[5], f[6], f[7]
+
+    def with_blob(b):
+        return image_util.pack(n, k, keep, nnz, s, offs, b)
+
+    def rejected(img):
+        with pytest.raises(salr.SalrError) as e:
+            salr.load(img)
+        return e.value.code == salr.binding.SALR_ERR_INVALID
+
+    o = offs.astype(np.int64) * 16
+    words = lambda b, blk: b[o[blk]:o[blk] + 1024].view("<u8")  # noqa: E731
+    # 1. eight more bits in a bitmap (16 more value bytes): the population no longer
+    #    gives the block's size
+    b = blob.copy()
+    wv = words(b, 0)
+    for free in np.flatnonzero(((wv[0] >> np.arange(64, dtype=np.uint64)) & 1) == 0)[:8]:
+        wv[0] |= np.uint64(1) << np.uint64(int(free))
+    assert rejected(with_blob(b))
+    # 2. a bit moved from row 0 to row 1 of a block: same size, wrong row counts
+    b = blob.copy()
+    wv = words(b, 0)
+    bits0 = (wv[0] >> np.arange(64, dtype=np.uint64)) & 1
+    bits1 = (wv[1] >> np.arange(64, dtype=np.uint64)) & 1
+    c = int(np.flatnonzero((bits0 == 1) & (bits1 == 0))[0])
+    wv[0] &= ~(np.uint64(1) << np.uint64(c))
+    wv[1] |= np.uint64(1) << np.uint64(c)
+    assert rejected(with_blob(b))
+    # 3. a kept value that is NaN
+    b = blob.copy()
+    b[o[3] + 1024:o[3] + 1026] = [0xC1, 0x7F]
+    assert rejected(with_blob(b))
+    # 4. non-zero padding after the values of a block that has some
+    blocks = len(offs) - 1
+    pops = [sum(bin(int(x)).count("1") for x in words(blob, i)) for i in range(blocks)]
+    i = next(i for i in range(blocks) if (1024 + 2 * pops[i]) % 16)
+    b = blob.copy()
+    b[o[i + 1] - 1] = 1
+    assert rejected(with_blob(b))
+    # the untouched image still loads
+    salr.load(good).free()
