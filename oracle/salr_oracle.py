@@ -22,6 +22,13 @@ technical summary, and the authors' abstract on the scholarfeed author page):
 * ``concat_adapters``: stacking adapters along rank (Methodology 3).
 * ``residual`` / ``truncated_svd_adapter``: E = W0 - W_hat and its rank-r truncated SVD
   (Methodology 2, "Residual Decomposition" and "Theoretical Guarantee").
+* ``randomized_svd_adapter``: the same adapter computed the way the GPU builder does,
+  by a randomized range finder with subspace (power) iteration and a dense SVD of the
+  small projected matrix (Halko, Martinsson and Tropp, "Finding structure with
+  randomness", SIAM Review 2011: the randomized subspace iteration, then the direct
+  SVD of the projected matrix).  The pages fix only the result, a rank-r truncated SVD;
+  the randomized route is this library's reading of how to reach it at scale.  The
+  random test matrix is an input, so both sides use the same draws.
 * ``abs_bound`` / ``check_tolerance``: the per-element and Frobenius acceptance test.
 
 Every function here is pinned by ``tests/test_oracle.py`` against brute force, closed
@@ -225,6 +232,36 @@ def truncated_svd_adapter(E, r: int):
     A = Vt[:r].T * root[None, :]
     B = root[:, None] * U[:, :r].T
     return A, B, sv
+
+
+def randomized_svd_adapter(E, r: int, omega, q: int):
+    """Rank-r adapter of E (N x K) from a randomized range finder, in fp64.
+
+    Steps, in the order of the published algorithm (randomized subspace iteration, then
+    the direct SVD): Q spans E Omega (Omega the K x l test matrix, given); q times, Q is
+    replaced by an orthonormal basis of E (orthonormal basis of E^T Q); then
+    B = Q^T E (l x K) is decomposed exactly, B = U_b S V^T, and U = Q U_b.  The adapter
+    pair is the rank-r part in the X A B orientation: A' = V_r S_r^(1/2) (K x r) and
+    B' = S_r^(1/2) U_r^T (r x N), so A' B' approximates E_r^T.  Orthonormal bases are
+    taken by Householder QR (a library step); the subspace, not the basis, is what the
+    result depends on.  Returns (A', B', singular values of B, descending).
+    """
+    E = np.asarray(E, dtype=np.float64)
+    omega = np.asarray(omega, dtype=np.float64)
+    n, k = E.shape
+    l = omega.shape[1]
+    if omega.shape[0] != k or not (1 <= r <= l <= min(n, k)) or q < 0:
+        raise OracleError("need omega K x l with 1 <= r <= l <= min(N, K) and q >= 0")
+    Q = np.linalg.qr(E @ omega)[0]
+    for _ in range(q):
+        Z = np.linalg.qr(E.T @ Q)[0]
+        Q = np.linalg.qr(E @ Z)[0]
+    B = Q.T @ E
+    Ub, sv, Vt = np.linalg.svd(B, full_matrices=False)
+    root = np.sqrt(sv[:r])
+    A = Vt[:r].T * root[None, :]
+    Bp = root[:, None] * (Q @ Ub[:, :r]).T
+    return A, Bp, sv
 
 
 def mse_factor(r: int, d: int, k: int) -> float:

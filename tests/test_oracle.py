@@ -355,6 +355,87 @@ def test_svd_truncation_is_optimal_against_random_rank_r():
         assert np.linalg.norm(E - cand) >= best - 1e-12
 
 
+def _known_spectrum(rng, N, K, sv):
+    q1, _ = np.linalg.qr(rng.standard_normal((N, N)))
+    q2, _ = np.linalg.qr(rng.standard_normal((K, K)))
+    k = len(sv)
+    return q1[:, :k] @ np.diag(sv) @ q2[:, :k].T, q1, q2
+
+
+def test_randomized_adapter_exact_when_rank_fits_the_sample():
+    # rank(E) <= l: the range finder captures range(E) exactly, so the result is the
+    # exact truncated SVD (closed form from the construction)
+    rng = np.random.default_rng(11)
+    sv = np.array([5.0, 3.0, 2.0, 1.5, 0.7, 0.2])
+    E, q1, q2 = _known_spectrum(rng, 40, 24, sv)
+    r, l = 4, 8
+    A, B, got = oracle.randomized_svd_adapter(E, r, rng.standard_normal((24, l)), 0)
+    assert np.allclose(got[:6], sv, rtol=1e-10) and np.all(np.abs(got[6:]) < 1e-10)
+    expect = q1[:, :r] @ np.diag(sv[:r]) @ q2[:, :r].T  # E_r
+    assert A.shape == (24, r) and B.shape == (r, 40)
+    assert np.allclose((A @ B).T, expect, atol=1e-10)
+
+
+def test_randomized_adapter_ritz_values_and_eckart_young_floor():
+    # singular values of Q^T E never exceed those of E (interlacing), and no rank-r
+    # product beats the truncated SVD's error
+    rng = np.random.default_rng(12)
+    E = rng.standard_normal((50, 36))
+    sv = np.linalg.svd(E, compute_uv=False)
+    total = (sv ** 2).sum()
+    for q in (0, 1, 3):
+        for r, l in ((3, 5), (8, 12)):
+            A, B, got = oracle.randomized_svd_adapter(E, r, rng.standard_normal((36, l)), q)
+            assert np.all(got <= sv[:l] * (1 + 1e-12))
+            err = np.linalg.norm(E - (A @ B).T) ** 2
+            assert err >= (total - (sv[:r] ** 2).sum()) * (1 - 1e-12)
+            # the adapter is the rank-r truncation of the projection Q Q^T E, so its
+            # error is the projection's error plus the dropped Ritz values
+            assert abs(err - (total - (got[:r] ** 2).sum())) <= 1e-9 * total
+
+
+def test_randomized_adapter_converges_on_a_decaying_spectrum():
+    # square, non-symmetric E with geometric singular values: subspace iteration on
+    # E and E^T reaches the truncated SVD; a wrong operand (E for E^T) would not
+    rng = np.random.default_rng(13)
+    sv = 0.7 ** np.arange(50)
+    E, _, _ = _known_spectrum(rng, 50, 50, sv)
+    r, l = 5, 10
+    opt = (sv[r:] ** 2).sum()
+    A, B, got = oracle.randomized_svd_adapter(E, r, rng.standard_normal((50, l)), 6)
+    err = np.linalg.norm(E - (A @ B).T) ** 2
+    assert err <= opt * (1 + 1e-8)
+    assert np.allclose(got[:r], sv[:r], rtol=1e-8)
+
+
+def test_randomized_adapter_depends_only_on_the_sampled_subspace():
+    rng = np.random.default_rng(14)
+    E = rng.standard_normal((30, 26))
+    om = rng.standard_normal((26, 9))
+    G = rng.standard_normal((9, 9)) + 3 * np.eye(9)
+    for q in (0, 2):
+        A1, B1, s1 = oracle.randomized_svd_adapter(E, 4, om, q)
+        A2, B2, s2 = oracle.randomized_svd_adapter(E, 4, om @ G, q)
+        assert np.allclose(s1, s2, rtol=1e-9)
+        assert np.allclose(A1 @ B1, A2 @ B2, atol=1e-9)
+
+
+def test_randomized_adapter_meets_the_stated_mse_factor_on_a_pruned_weight():
+    # the pages' guarantee, (1 - r/min(d, k)) of the residual energy left, holds for the
+    # randomized adapter of a pruned synthetic weight too (its top singular values are
+    # above the mean, so even a partial capture clears the bound)
+    wl = synth.WORKLOADS["tiny"]
+    w = synth.weight(wl)
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    E = oracle.residual(w, wp)
+    total = np.linalg.norm(E) ** 2
+    rng = np.random.default_rng(15)
+    for r in (8, 32):
+        A, B, _ = oracle.randomized_svd_adapter(E, r, rng.standard_normal((wl.K, r + 8)), 2)
+        err = np.linalg.norm(E - (A @ B).T) ** 2
+        assert err <= oracle.mse_factor(r, wl.N, wl.K) * total
+
+
 def test_mse_factor_values():
     assert oracle.mse_factor(64, 4096, 4096) == 1 - 64 / 4096
     assert oracle.mse_factor(8, 256, 128) == 1 - 8 / 128
