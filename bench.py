@@ -87,6 +87,16 @@ def dist_env():
     return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def max_sm_mhz():
+    try:
+        out = subprocess.run(["nvidia-smi", "--id=0", "--query-gpu=clocks.max.sm",
+                              "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                             timeout=20).stdout
+        return float(out.strip().splitlines()[0])
+    except Exception:
+        return None
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -279,6 +289,66 @@ def run_encode_report(args):
     print(json.dumps(line), flush=True)
 
 
+def run_adapter_report(args):
+    """salr_residual_adapter on the workload's W: time, fp32 FMA rate against the
+    CUDA-core peak, and the residual energy it leaves against the pages' factor."""
+    import torch
+
+    from sparse_rank_linear_b200.build import build
+    import sparse_rank_linear_b200 as salr
+
+    build()
+    salr.load_library()
+    wl = workload()
+    N, K = wl.N, wl.K
+    r = wl.ranks[0]
+    l = min(r + 16, 160, N, K)
+    q = 2
+    s = wl.sparsity
+    w_bits = synth.weight(wl)
+    W = torch.from_numpy(np.ascontiguousarray(w_bits).view(np.int16)).view(torch.bfloat16).cuda()
+    h = salr.encode(W, s)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(0)
+    omega = torch.randn(K, l, generator=gen, device="cuda", dtype=torch.float32)
+    salr.residual_adapter(W, h, r, q=q, omega=omega)  # warm
+    ms, wall = [], []
+    for _ in range(max(3, args.steps)):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        e0.record()
+        A, B, sig = salr.residual_adapter(W, h, r, q=q, omega=omega)  # synchronous
+        e1.record()
+        torch.cuda.synchronize()
+        wall.append(time.perf_counter() - t0)
+        ms.append(e0.elapsed_time(e1))
+    # measurement only: the residual and the energy the adapter leaves, in fp32 torch
+    E = W.float() - h.decode().float()
+    total = float((E.double() ** 2).sum())
+    err = float(((E - (A.float() @ B.float()).T).double() ** 2).sum())
+    t = statistics.median(ms) * 1e-3
+    lp = (l + 31) // 32 * 32
+    flops = (4 + 4 * q) * N * K * l  # the E and E^T products (the dominant work)
+    sm = torch.cuda.get_device_properties(0).multi_processor_count
+    clk = max_sm_mhz() or 1965.0
+    fp32_peak = sm * 128 * 2 * clk * 1e6 / 1e12
+    line = {"metric": "SALR residual adapter build (randomized truncated SVD of W0 - W_hat)",
+            "value": t * 1e3, "unit": "ms", "higher_is_better": False, "dtype": "f32",
+            "data": "synthetic", "workload": f"{WORKLOAD} N={N} K={K} r={r} l={l} q={q} "
+                                            f"sparsity={s:.6g}",
+            "steps": max(3, args.steps), "wall_ms": statistics.median(wall) * 1e3,
+            "roofline": {"bound": "alu", "achieved": flops / t / 1e12, "peak": fp32_peak,
+                         "unit": "TFLOP/s", "frac": flops / t / 1e12 / fp32_peak,
+                         "peak_source": f"{sm} SMs x 128 fp32 lanes x 2 x {clk:.0f} MHz",
+                         "algorithmic_flops": flops, "padded_columns": lp},
+            "residual_energy_left": err / total,
+            "pages_factor_bound": 1.0 - r / min(N, K),
+            "sigma_top": [float(x) for x in sig[:4].cpu()]}
+    h.free()
+    print(json.dumps(line), flush=True)
+
+
 def traffic_for(kname, workload):
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -303,6 +373,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["salr", "reference"], default="salr")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--adapter-report", action="store_true",
+                    help="time salr_residual_adapter on the workload's weight")
     ap.add_argument("--encode-report", action="store_true",
                     help="time salr_encode on Llama3-8B-shaped layers and report sizes")
     args = ap.parse_args()
@@ -315,6 +387,8 @@ def main():
         return run_reference(args)
     if args.encode_report:
         return run_encode_report(args)
+    if args.adapter_report:
+        return run_adapter_report(args)
 
     import torch
     import torch.distributed as dist

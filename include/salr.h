@@ -23,6 +23,9 @@
  *     calls are stream-ordered unless stated otherwise.
  *   - Every call returns a salr_status.  Argument errors are detected on the host before
  *     any work is queued; nothing is written in that case.
+ *   - Handles and the scratch of salr_encode, salr_load and salr_residual_adapter take
+ *     device memory from a stream-ordered pool the library owns on each device; memory
+ *     given back to it stays reserved for reuse, up to 1 GiB per device.
  *   - The library never traps or spins without a bound on the GPU.  Errors found on the
  *     device (a NaN in W, a pipeline wait that ran out of time) are recorded in the
  *     handle's status word; salr_encode reports them itself, salr_sync_status reads them.
@@ -227,6 +230,38 @@ SALR_API int salr_save(salr_handle h, void* buf, int64_t buf_bytes, void* stream
  * rules) and frees everything the call allocated.  Synchronises `stream`.
  */
 SALR_API int salr_load(const void* buf, int64_t buf_bytes, void* stream, salr_handle* out);
+
+/*
+ * salr_residual_adapter - the rank-r adapter of what pruning removed from W0.
+ *
+ * Defined by: technical summary, Methodology 2 ("Residual Decomposition": E = W - W_hat,
+ * its rank-r truncated SVD E_r kept as a low-rank adapter; "Theoretical Guarantee": the
+ * per-entry error then shrinks by 1 - r/min(d, k)).  Computed by a randomized range
+ * finder with subspace iteration and a direct SVD of the projected matrix (Halko,
+ * Martinsson and Tropp, SIAM Review 2011): the pages fix the result, not the route.
+ *
+ * W       device, N x K bf16: the dense frozen base that `h` was encoded from.  E is W
+ *         where the handle's mask drops an entry and 0 where it keeps one (exact).
+ * r       adapter rank, 1 <= r <= l.
+ * omega   device, K x l fp32 row-major: the random test matrix (drawn by the caller,
+ *         e.g. standard normal; only the space its columns span matters).  Read only.
+ * l       columns of omega, r <= l <= min(160, N, K); l - r is the oversampling.
+ * q       subspace iterations, 0 <= q <= 16 (each multiplies by E^T and E once more).
+ * A_out   device, K x r bf16 (row-major), B_out device, r x N bf16 (row-major): the
+ *         adapter in the X A B orientation, A' = V_r S_r^(1/2) and B' = S_r^(1/2) U_r^T,
+ *         so that A' B' approximates E_r^T and X A' B' approximates X E_r^T.  Directions
+ *         whose singular value is at or below 1e-6 of the largest get zero columns/rows.
+ * sigma_out  device, r fp32, or NULL: the estimated singular values, descending.
+ *
+ * Arithmetic: E times the tall bases in fp32 on CUDA cores; Gram matrices in fp64;
+ * orthonormal bases by CholeskyQR twice; the small symmetric eigenproblem by cyclic
+ * Jacobi in fp64.  Scratch (about 2 N K + 4 (N + 3 K) l' bytes, l' = l rounded up to 32)
+ * comes from the stream-ordered allocator and is released before the call returns.
+ * Synchronises `stream`.  SALR_ERR_TIMEOUT if the Jacobi iteration hit its sweep bound.
+ */
+SALR_API int salr_residual_adapter(const void* W, salr_handle h, int64_t r, const void* omega,
+                                   int64_t l, int q, void* A_out, void* B_out, void* sigma_out,
+                                   void* stream);
 
 /* salr_sync_status - synchronise `stream`, return the first device-side error recorded
  * for this handle since the last call (SALR_OK if none) and clear it. */

@@ -6,7 +6,7 @@ a ctypes binding of the C ABI in ``include/salr.h``; importing it does not load 
 library, the first call does (and fails loudly if it has not been built).
 """
 from .binding import (SIGNATURES, SalrError, Weight, encode, linear, linear_host, load,
-                      load_library, status_string)
+                      load_library, residual_adapter, status_string)
 
 __all__ = ["SIGNATURES", "SalrError", "Weight", "encode", "linear", "linear_host", "load",
-           "load_library", "status_string"]
+           "load_library", "residual_adapter", "status_string"]

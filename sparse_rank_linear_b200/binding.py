@@ -35,6 +35,7 @@ SIGNATURES = {
     "salr_save_size": (_I, [_P, ctypes.POINTER(_I64)]),
     "salr_save": (_I, [_P, _P, _I64, _P]),
     "salr_load": (_I, [_P, _I64, _P, ctypes.POINTER(_P)]),
+    "salr_residual_adapter": (_I, [_P, _P, _I64, _P, _I64, _I, _P, _P, _P, _P]),
     "salr_sync_status": (_I, [_P, _P]),
     "salr_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -194,6 +195,32 @@ def load(image: bytes, stream=None) -> Weight:
                                                  len(data), _stream_ptr(stream),
                                                  ctypes.byref(h)))
     return Weight(h)
+
+
+def residual_adapter(W, weight: Weight, r: int, q: int = 2, oversample: int = 16, omega=None,
+                     seed: int = 0, stream=None):
+    """salr_residual_adapter: the rank-r adapter (A' K x r, B' r x N, bf16) of W minus its
+    pruned form, and the estimated singular values (r, fp32).  ``omega`` (K x l fp32,
+    CUDA) is the random test matrix; by default a seeded standard normal one with
+    l = r + oversample columns (capped at 160 and at min(N, K))."""
+    import torch
+    inf = weight.info()
+    N, K = inf["N"], inf["K"]
+    _require(W, "W", (N, K))
+    if omega is None:
+        l = min(r + oversample, 160, N, K)
+        g = torch.Generator(device=W.device)
+        g.manual_seed(seed)
+        omega = torch.randn(K, l, generator=g, device=W.device, dtype=torch.float32)
+    if omega.dtype != torch.float32 or not omega.is_contiguous() or omega.shape[0] != K:
+        raise ValueError("omega must be a contiguous K x l float32 tensor")
+    A = torch.empty(K, r, dtype=torch.bfloat16, device=W.device)
+    B = torch.empty(r, N, dtype=torch.bfloat16, device=W.device)
+    sigma = torch.empty(r, dtype=torch.float32, device=W.device)
+    _check("salr_residual_adapter", load_library().salr_residual_adapter(
+        _ptr(W), weight.handle, r, _ptr(omega), omega.shape[1], q, _ptr(A), _ptr(B),
+        _ptr(sigma), _stream_ptr(stream)))
+    return A, B, sigma
 
 
 def linear(X, weight: Weight, A_cat=None, B_cat=None, Y=None, stream=None):

@@ -16,6 +16,7 @@
 #include "salr_codec.cuh"
 #include "salr_prefill.cuh"
 #include "salr_stream.cuh"
+#include "salr_svd.cuh"
 
 using namespace salr;
 
@@ -114,18 +115,57 @@ cudaError_t dev_alloc(void** p, size_t bytes) {
   return cudaMalloc(p, bytes);
 }
 
-// Stream-ordered scratch (freed with cudaFreeAsync on the same stream).
+// The library's stream-ordered memory pool on each device.  Freed blocks stay reserved
+// for reuse up to 1 GiB (the default pool would hand them back to the driver at every
+// synchronisation, and mapping them again costs about as much as a cudaMalloc).
+constexpr uint64_t kPoolKeepBytes = 1ull << 30;
+
+cudaError_t library_pool(int dev, cudaMemPool_t* out) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = kPoolKeepBytes;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return e;
+    }
+    pools[dev] = pool;
+  }
+  *out = pools[dev];
+  return cudaSuccess;
+}
+
+// Stream-ordered allocation from the library pool (freed with cudaFreeAsync).
 cudaError_t dev_alloc_async(void** p, size_t bytes, cudaStream_t st) {
   if (fake_oom()) return cudaErrorMemoryAllocation;
-  return cudaMallocAsync(p, bytes, st);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  cudaMemPool_t pool;
+  if ((e = library_pool(dev, &pool)) != cudaSuccess) return e;
+  return cudaMallocFromPoolAsync(p, bytes, pool, st);
 }
 
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
-// The handle's device memory, [status word][offset table][blob], in one allocation.
-cudaError_t alloc_handle_memory(salr_weight_s* h, int64_t blob_capacity) {
+// The handle's device memory, [status word][offset table][blob], in one allocation from
+// the library pool, ordered on `st` (the calls that make a handle synchronise `st`
+// before returning it, so any stream may use it afterwards).
+cudaError_t alloc_handle_memory(salr_weight_s* h, int64_t blob_capacity, cudaStream_t st) {
   const size_t offs = round256((h->nblocks + 1) * sizeof(uint32_t));
-  const cudaError_t e = dev_alloc(reinterpret_cast<void**>(&h->mem), 256 + offs + blob_capacity);
+  const cudaError_t e =
+      dev_alloc_async(reinterpret_cast<void**>(&h->mem), 256 + offs + blob_capacity, st);
   if (e != cudaSuccess) return e;
   h->status = reinterpret_cast<int*>(h->mem);
   h->offsets = reinterpret_cast<uint32_t*>(h->mem + 256);
@@ -171,11 +211,15 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
 }
 
 void release(salr_weight_s* h) {
+  int cur = -1;
+  const bool switched = cudaGetDevice(&cur) == cudaSuccess && cur != h->device &&
+                        cudaSetDevice(h->device) == cudaSuccess;
   cudaFree(h->sscr.acc);
   cudaFree(h->sscr.counters);
   cudaFree(h->sscr.tacc);
   cudaFree(h->sscr.tflags);
-  cudaFree(h->mem);
+  // pool memory: every caller of release() has synchronised the work that used it
+  if (h->mem) cudaFreeAsync(h->mem, 0);
   cudaFree(h->work.ws);
   cudaFree(h->work.counters);
   cudaFree(h->tscr.T);
@@ -183,6 +227,7 @@ void release(salr_weight_s* h) {
   cudaFree(h->tscr.counters);
   cudaFree(h->x_stage);
   cudaFree(h->y_stage);
+  if (switched) cudaSetDevice(cur);
   h->magic = 0;
   delete h;
 }
@@ -531,7 +576,7 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
     return code;
   };
   cudaError_t e;
-  if ((e = alloc_handle_memory(h, capacity)) != cudaSuccess ||
+  if ((e = alloc_handle_memory(h, capacity, st)) != cudaSuccess ||
       (e = dev_alloc_async(reinterpret_cast<void**>(&scratch), bits_bytes + size_bytes + 256,
                            st)) != cudaSuccess)
     return fail(cuda_status(e));
@@ -858,7 +903,7 @@ int salr_load(const void* buf, int64_t buf_bytes, void* stream, salr_handle* out
     return code;
   };
   cudaError_t e;
-  if ((e = alloc_handle_memory(h, h->blob_bytes)) != cudaSuccess ||
+  if ((e = alloc_handle_memory(h, h->blob_bytes, st)) != cudaSuccess ||
       (e = dev_alloc(reinterpret_cast<void**>(&row_keep), hd.N * sizeof(uint32_t))) !=
           cudaSuccess ||
       (e = dev_alloc(reinterpret_cast<void**>(&nnz_d), sizeof(unsigned long long))) !=
@@ -891,6 +936,204 @@ int salr_load(const void* buf, int64_t buf_bytes, void* stream, salr_handle* out
   cudaFree(row_keep);
   cudaFree(nnz_d);
   publish(h, out);
+  return SALR_OK;
+}
+
+// ------------------------------------------------------------------------------------
+// salr_residual_adapter: the rank-r adapter of the pruning residual (salr_svd.cuh).
+// ------------------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+template <typename TA, bool TR, int MODE>
+cudaError_t launch_skinny(const TA* A, int lda, int rows, int red, const float* Bm, int ldb,
+                          int ncols, float* outf, uint16_t* outb, int ldo, int sms,
+                          cudaStream_t st) {
+  const int tiles = rows / 64;
+  int splits = 1;
+  if (MODE == 0) splits = std::max(1, std::min(red / 32, (2 * sms + tiles - 1) / tiles));
+  const int chunk = (red / 32 + splits - 1) / splits * 32;
+  splits = (red + chunk - 1) / chunk;
+  skinny_gemm_kernel<TA, TR, MODE><<<dim3(tiles, splits), 256, 0, st>>>(
+      A, lda, rows, red, chunk, Bm, ldb, ncols, outf, outb, ldo);
+  return cudaGetLastError();
+}
+
+struct SvdScratch {
+  uint16_t* E;
+  float *Y, *Z, *S, *Om, *Rinv, *MA, *MB, *sig;
+  double* G;
+  int* status;
+};
+
+// Y (rows x lp, l live columns) <- a basis of its columns by CholeskyQR: Y R^-1 with
+// R^T R = Y^T Y.  One pass leaves the basis orthonormal up to about eps cond(Y)^2, which
+// is all the subspace iteration needs between products; the basis the projection uses
+// takes a second pass, which restores orthogonality to rounding level.  Each pass
+// writes the spare buffer and swaps it with Y (all three tall buffers have one size).
+cudaError_t orthonormalise(float*& Y, int rows, int l, int lp, int passes, SvdScratch& s,
+                           int sms, cudaStream_t st) {
+  const int grid = std::max(1, std::min(sms, (rows + 31) / 32));
+  const int rpc = ((rows + grid - 1) / grid + 31) / 32 * 32;
+  const int gsmem = l * l * static_cast<int>(sizeof(double));
+  const int csmem = l * (l + 1) * static_cast<int>(sizeof(double));
+  for (int pass = 0; pass < passes; ++pass) {
+    cudaError_t e = cudaMemsetAsync(s.G, 0, static_cast<size_t>(l) * l * sizeof(double), st);
+    if (e != cudaSuccess) return e;
+    gram_kernel<<<(rows + rpc - 1) / rpc, 1024, gsmem, st>>>(Y, lp, rows, l, rpc, s.G);
+    chol_inv_kernel<<<1, 1024, csmem, st>>>(s.G, l, s.Rinv, lp);
+    e = launch_skinny<float, false, 1>(Y, lp, rows, lp, s.Rinv, lp, lp, s.S, nullptr, lp, sms, st);
+    if (e != cudaSuccess) return e;
+    std::swap(Y, s.S);
+  }
+  return cudaSuccess;
+}
+
+int svd_kernel_attributes(int dev) {
+  static bool set[64] = {false};
+  if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
+  if (set[dev]) return SALR_OK;
+  const int big = kSvdMaxL * (kSvdMaxL + 1) * static_cast<int>(sizeof(double));
+  SALR_TRY(cudaFuncSetAttribute(gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kSvdMaxL * kSvdMaxL * static_cast<int>(sizeof(double))));
+  SALR_TRY(cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+  SALR_TRY(cudaFuncSetAttribute(jacobi_eig_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+  set[dev] = true;
+  return SALR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int salr_residual_adapter(const void* W, salr_handle h, int64_t r, const void* omega, int64_t l,
+                          int q, void* A_out, void* B_out, void* sigma_out, void* stream) {
+  if (!valid_handle(h) || !W || !omega || !A_out || !B_out) return SALR_ERR_INVALID;
+  if (r < 1 || l < r || l > kSvdMaxL || l > h->N || l > h->K || q < 0 || q > 16)
+    return SALR_ERR_INVALID;
+  if (!aligned16(W) || (reinterpret_cast<uintptr_t>(omega) & 3u) ||
+      (reinterpret_cast<uintptr_t>(A_out) & 1u) || (reinterpret_cast<uintptr_t>(B_out) & 1u) ||
+      (reinterpret_cast<uintptr_t>(sigma_out) & 3u))
+    return SALR_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int N = static_cast<int>(h->N), K = static_cast<int>(h->K);
+  const int L = static_cast<int>(l), R = static_cast<int>(r);
+  const int LP = (L + 31) / 32 * 32;
+  const int sms = device_sms(h->device);
+  const int attr = svd_kernel_attributes(h->device);
+  if (attr != SALR_OK) return attr;
+
+  // scratch, one stream-ordered allocation
+  const size_t e_bytes = round256(static_cast<size_t>(N) * K * sizeof(uint16_t));
+  const size_t y_bytes = round256(static_cast<size_t>(N) * LP * sizeof(float));
+  const size_t z_bytes = round256(static_cast<size_t>(K) * LP * sizeof(float));
+  const size_t s_bytes = std::max(y_bytes, z_bytes);
+  const size_t m_bytes = round256(static_cast<size_t>(LP) * LP * sizeof(float));
+  const size_t d_bytes = round256(static_cast<size_t>(L) * L * sizeof(double));
+  const size_t sig_bytes = round256(static_cast<size_t>(LP) * sizeof(float));
+  const size_t f32_bytes = 3 * s_bytes + z_bytes + 3 * m_bytes + sig_bytes;
+  const size_t total = e_bytes + f32_bytes + d_bytes + 256;
+  uint8_t* mem = nullptr;
+  cudaError_t e = dev_alloc_async(reinterpret_cast<void**>(&mem), total, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  SvdScratch sc;
+  uint8_t* p = mem;
+  sc.E = reinterpret_cast<uint16_t*>(p);
+  p += e_bytes;
+  uint8_t* f32 = p;
+  sc.Y = reinterpret_cast<float*>(p);
+  p += s_bytes;
+  sc.Z = reinterpret_cast<float*>(p);
+  p += s_bytes;
+  sc.Om = reinterpret_cast<float*>(p);
+  p += z_bytes;
+  sc.S = reinterpret_cast<float*>(p);
+  p += s_bytes;
+  sc.Rinv = reinterpret_cast<float*>(p);
+  p += m_bytes;
+  sc.MA = reinterpret_cast<float*>(p);
+  p += m_bytes;
+  sc.MB = reinterpret_cast<float*>(p);
+  p += m_bytes;
+  sc.sig = reinterpret_cast<float*>(p);
+  p += sig_bytes;
+  sc.G = reinterpret_cast<double*>(p);
+  p += d_bytes;
+  sc.status = reinterpret_cast<int*>(p);
+
+  auto run = [&]() -> cudaError_t {
+    cudaError_t err;
+    // every fp32 buffer starts at zero: padding columns stay zero throughout
+    if ((err = cudaMemsetAsync(f32, 0, f32_bytes, st)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(sc.status, 0, sizeof(int), st)) != cudaSuccess) return err;
+    if ((err = cudaMemcpy2DAsync(sc.Om, LP * sizeof(float), omega, L * sizeof(float),
+                                 L * sizeof(float), K, cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
+      return err;
+    residual_kernel<<<static_cast<unsigned>(h->nblocks), kBlockRows, 0, st>>>(
+        static_cast<const uint16_t*>(W), h->blob, h->offsets, K, sc.E);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    // Y = E Omega, Q = orth(Y)
+    if ((err = launch_skinny<uint16_t, false, 0>(sc.E, K, N, K, sc.Om, LP, L, sc.Y, nullptr, LP,
+                                                 sms, st)) != cudaSuccess)
+      return err;
+    if ((err = orthonormalise(sc.Y, N, L, LP, q > 0 ? 1 : 2, sc, sms, st)) != cudaSuccess)
+      return err;
+    for (int it = 0; it < q; ++it) {
+      if ((err = cudaMemsetAsync(sc.Z, 0, s_bytes, st)) != cudaSuccess) return err;
+      if ((err = launch_skinny<uint16_t, true, 0>(sc.E, K, K, N, sc.Y, LP, L, sc.Z, nullptr, LP,
+                                                  sms, st)) != cudaSuccess)
+        return err;
+      if ((err = orthonormalise(sc.Z, K, L, LP, 1, sc, sms, st)) != cudaSuccess) return err;
+      if ((err = cudaMemsetAsync(sc.Y, 0, s_bytes, st)) != cudaSuccess) return err;
+      if ((err = launch_skinny<uint16_t, false, 0>(sc.E, K, N, K, sc.Z, LP, L, sc.Y, nullptr, LP,
+                                                   sms, st)) != cudaSuccess)
+        return err;
+      if ((err = orthonormalise(sc.Y, N, L, LP, it + 1 == q ? 2 : 1, sc, sms, st)) !=
+          cudaSuccess)
+        return err;
+    }
+    // Z = E^T Q = B^T; Z^T Z = B B^T, diagonalised on one CTA
+    if ((err = cudaMemsetAsync(sc.Z, 0, s_bytes, st)) != cudaSuccess) return err;
+    if ((err = launch_skinny<uint16_t, true, 0>(sc.E, K, K, N, sc.Y, LP, L, sc.Z, nullptr, LP,
+                                                sms, st)) != cudaSuccess)
+      return err;
+    if ((err = cudaMemsetAsync(sc.G, 0, static_cast<size_t>(L) * L * sizeof(double), st)) !=
+        cudaSuccess)
+      return err;
+    {
+      const int grid = std::max(1, std::min(sms, (K + 31) / 32));
+      const int rpc = ((K + grid - 1) / grid + 31) / 32 * 32;
+      gram_kernel<<<(K + rpc - 1) / rpc, 1024, L * L * static_cast<int>(sizeof(double)), st>>>(
+          sc.Z, LP, K, L, rpc, sc.G);
+    }
+    jacobi_eig_kernel<<<1, 1024, 2 * L * (L | 1) * static_cast<int>(sizeof(float)), st>>>(
+        sc.G, L, R, sc.MA, sc.MB, LP, sc.sig, sc.status);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    // A' = Z U_r S_r^(-1/2) (K x r), B' = (Q U_r S_r^(1/2))^T (r x N)
+    if ((err = launch_skinny<float, false, 2>(sc.Z, LP, K, LP, sc.MA, LP, R, nullptr,
+                                              static_cast<uint16_t*>(A_out), R, sms, st)) !=
+        cudaSuccess)
+      return err;
+    if ((err = launch_skinny<float, false, 3>(sc.Y, LP, N, LP, sc.MB, LP, R, nullptr,
+                                              static_cast<uint16_t*>(B_out), N, sms, st)) !=
+        cudaSuccess)
+      return err;
+    if (sigma_out &&
+        (err = cudaMemcpyAsync(sigma_out, sc.sig, R * sizeof(float), cudaMemcpyDeviceToDevice,
+                               st)) != cudaSuccess)
+      return err;
+    return cudaSuccess;
+  };
+  e = run();
+  int status = 0;
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(&status, sc.status, sizeof(int), cudaMemcpyDeviceToHost, st);
+  cudaFreeAsync(mem, st);
+  const cudaError_t es = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (es != cudaSuccess) return cuda_status(es);
+  if (status & DEV_ERR_TIMEOUT) return SALR_ERR_TIMEOUT;
   return SALR_OK;
 }
 

@@ -76,6 +76,7 @@ def test_bad_arguments_rejected_on_host(lib):
         n = ctypes.c_int64()
         assert lib.salr_save_size(bad, ctypes.byref(n)) == 1
         assert lib.salr_save(bad, fake, 1 << 20, P(0)) == 1
+        assert lib.salr_residual_adapter(fake, bad, 8, fake, 16, 2, fake, fake, None, P(0)) == 1
 
 
 def test_fake_oom_reported(lib):
