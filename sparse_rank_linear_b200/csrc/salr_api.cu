@@ -317,28 +317,32 @@ template <int BNT>
 int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb,
                    const CUtensorMap& tt, int grid, cudaStream_t st) {
   using L = PrefillLayout<BNT>;
-  // One decoded-tile slot per decoder group plus one; as many X tiles as leave room for
-  // one compact-block slot per decoder group; the rest of shared memory for compact
-  // blocks.  The compact-block slots come in a multiple of the group count, so that slot
-  // s only ever holds blocks of group s mod 4: a group then never waits on a slot whose
-  // previous fill it has not consumed itself, and a parity wait can never pass on a phase
-  // two fills old.  Large blocks (little or no pruning) may not leave room for that: then
-  // one decoded-tile slot per group.  That ring is safe for any count of at least the
-  // group count: a group's wait for the consumption of block it - SA follows its own
-  // earlier wait, at block it - 4, which saw block it - 4 - SA >= it - 2 SA consumed (the
-  // MMA consumes in order), so the slot can never be two phases behind.
-  int sa = kPreGroups + 1, sx = kPreMaxX, sc = 0;
-  for (; sa >= kPreGroups; --sa) {
-    for (sx = kPreMaxX; sx >= 2; --sx) {
-      sc = (kSmemLimit - L::smem_bytes(sa, sx, 0, p.cbuf)) / p.cbuf;
-      if (sc >= kPreGroups) break;
+  // Ring sizes.  Among 5 or 4 decoded-tile slots and 4 to 2 X slots, take the layout
+  // with the most compact-block slots (a multiple of the group count, at most kPreMaxC):
+  // compact blocks come from HBM and need the deepest queue, X tiles mostly hit L2.  Ties
+  // go to more X slots, then more decoded-tile slots.
+  //   The compact-block slots come in a multiple of the group count, so that slot s only
+  // ever holds blocks of group s mod 4: a group then never waits on a slot whose previous
+  // fill it has not consumed itself, and a parity wait can never pass on a phase two
+  // fills old.  The decoded-tile ring is safe for any count of at least the group count:
+  // a group's wait for the consumption of block it - SA follows its own earlier wait, at
+  // block it - 4, which saw block it - 4 - SA >= it - 2 SA consumed (the MMA consumes in
+  // order), so the slot can never be two phases behind.
+  int sa = 0, sx = 0, sc = 0;
+  for (int a = kPreGroups + 1; a >= kPreGroups; --a) {
+    for (int x = kPreMaxX; x >= 2; --x) {
+      int c = (kSmemLimit - L::smem_bytes(a, x, 0, p.cbuf)) / p.cbuf;
+      if (c > kPreMaxC) c = kPreMaxC;
+      c -= c % kPreGroups;
+      if (c > sc || (c == sc && c > 0 && (x > sx || (x == sx && a > sa)))) {
+        sa = a;
+        sx = x;
+        sc = c;
+      }
     }
-    if (sx >= 2 && sc >= kPreGroups) break;
   }
-  if (sa < kPreGroups || sx < 2 || sc < kPreGroups) return SALR_ERR_UNSUPPORTED;
+  if (sc < kPreGroups) return SALR_ERR_UNSUPPORTED;
   p.sa = sa;
-  if (sc > kPreMaxC) sc = kPreMaxC;
-  sc -= sc % kPreGroups;
   p.sx = sx;
   p.sc = sc;
   if (L::table_off(p.sa, p.sx, p.sc, p.cbuf) < L::kAdapterBytes) return SALR_ERR_UNSUPPORTED;
@@ -716,7 +720,9 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     tp.R16 = R16;
     tp.kblocks = KB;
     tp.TT = TT;
-    tp.splits = TT < sms ? std::min(KB, sms / TT) : 1;
+    // at least four K blocks per CTA: the split sums meet in L2, and a few blocks per
+    // CTA keep that reduction narrow while still filling the GPU
+    tp.splits = TT < sms ? std::max(1, std::min(KB / 4, sms / TT)) : 1;
     rc = bnt == 128 ? launch_t<128>(tp, tx, ta, TT * tp.splits, st)
                     : launch_t<256>(tp, tx, ta, TT * tp.splits, st);
     if (rc != SALR_OK) return rc;

@@ -318,13 +318,23 @@ __global__ void __launch_bounds__(kPreThreads, 1)
       if (lane == 0) last = atomicAdd(p.counters + cidx, 1u) == static_cast<uint32_t>(p.splits - 1);
       if (__shfl_sync(0xffffffffu, last, 0)) {
         __threadfence();
-        for (int c = 0; c < mvalid; c += 4) {
-          const float4 t4 = __ldcg(reinterpret_cast<const float4*>(sum + c));
-          const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+        // 32 tokens per L2 round trip: a chunk's loads all go out before its stores
+        for (int c0 = 0; c0 < mvalid; c0 += 32) {
+          float4 t4[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (c + e < mvalid) Y[(row0 + c + e) * p.N + n] = __float2bfloat16_rn(tv[e]);
-          __stcg(reinterpret_cast<float4*>(sum + c), make_float4(0.f, 0.f, 0.f, 0.f));
+          for (int g = 0; g < 8; ++g)
+            t4[g] = c0 + 4 * g < mvalid ? __ldcg(reinterpret_cast<const float4*>(sum + c0 + 4 * g))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const int c = c0 + 4 * g;
+            if (c >= mvalid) continue;
+            const float tv[4] = {t4[g].x, t4[g].y, t4[g].z, t4[g].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (c + e < mvalid) Y[(row0 + c + e) * p.N + n] = __float2bfloat16_rn(tv[e]);
+            __stcg(reinterpret_cast<float4*>(sum + c), make_float4(0.f, 0.f, 0.f, 0.f));
+          }
         }
         if (lane == 0) p.counters[cidx] = 0u;
       }
@@ -518,13 +528,24 @@ __global__ void __launch_bounds__(kTThreads, 1)
         if (__shfl_sync(0xffffffffu, last, 0)) {
           __threadfence();
           if (r < p.R16) {
-            for (int c = 0; c < mvalid; c += 4) {
-              const float4 t4 = __ldcg(reinterpret_cast<const float4*>(sum + c));
-              const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+            // 32 tokens per L2 round trip: a chunk's loads all go out before its stores
+            for (int c0 = 0; c0 < mvalid; c0 += 32) {
+              float4 t4[8];
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (c + e < mvalid) T[(row0 + c + e) * 128 + r] = __float2bfloat16_rn(tv[e]);
-              __stcg(reinterpret_cast<float4*>(sum + c), make_float4(0.f, 0.f, 0.f, 0.f));
+              for (int g = 0; g < 8; ++g)
+                t4[g] = c0 + 4 * g < mvalid
+                            ? __ldcg(reinterpret_cast<const float4*>(sum + c0 + 4 * g))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int g = 0; g < 8; ++g) {
+                const int c = c0 + 4 * g;
+                if (c >= mvalid) continue;
+                const float tv[4] = {t4[g].x, t4[g].y, t4[g].z, t4[g].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (c + e < mvalid) T[(row0 + c + e) * 128 + r] = __float2bfloat16_rn(tv[e]);
+                __stcg(reinterpret_cast<float4*>(sum + c), make_float4(0.f, 0.f, 0.f, 0.f));
+              }
             }
           }
           if (lane == 0) p.counters[j * 4 + q] = 0u;

@@ -616,14 +616,27 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         if (*gflag == 0) {
           if (lead) stream_timeout(p, ctrl);
         } else {
-          for (int e = r; e < BNT * p.R16; e += 128) {
-            const int m = e / p.R16, j = e % p.R16;
-            float v = 0.0f;
-            if (m < p.M && j < p.R) v = __ldcg(&p.tacc[m * p.R16 + j]);
-            const int chunk = j >> 6, cc = j & 63;
-            uint8_t* dst = tbuf + chunk * (BNT * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
-                           (((cc >> 3) ^ (m & 7)) << 4) + (cc & 7) * 2;
-            *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
+          // 8 entries per thread per L2 round trip: a batch's loads go out before its
+          // shared-memory stores
+          for (int e0 = r; e0 < BNT * p.R16; e0 += 128 * 8) {
+            float v[8];
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              const int e = e0 + 128 * g;
+              const int m = e / p.R16, j = e % p.R16;
+              v[g] = (e < BNT * p.R16 && m < p.M && j < p.R) ? __ldcg(&p.tacc[m * p.R16 + j])
+                                                            : 0.0f;
+            }
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              const int e = e0 + 128 * g;
+              if (e >= BNT * p.R16) continue;
+              const int m = e / p.R16, j = e % p.R16;
+              const int chunk = j >> 6, cc = j & 63;
+              uint8_t* dst = tbuf + chunk * (BNT * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
+                             (((cc >> 3) ^ (m & 7)) << 4) + (cc & 7) * 2;
+              *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v[g]);
+            }
           }
           fence_proxy_async_smem();
         }
