@@ -345,7 +345,6 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   p.sa = sa;
   p.sx = sx;
   p.sc = sc;
-  if (L::table_off(p.sa, p.sx, p.sc, p.cbuf) < L::kAdapterBytes) return SALR_ERR_UNSUPPORTED;
   const int smem = L::smem_bytes(p.sa, p.sx, p.sc, p.cbuf);
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -708,7 +707,8 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     rc = ensure_tscratch(h, M, st);
     if (rc != SALR_OK) return rc;
     if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
-    if (!make_map(&tb, B_cat, h->N, R, 64, R16)) return SALR_ERR_CUDA;
+    // B_cat^T in chunks of 64 ranks (ranks past R read as zero)
+    if (!make_map(&tb, B_cat, h->N, R, 64, 64)) return SALR_ERR_CUDA;
     if (!make_map(&tt, h->tscr.T, 128, M, 64, bnt)) return SALR_ERR_CUDA;
     TParams tp{};
     tp.T = h->tscr.T;
@@ -747,7 +747,9 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     pp.acc = h->work.ws;
     pp.counters = h->work.counters;
   }
-  const int grid = RT * TT * pp.splits;
+  // persistent: at most one CTA per SM, each taking units cta, cta + grid, ...
+  pp.units = RT * TT * pp.splits;
+  const int grid = std::min(pp.units, sms);
   return bnt == 128 ? launch_prefill<128>(pp, tx, tb, tt, grid, st)
                     : launch_prefill<256>(pp, tx, tb, tt, grid, st);
 }

@@ -32,10 +32,11 @@ namespace salr {
 
 constexpr int kPreDecoders = 16;
 constexpr int kPreGroups = 4;                             // decoder groups (blocks in flight)
+static_assert((kPreGroups & (kPreGroups - 1)) == 0, "group of iteration g is g & (groups - 1)");
 constexpr int kPreThreads = 32 * (7 + kPreDecoders);      // + producer, MMA, 4 epilogue, X loader
 constexpr int kPreMaxC = 8, kPreMaxA = 6, kPreMaxX = 4;    // ring depths
 constexpr int kPreMaxKBlocks = 512;  // K <= 32768
-constexpr int kPreCtrlBytes = 3072;
+constexpr int kPreCtrlBytes = 5120;
 constexpr int kPreTileBytes = 16384;
 
 struct PrefillParams {
@@ -50,6 +51,7 @@ struct PrefillParams {
   int kblocks;         // K / 64
   int TT;              // token tiles
   int splits;          // K splits per output tile
+  int units;           // work units: weight row tiles x token tiles x K splits
   int cbuf;            // bytes of a compact-block slot, multiple of 1024
   int sc, sa, sx;      // ring depths: compact blocks, decoded tiles, X tiles
 };
@@ -58,18 +60,17 @@ struct PrefillCtrl {
   uint64_t cfull[kPreMaxC], cempty[kPreMaxC];
   uint64_t dec[kPreMaxA], aempty[kPreMaxA];
   uint64_t xfull[kPreMaxX], xempty[kPreMaxX];
-  uint64_t tfull, bcfull, fin;
+  uint64_t accfull[2], accempty[2];  // the two TMEM accumulators: MMA -> epilogue -> MMA
+  uint64_t adfull[kPreGroups];       // per decoder group: the B_cat^T copy it requested
+  uint64_t fin;
   uint32_t tmem;
   int abort;
-  int flag;
-  uint32_t off[kPreMaxKBlocks + 1];
+  uint32_t off[2][kPreMaxKBlocks + 1];  // block offsets of the current and the next unit
 };
 static_assert(sizeof(PrefillCtrl) <= kPreCtrlBytes, "control block");
 
 // Shared-memory layout: [decoded tiles: sa x 16 KB][X tiles: sx x BNT*128][compact blocks:
-// sc x cbuf][chunk tables: 4 x 4 KB][nibble table][control].  After the K loop the
-// adapter's operands reuse the front: the B_cat^T tile [128 x R16] at offset 0 (<= 32 KB)
-// and the t tile [BNT x 128] (two 64-rank chunks) at 32 KB.
+// sc x cbuf][chunk tables: 4 x 4 KB][nibble table][control].
 template <int BNT>
 struct PrefillLayout {
   static constexpr int kXbuf = BNT * 128;
@@ -82,7 +83,6 @@ struct PrefillLayout {
     return table_off(sa, sx, sc, cbuf) + kPreGroups * 4096 + 128 /*nibbles*/ + kPreCtrlBytes +
            1024 /*align*/;
   }
-  static constexpr int kAdapterBytes = 32768 + 2 * kXbuf;  // B_cat^T tile + t tile
 };
 
 __device__ __forceinline__ void pre_timeout(int* status, PrefillCtrl* c) {
@@ -93,6 +93,43 @@ __device__ __forceinline__ bool pre_aborted(PrefillCtrl* c) {
   return *reinterpret_cast<volatile int*>(&c->abort) != 0;
 }
 
+// Slot and phase of a ring walked in order (cheaper than dividing the iteration count).
+struct RingCursor {
+  uint32_t s = 0, ph = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++s == static_cast<uint32_t>(n)) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
+// One work unit: weight row tile i, token tile j, K split s, and its K-block range.
+struct PreUnit {
+  int i, j, sidx, kb0, nk, nad;  // nad: adapter iterations (64 ranks each) after the K blocks
+};
+__device__ __forceinline__ PreUnit pre_unit(const PrefillParams& p, int u) {
+  PreUnit w;
+  w.j = u % p.TT;
+  const int rest = u / p.TT;
+  w.sidx = rest % p.splits;
+  w.i = rest / p.splits;
+  w.kb0 = static_cast<int>(static_cast<long long>(w.sidx) * p.kblocks / p.splits);
+  const int kb1 = static_cast<int>(static_cast<long long>(w.sidx + 1) * p.kblocks / p.splits);
+  w.nk = kb1 - w.kb0;
+  w.nad = (p.R16 > 0 && w.sidx == 0) ? (p.R16 + 63) / 64 : 0;
+  return w;
+}
+
+// Persistent: one CTA per SM takes units blockIdx.x, blockIdx.x + gridDim.x, ...  Every
+// role walks the same sequence of iterations g (the K blocks of each unit, then its
+// adapter chunks), so ring slot g % S and phase (g / S) & 1 agree between roles across
+// units, and the rings run on from one unit into the next.  An adapter chunk is one more
+// iteration: its decoder group copies 64 ranks of B_cat^T (an MN-major 128 x 64 tile)
+// into the decoded-tile slot instead of decoding, the X loader copies the matching 64
+// ranks of t, and its compact-block slot turn carries no data.  Accumulators alternate
+// between two TMEM column ranges, so that the epilogue of one unit overlaps the MMAs of
+// the next.
 template <int BNT>
 __global__ void __launch_bounds__(kPreThreads, 1)
     salr_prefill_kernel(const __grid_constant__ PrefillParams p,
@@ -110,23 +147,11 @@ __global__ void __launch_bounds__(kPreThreads, 1)
   uint8_t* tables = smem + L::table_off(SA, SX, SC, p.cbuf);
   uint2* ntab = reinterpret_cast<uint2*>(tables + kPreGroups * 4096);
   PrefillCtrl* ctrl = reinterpret_cast<PrefillCtrl*>(tables + kPreGroups * 4096 + 128);
-  uint8_t* bcbuf = smem;           // after the K loop only
-  uint8_t* tbuf = smem + 32768;    // after the K loop only
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool adapter = p.R16 > 0;
-  // work unit: token tile j (fastest), K split s, weight row tile i
-  const int cta = blockIdx.x;
-  const int j = cta % p.TT;
-  const int rest = cta / p.TT;
-  const int sidx = rest % p.splits;
-  const int i = rest / p.splits;
-  const int kb0 = static_cast<int>(static_cast<long long>(sidx) * p.kblocks / p.splits);
-  const int kb1 = static_cast<int>(static_cast<long long>(sidx + 1) * p.kblocks / p.splits);
-  const int nk = kb1 - kb0;
-  const bool add_adapter = adapter && sidx == 0;
+  const int G = gridDim.x, cta = blockIdx.x;
   constexpr int WPG = kPreDecoders / kPreGroups;
-  constexpr uint32_t kCols = BNT < 32 ? 32 : BNT;
+  constexpr uint32_t kCols = 2 * BNT;  // two accumulators
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SC; ++s) {
@@ -141,18 +166,16 @@ __global__ void __launch_bounds__(kPreThreads, 1)
       mbar_init(&ctrl->xfull[s], 1);
       mbar_init(&ctrl->xempty[s], 1);
     }
-    mbar_init(&ctrl->tfull, 1);
-    mbar_init(&ctrl->bcfull, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctrl->accfull[b], 1);
+      mbar_init(&ctrl->accempty[b], 4);
+    }
+    for (int g = 0; g < kPreGroups; ++g) mbar_init(&ctrl->adfull[g], 1);
     mbar_init(&ctrl->fin, 1);
     ctrl->abort = 0;
-    ctrl->flag = 0;
     fence_mbar_init();
   }
   if (threadIdx.x < 16) ntab[threadIdx.x] = nibble_entry(threadIdx.x);
-  if (warp == 0) {
-    const uint32_t* src = p.offsets + static_cast<size_t>(i) * p.kblocks + kb0;
-    for (int t = lane; t <= nk; t += 32) ctrl->off[t] = src[t];
-  }
   if (warp == 1) tmem_alloc(&ctrl->tmem, kCols);
   tc_fence_before();
   __syncthreads();
@@ -161,60 +184,86 @@ __global__ void __launch_bounds__(kPreThreads, 1)
 
   if (warp == 0) {
     // ================================================================ compact-block producer
-    if (lane == 0) {
-      int issued = 0;
-      bool bc_issued = false;
-      for (int it = 0; it < nk; ++it) {
-        const int s = it % SC;
-        if (!mbar_wait(&ctrl->cempty[s], ((it / SC) & 1) ^ 1) || pre_aborted(ctrl)) {
-          pre_timeout(p.status, ctrl);
-          break;
+    // Each unit's block offsets sit in one of two shared buffers: the whole warp starts
+    // the copy of the next unit's offsets (cp.async) before lane 0 issues this unit's
+    // blocks, and waits for it after, so the next unit's first copy goes out at once.
+    uint32_t g = 0, gi = 0;  // iterations walked / slot turns issued
+    RingCursor cc;           // lane 0's compact-ring cursor
+    bool ok = true;
+    int ob = 0;
+    if (cta < p.units) {
+      const PreUnit w = pre_unit(p, cta);
+      const uint32_t* src = p.offsets + static_cast<size_t>(w.i) * p.kblocks + w.kb0;
+      for (int t = lane; t <= w.nk; t += 32) ctrl->off[0][t] = src[t];
+    }
+    __syncwarp();
+    for (int u = cta; u < p.units && ok; u += G) {
+      const PreUnit w = pre_unit(p, u);
+      if (u + G < p.units) {
+        const PreUnit wn = pre_unit(p, u + G);
+        const uint32_t* src = p.offsets + static_cast<size_t>(wn.i) * p.kblocks + wn.kb0;
+        for (int t = lane; t <= wn.nk; t += 32) cp_async4(&ctrl->off[ob ^ 1][t], src + t);
+      }
+      if (lane == 0) {
+        const uint32_t* off = ctrl->off[ob];
+        for (int it = 0; it < w.nk + w.nad; ++it, cc.next(SC)) {
+          const uint32_t s = cc.s;
+          if (!mbar_wait(&ctrl->cempty[s], cc.ph ^ 1) || pre_aborted(ctrl)) {
+            pre_timeout(p.status, ctrl);
+            ok = false;
+            break;
+          }
+          if (it < w.nk) {
+            const uint32_t o0 = off[it], o1 = off[it + 1];
+            mbar_arrive_expect_tx(&ctrl->cfull[s], (o1 - o0) * 16u);
+            bulk_g2s(cbuf(s), p.blob + static_cast<size_t>(o0) * 16, (o1 - o0) * 16u,
+                     &ctrl->cfull[s]);
+          } else {
+            mbar_arrive(&ctrl->cfull[s]);  // an adapter iteration: the turn carries no data
+          }
+          gi = g + it + 1;
         }
-        const uint32_t o0 = ctrl->off[it], o1 = ctrl->off[it + 1];
-        mbar_arrive_expect_tx(&ctrl->cfull[s], (o1 - o0) * 16u);
-        bulk_g2s(cbuf(s), p.blob + static_cast<size_t>(o0) * 16, (o1 - o0) * 16u, &ctrl->cfull[s]);
-        issued = it + 1;
       }
-      if (add_adapter && !pre_aborted(ctrl)) {
-        // the adapter operands go where the rings were: wait until every MMA read them
-        if (!mbar_wait(&ctrl->tfull, 0)) {
-          pre_timeout(p.status, ctrl);
-        } else {
-          prefetch_tmap(&tmB);
-          prefetch_tmap(&tmT);
-          const int nch = (p.R16 + 63) / 64;
-          mbar_arrive_expect_tx(&ctrl->bcfull, 256u * p.R16 + nch * L::kXbuf);
-          tma_load_2d(bcbuf, &tmB, i * 128, 0, &ctrl->bcfull);
-          tma_load_2d(bcbuf + p.R16 * 128, &tmB, i * 128 + 64, 0, &ctrl->bcfull);
-          for (int c = 0; c < nch; ++c) tma_load_2d(tbuf + c * L::kXbuf, &tmT, c * 64, j * BNT, &ctrl->bcfull);
-          bc_issued = true;
-        }
-      }
-      if (pre_aborted(ctrl)) {
-        // let every copy this thread started land before the CTA can exit
-        for (int it = issued - SC < 0 ? 0 : issued - SC; it < issued; ++it)
-          mbar_wait(&ctrl->cfull[it % SC], (it / SC) & 1);
-        if (bc_issued) mbar_wait(&ctrl->bcfull, 0);
-      }
+      cp_async_wait_all();
+      __syncwarp();  // the next unit's offsets, copied by every lane, are visible to lane 0
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      g += w.nk + w.nad;
+      ob ^= 1;
+    }
+    cp_async_wait_all();
+    if (lane == 0 && pre_aborted(ctrl)) {
+      // let every copy this thread started land before the CTA can exit
+      for (uint32_t x = gi > static_cast<uint32_t>(SC) ? gi - SC : 0; x < gi; ++x)
+        mbar_wait(&ctrl->cfull[x % SC], (x / SC) & 1);
     }
   } else if (warp == 6) {
-    // ================================================================ X-tile producer
+    // ================================================================ X / t tile producer
     if (lane == 0) {
       prefetch_tmap(&tmX);
-      int issued = 0;
-      for (int it = 0; it < nk; ++it) {
-        const int s = it % SX;
-        if (!mbar_wait(&ctrl->xempty[s], ((it / SX) & 1) ^ 1) || pre_aborted(ctrl)) {
-          pre_timeout(p.status, ctrl);
-          break;
+      if (p.R16 > 0) prefetch_tmap(&tmT);
+      uint32_t g = 0, gi = 0;
+      RingCursor xc;
+      bool ok = true;
+      for (int u = cta; u < p.units && ok; u += G) {
+        const PreUnit w = pre_unit(p, u);
+        for (int it = 0; it < w.nk + w.nad; ++it, ++g, xc.next(SX)) {
+          const uint32_t s = xc.s;
+          if (!mbar_wait(&ctrl->xempty[s], xc.ph ^ 1) || pre_aborted(ctrl)) {
+            pre_timeout(p.status, ctrl);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctrl->xfull[s], L::kXbuf);
+          if (it < w.nk)
+            tma_load_2d(xbuf(s), &tmX, (w.kb0 + it) * 64, w.j * BNT, &ctrl->xfull[s]);
+          else
+            tma_load_2d(xbuf(s), &tmT, (it - w.nk) * 64, w.j * BNT, &ctrl->xfull[s]);
+          gi = g + 1;
         }
-        mbar_arrive_expect_tx(&ctrl->xfull[s], L::kXbuf);
-        tma_load_2d(xbuf(s), &tmX, (kb0 + it) * 64, j * BNT, &ctrl->xfull[s]);
-        issued = it + 1;
       }
       if (pre_aborted(ctrl)) {
-        for (int it = issued - SX < 0 ? 0 : issued - SX; it < issued; ++it)
-          mbar_wait(&ctrl->xfull[it % SX], (it / SX) & 1);
+        for (uint32_t x = gi > static_cast<uint32_t>(SX) ? gi - SX : 0; x < gi; ++x)
+          mbar_wait(&ctrl->xfull[x % SX], (x / SX) & 1);
       }
     }
   } else if (warp == 1) {
@@ -226,43 +275,46 @@ __global__ void __launch_bounds__(kPreThreads, 1)
       const uint64_t xdesc0 = smem_desc_sw128(smem_u32(xbuf(0)), 16, 1024);
       constexpr uint32_t astep = kPreTileBytes >> 4, xstep = L::kXbuf >> 4;
       bool ok = true;
-      int sa = 0, sx = 0;
-      uint32_t pa = 0, px = 0;
-      for (int it = 0; it < nk; ++it) {
-        if (!mbar_wait(&ctrl->dec[sa], pa) || !mbar_wait(&ctrl->xfull[sx], px) || pre_aborted(ctrl)) {
+      RingCursor ac, xc;
+      int t = 0;
+      for (int u = cta; u < p.units && ok; u += G, ++t) {
+        const PreUnit w = pre_unit(p, u);
+        const int b = t & 1;
+        const uint32_t acc = tmem + static_cast<uint32_t>(b * BNT);
+        if (!mbar_wait(&ctrl->accempty[b], ((t >> 1) & 1) ^ 1) || pre_aborted(ctrl)) {
           pre_timeout(p.status, ctrl);
-          ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t da = adesc0 + sa * astep, dx = xdesc0 + sx * xstep;
-        mma_bf16_ss(tmem, da, dx, idesc, it != 0);
-        mma_bf16_ss(tmem, da + 2, dx + 2, idesc, 1u);
-        mma_bf16_ss(tmem, da + 4, dx + 4, idesc, 1u);
-        mma_bf16_ss(tmem, da + 6, dx + 6, idesc, 1u);
-        mma_commit(&ctrl->aempty[sa]);
-        mma_commit(&ctrl->xempty[sx]);
-        if (++sa == SA) {
-          sa = 0;
-          pa ^= 1u;
-        }
-        if (++sx == SX) {
-          sx = 0;
-          px ^= 1u;
-        }
-      }
-      mma_commit(&ctrl->tfull);
-      if (ok && add_adapter) {
-        if (!mbar_wait(&ctrl->bcfull, 0) || pre_aborted(ctrl)) {
-          pre_timeout(p.status, ctrl);
-        } else {
+        for (int it = 0; it < w.nk + w.nad; ++it, ac.next(SA), xc.next(SX)) {
+          const uint32_t sa = ac.s, sx = xc.s;
+          if (!mbar_wait(&ctrl->dec[sa], ac.ph) || !mbar_wait(&ctrl->xfull[sx], xc.ph) ||
+              pre_aborted(ctrl)) {
+            pre_timeout(p.status, ctrl);
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint32_t b0 = smem_u32(bcbuf), t0 = smem_u32(tbuf);
-          for (int k = 0; k < p.R16 / 16; ++k)
-            mma_bf16_ss(tmem, smem_desc_sw128(b0 + 2048 * k, p.R16 * 128, 1024),
-                        smem_desc_sw128(t0 + (k >> 2) * (BNT * 128) + (k & 3) * 32, 16, 1024),
-                        idesc_mn, 1u);
+          const uint64_t dx = xdesc0 + sx * xstep;
+          if (it < w.nk) {
+            const uint64_t da = adesc0 + sa * astep;
+            mma_bf16_ss(acc, da, dx, idesc, it != 0);
+            mma_bf16_ss(acc, da + 2, dx + 2, idesc, 1u);
+            mma_bf16_ss(acc, da + 4, dx + 4, idesc, 1u);
+            mma_bf16_ss(acc, da + 6, dx + 6, idesc, 1u);
+          } else {
+            // B_cat^T chunk, MN-major: two 64-row halves 8 KB apart, 16 ranks = 2 KB
+            const int c = it - w.nk;
+            const int kk = min(4, (p.R16 - 64 * c) / 16);
+            const uint32_t a0 = smem_u32(abuf(sa));
+            for (int k = 0; k < kk; ++k)
+              mma_bf16_ss(acc, smem_desc_sw128(a0 + 2048 * k, 8192, 1024), dx + 2 * k, idesc_mn,
+                          1u);
+          }
+          mma_commit(&ctrl->aempty[sa]);
+          mma_commit(&ctrl->xempty[sx]);
         }
+        if (ok) mma_commit(&ctrl->accfull[b]);
       }
       mma_commit(&ctrl->fin);
       // every MMA of this CTA has finished before TMEM can be released
@@ -270,101 +322,141 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     }
   } else if (warp < 6) {
     // ================================================================ epilogue (warps 2-5)
-    // Decisions guarding warp-collective instructions or the group barrier are made
-    // uniform first (a vote, then one shared flag).
     const int q = warp & 3;  // TMEM lane quarter
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     const int r = 32 * q + lane;  // weight row within the tile
-    bool ok = mbar_wait(&ctrl->fin, 0);
-    if (!ok) pre_timeout(p.status, ctrl);
-    ok = __all_sync(0xffffffffu, ok);
-    named_bar(1, 128);
-    if (threadIdx.x == 64) ctrl->flag = (ok && !pre_aborted(ctrl)) ? 2 : 0;
-    named_bar(1, 128);
-    const bool go = *reinterpret_cast<volatile int*>(&ctrl->flag) == 2;
-    tc_fence_after();
-    const int mvalid = min(BNT, p.M - j * BNT);
-    const size_t n = static_cast<size_t>(i) * 128 + r;
-    const size_t row0 = static_cast<size_t>(j) * BNT;
     __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(p.Y);
-    if (go && p.splits == 1) {
-      for (int c = 0; c < BNT; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_base + c, v);
-        tmem_ld_wait();
+    int t = 0;
+    for (int u = cta; u < p.units; u += G, ++t) {
+      const PreUnit w = pre_unit(p, u);
+      const int b = t & 1;
+      const uint32_t acc = tmem + static_cast<uint32_t>(b * BNT);
+      bool ok = mbar_wait(&ctrl->accfull[b], (t >> 1) & 1) && !pre_aborted(ctrl);
+      if (!ok) pre_timeout(p.status, ctrl);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int mvalid = min(BNT, p.M - w.j * BNT);
+      const size_t n = static_cast<size_t>(w.i) * 128 + r;
+      const size_t row0 = static_cast<size_t>(w.j) * BNT;
+      if (p.splits == 1) {
+        for (int c = 0; c < BNT; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(acc + lane_base + c, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (c + e < mvalid)
-            Y[(row0 + c + e) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
-      }
-    } else if (go) {
-      // split K: add into the tile's fp32 sum in L2 (row n, token-contiguous), count in
-      // per warp; the warp that arrives last for these 32 rows writes Y and clears both
-      float* sum = p.acc + n * p.Mp + row0;
-      for (int c = 0; c < BNT; c += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_base + c, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; e += 4)
-          if (c + e < mvalid)
-            red_add_v4f32(sum + c + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                          __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-      }
-      __threadfence();
-      __syncwarp();
-      uint32_t last = 0;
-      const size_t cidx = (static_cast<size_t>(i) * p.TT + j) * 4 + q;
-      if (lane == 0) last = atomicAdd(p.counters + cidx, 1u) == static_cast<uint32_t>(p.splits - 1);
-      if (__shfl_sync(0xffffffffu, last, 0)) {
-        __threadfence();
-        // 32 tokens per L2 round trip: a chunk's loads all go out before its stores
-        for (int c0 = 0; c0 < mvalid; c0 += 32) {
-          float4 t4[8];
-#pragma unroll
-          for (int g = 0; g < 8; ++g)
-            t4[g] = c0 + 4 * g < mvalid ? __ldcg(reinterpret_cast<const float4*>(sum + c0 + 4 * g))
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const int c = c0 + 4 * g;
-            if (c >= mvalid) continue;
-            const float tv[4] = {t4[g].x, t4[g].y, t4[g].z, t4[g].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (c + e < mvalid) Y[(row0 + c + e) * p.N + n] = __float2bfloat16_rn(tv[e]);
-            __stcg(reinterpret_cast<float4*>(sum + c), make_float4(0.f, 0.f, 0.f, 0.f));
-          }
+          for (int e = 0; e < 16; ++e)
+            if (c + e < mvalid)
+              Y[(row0 + c + e) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
         }
-        if (lane == 0) p.counters[cidx] = 0u;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->accempty[b]);
+      } else {
+        // split K: add into the tile's fp32 sum in L2 (row n, token-contiguous), count in
+        // per warp; the warp that arrives last for these 32 rows writes Y and clears both
+        float* sum = p.acc + n * p.Mp + row0;
+        for (int c = 0; c < BNT; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(acc + lane_base + c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            if (c + e < mvalid)
+              red_add_v4f32(sum + c + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                            __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->accempty[b]);
+        __threadfence();
+        __syncwarp();
+        uint32_t last = 0;
+        const size_t cidx = (static_cast<size_t>(w.i) * p.TT + w.j) * 4 + q;
+        if (lane == 0) last = atomicAdd(p.counters + cidx, 1u) == static_cast<uint32_t>(p.splits - 1);
+        if (__shfl_sync(0xffffffffu, last, 0)) {
+          __threadfence();
+          // 32 tokens per L2 round trip: a chunk's loads all go out before its stores
+          for (int c0 = 0; c0 < mvalid; c0 += 32) {
+            float4 t4[8];
+#pragma unroll
+            for (int gq = 0; gq < 8; ++gq)
+              t4[gq] = c0 + 4 * gq < mvalid
+                           ? __ldcg(reinterpret_cast<const float4*>(sum + c0 + 4 * gq))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int gq = 0; gq < 8; ++gq) {
+              const int c = c0 + 4 * gq;
+              if (c >= mvalid) continue;
+              const float tv[4] = {t4[gq].x, t4[gq].y, t4[gq].z, t4[gq].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (c + e < mvalid) Y[(row0 + c + e) * p.N + n] = __float2bfloat16_rn(tv[e]);
+              __stcg(reinterpret_cast<float4*>(sum + c), make_float4(0.f, 0.f, 0.f, 0.f));
+            }
+          }
+          if (lane == 0) p.counters[cidx] = 0u;
+        }
       }
     }
   } else {
     // ================================================================ decoders (warps 7-22)
-    // four groups of four warps, group g on blocks g, g + 4, ..., each warp on 32 rows
+    // four groups of four warps; group x takes the iterations g = x mod 4, each warp 32
+    // rows of a block (or, for an adapter chunk, the group's leader copies B_cat^T)
     constexpr int RPW = 128 / WPG;
     const int dw = warp - 7;
-    const int g = dw / WPG, wg = dw % WPG;
-    uint32_t* cs = reinterpret_cast<uint32_t*>(tables + g * 4096);
-    for (int it = g; it < nk; it += kPreGroups) {
-      const int sc = it % SC, sa = it % SA;
-      if (!mbar_wait(&ctrl->cfull[sc], (it / SC) & 1) || pre_aborted(ctrl)) {
-        pre_timeout(p.status, ctrl);
-        break;
-      }
-      const uint8_t* cb = cbuf(sc);
-      build_chunk_table<RPW>(reinterpret_cast<const uint64_t*>(cb), cs, wg, lane);
-      __syncwarp();
-      if (!mbar_wait(&ctrl->aempty[sa], ((it / SA) & 1) ^ 1)) {
-        pre_timeout(p.status, ctrl);
-        break;
-      }
-      expand_rows<RPW>(cb + kBitmapBytes, cs, abuf(sa), wg, lane, ntab);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&ctrl->dec[sa]);
-        mbar_arrive(&ctrl->cempty[sc]);
+    const int grp = dw / WPG, wg = dw % WPG;
+    uint32_t* cs = reinterpret_cast<uint32_t*>(tables + grp * 4096);
+    if (p.R16 > 0 && wg == 0 && lane == 0) prefetch_tmap(&tmB);
+    uint32_t g = 0, adn = 0;
+    RingCursor cc, ac;  // walked on every iteration, this group's or not
+    bool ok = true;
+    for (int u = cta; u < p.units && ok; u += G) {
+      const PreUnit w = pre_unit(p, u);
+      for (int it = 0; it < w.nk + w.nad; ++it, ++g, cc.next(SC), ac.next(SA)) {
+        if (static_cast<int>(g & (kPreGroups - 1)) != grp) continue;
+        const uint32_t sc = cc.s, sa = ac.s;
+        if (!mbar_wait(&ctrl->cfull[sc], cc.ph) || pre_aborted(ctrl)) {
+          pre_timeout(p.status, ctrl);
+          ok = false;
+          break;
+        }
+        if (it < w.nk) {
+          const uint8_t* cb = cbuf(sc);
+          build_chunk_table<RPW>(reinterpret_cast<const uint64_t*>(cb), cs, wg, lane);
+          __syncwarp();
+          if (!mbar_wait(&ctrl->aempty[sa], ac.ph ^ 1)) {
+            pre_timeout(p.status, ctrl);
+            ok = false;
+            break;
+          }
+          expand_rows<RPW>(cb + kBitmapBytes, cs, abuf(sa), wg, lane, ntab);
+          fence_proxy_async_smem();
+        } else {
+          if (!mbar_wait(&ctrl->aempty[sa], ac.ph ^ 1)) {
+            pre_timeout(p.status, ctrl);
+            ok = false;
+            break;
+          }
+          if (wg == 0 && lane == 0) {
+            const int c = it - w.nk;
+            mbar_arrive_expect_tx(&ctrl->adfull[grp], kPreTileBytes);
+            tma_load_2d(abuf(sa), &tmB, w.i * 128, c * 64, &ctrl->adfull[grp]);
+            tma_load_2d(abuf(sa) + 8192, &tmB, w.i * 128 + 64, c * 64, &ctrl->adfull[grp]);
+          }
+          // every warp of the group waits for the copy (a bounded wait also lets the
+          // copy land before the CTA can exit)
+          if (!mbar_wait(&ctrl->adfull[grp], adn & 1)) {
+            pre_timeout(p.status, ctrl);
+            ok = false;
+            break;
+          }
+          ++adn;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&ctrl->dec[sa]);
+          mbar_arrive(&ctrl->cempty[sc]);
+        }
       }
     }
   }

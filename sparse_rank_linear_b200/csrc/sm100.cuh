@@ -96,6 +96,16 @@ __device__ __forceinline__ void red_add_v4f32(float* p, float a, float b, float 
 
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor cores, TMA) before signalling a consumer.
+// 4-byte asynchronous global -> shared copy (completion via cp.async.wait_all).
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
