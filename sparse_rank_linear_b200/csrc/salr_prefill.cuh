@@ -6,21 +6,22 @@
 //   rounded once to bf16 into a [M x 128] scratch.  Grid: token tiles x K splits.  With
 //   several splits, each adds its fp32 part into a sum in L2 (vector reductions), and the
 //   last split of a token tile to count itself in converts the sum and clears it.
-// * salr_prefill_kernel: one CTA per (128-row weight tile, token tile, K split).  Each
-//   128 x 64 bitmap block arrives by one bulk copy and the matching X tile by tensor TMA.
-//   Decoder warps expand the block into the 128-byte-swizzled tile (stage 1, Methodology
-//   4) with the same device functions as the small-M kernel; tcgen05 MMAs multiply it
-//   (stage 2).  After the K blocks,
-//   the CTA of split 0 adds B_cat^T t^T with R/16 more MMAs.  The epilogue writes Y; with
-//   several K splits, each adds into an fp32 sum in L2 whose last contributor writes Y.
+// * salr_prefill_kernel: persistent, one CTA per SM over the work units (128-row weight
+//   tile, token tile, K split).  Each 128 x 64 bitmap block arrives by one bulk copy and
+//   the matching X tile by tensor TMA.  Decoder warps expand the block into the
+//   128-byte-swizzled tile (stage 1, Methodology 4) with the same device functions as
+//   the small-M kernel; tcgen05 MMAs multiply it (stage 2).  The adapter's up projection
+//   B_cat^T t^T runs as extra iterations of the same pipeline after a unit's K blocks (on
+//   split 0).  The epilogue writes Y; with several K splits, each adds into an fp32 sum in
+//   L2 whose last contributor writes Y.
 //
-// Orientation as in the small-M kernel: D[128 weight rows x BNT tokens] in TMEM.
-// Rings: compact blocks (producer -> decoders), decoded tiles (decoders -> MMA) and X
-// tiles (X loader -> MMA), so that the copy latency and the decode of a block overlap the
-// MMAs of earlier blocks; four decoder groups each work on a different block.
-// Warp roles (736 threads): 0 compact-block producer, 1 TMEM allocator + MMA issuer, 2-5
-// epilogue, 6 X-tile producer, 7-22 decoders.  Every wait is bounded; a timeout is
-// recorded in the status word.
+// Orientation as in the small-M kernel: D[128 weight rows x BNT tokens] in TMEM, two
+// accumulators used by alternate units.  Rings: compact blocks (producer -> decoders),
+// decoded tiles (decoders -> MMA) and X tiles (X loader -> MMA), so that the copy latency
+// and the decode of a block overlap the MMAs of earlier blocks; four decoder groups each
+// work on a different block.  Warp roles (736 threads): 0 compact-block producer, 1 TMEM
+// allocator + MMA issuer, 2-5 epilogue, 6 X-tile producer, 7-22 decoders.  Every wait is
+// bounded; a timeout is recorded in the status word.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
