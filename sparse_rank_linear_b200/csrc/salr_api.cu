@@ -315,7 +315,7 @@ int launch_t(const TParams& p, const CUtensorMap& tx, const CUtensorMap& ta, int
 
 template <int BNT>
 int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb,
-                   const CUtensorMap& tt, int grid, cudaStream_t st) {
+                   const CUtensorMap& tt, int grid, bool after_t, cudaStream_t st) {
   using L = PrefillLayout<BNT>;
   // Ring sizes.  Among 5 or 4 decoded-tile slots and 4 to 2 X slots, take the layout
   // with the most compact-block slots (a multiple of the group count, at most kPreMaxC):
@@ -355,8 +355,20 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
     attr_set[dev] = true;
   }
-  salr_prefill_kernel<BNT><<<grid, kPreThreads, smem, st>>>(p, tx, tb, tt);
-  SALR_TRY(cudaGetLastError());
+  // Directly after the t kernel, the launch may overlap it (programmatic stream
+  // serialization): the t kernel started only once everything before it had completed,
+  // and the layer kernel waits for the t kernel itself before its first read of t.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPreThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_t ? 1 : 0;
+  SALR_TRY(cudaLaunchKernelEx(&cfg, salr_prefill_kernel<BNT>, p, tx, tb, tt));
   return SALR_OK;
 }
 
@@ -703,30 +715,8 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   std::memset(&tb, 0, sizeof(tb));
   std::memset(&tt, 0, sizeof(tt));
   if (!make_map(&tx, X, h->K, M, 64, bnt)) return SALR_ERR_CUDA;
-  if (R > 0) {
-    rc = ensure_tscratch(h, M, st);
-    if (rc != SALR_OK) return rc;
-    if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
-    // B_cat^T in chunks of 64 ranks (ranks past R read as zero)
-    if (!make_map(&tb, B_cat, h->N, R, 64, 64)) return SALR_ERR_CUDA;
-    if (!make_map(&tt, h->tscr.T, 128, M, 64, bnt)) return SALR_ERR_CUDA;
-    TParams tp{};
-    tp.T = h->tscr.T;
-    tp.T32 = h->tscr.T32;
-    tp.counters = h->tscr.counters;
-    tp.status = h->status;
-    tp.M = static_cast<int>(M);
-    tp.Mp = static_cast<int>(Mp);
-    tp.R16 = R16;
-    tp.kblocks = KB;
-    tp.TT = TT;
-    // at least four K blocks per CTA: the split sums meet in L2, and a few blocks per
-    // CTA keep that reduction narrow while still filling the GPU
-    tp.splits = TT < sms ? std::max(1, std::min(KB / 4, sms / TT)) : 1;
-    rc = bnt == 128 ? launch_t<128>(tp, tx, ta, TT * tp.splits, st)
-                    : launch_t<256>(tp, tx, ta, TT * tp.splits, st);
-    if (rc != SALR_OK) return rc;
-  }
+  // the layer kernel's parameters and scratch first: nothing may be queued between the
+  // t kernel and the layer kernel, which may start while t is still running
   PrefillParams pp{};
   pp.blob = h->blob;
   pp.offsets = h->offsets;
@@ -750,8 +740,36 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   // persistent: at most one CTA per SM, each taking units cta, cta + grid, ...
   pp.units = RT * TT * pp.splits;
   const int grid = std::min(pp.units, sms);
-  return bnt == 128 ? launch_prefill<128>(pp, tx, tb, tt, grid, st)
-                    : launch_prefill<256>(pp, tx, tb, tt, grid, st);
+  if (R > 0) {
+    rc = ensure_tscratch(h, M, st);
+    if (rc != SALR_OK) return rc;
+    if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
+    // B_cat^T in chunks of 64 ranks (ranks past R read as zero)
+    if (!make_map(&tb, B_cat, h->N, R, 64, 64)) return SALR_ERR_CUDA;
+    if (!make_map(&tt, h->tscr.T, 128, M, 64, bnt)) return SALR_ERR_CUDA;
+    TParams tp{};
+    tp.T = h->tscr.T;
+    tp.T32 = h->tscr.T32;
+    tp.counters = h->tscr.counters;
+    tp.status = h->status;
+    tp.M = static_cast<int>(M);
+    tp.Mp = static_cast<int>(Mp);
+    tp.R16 = R16;
+    tp.kblocks = KB;
+    tp.TT = TT;
+    // At least four K blocks per CTA: the split sums meet in L2, and a few blocks per CTA
+    // keep that reduction narrow.  The layer kernel launches as soon as the t kernel has
+    // started and needs t only for its adapter iterations, at the end of each unit; when
+    // the layer kernel leaves SMs free, the t kernel keeps to those, so that both run at
+    // once and no layer CTA waits for an SM.
+    const int free_sms = grid < sms ? sms - grid : sms;
+    tp.splits = std::max(1, std::min(KB / 4, free_sms / TT));
+    rc = bnt == 128 ? launch_t<128>(tp, tx, ta, TT * tp.splits, st)
+                    : launch_t<256>(tp, tx, ta, TT * tp.splits, st);
+    if (rc != SALR_OK) return rc;
+  }
+  return bnt == 128 ? launch_prefill<128>(pp, tx, tb, tt, grid, R > 0, st)
+                    : launch_prefill<256>(pp, tx, tb, tt, grid, R > 0, st);
 }
 
 int salr_linear_host(const void* X_host, int64_t M, salr_handle h, const void* A_cat,

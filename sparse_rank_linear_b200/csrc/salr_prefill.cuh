@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kPreThreads, 1)
       if (p.R16 > 0) prefetch_tmap(&tmT);
       uint32_t g = 0, gi = 0;
       RingCursor xc;
-      bool ok = true;
+      bool ok = true, t_ready = false;
       for (int u = cta; u < p.units && ok; u += G) {
         const PreUnit w = pre_unit(p, u);
         for (int it = 0; it < w.nk + w.nad; ++it, ++g, xc.next(SX)) {
@@ -253,6 +253,11 @@ __global__ void __launch_bounds__(kPreThreads, 1)
             pre_timeout(p.status, ctrl);
             ok = false;
             break;
+          }
+          if (it == w.nk && !t_ready) {
+            // t comes from the kernel launched just before this one, which may still run
+            griddep_wait();
+            t_ready = true;
           }
           mbar_arrive_expect_tx(&ctrl->xfull[s], L::kXbuf);
           if (it < w.nk)
@@ -506,6 +511,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   TCtrl* ctrl = reinterpret_cast<TCtrl*>(smem + kTStages * L::kStage);
+  // the layer kernel that follows may start now: it waits for this grid before reading t
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x % p.TT, sidx = blockIdx.x / p.TT;
   const int kb0 = static_cast<int>(static_cast<long long>(sidx) * p.kblocks / p.splits);
