@@ -87,6 +87,25 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def max_over_ranks(value, ws, device):
+    """The largest of every rank's value (a replica run ends when its slowest rank does);
+    the value itself with one rank.  ``device`` is where the process group's backend
+    keeps tensors: "cuda" for NCCL, "cpu" for gloo."""
+    if ws <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(ws, steps, tokens, total_ms):
+    """Tokens per second of the whole job: every rank processed ``steps`` calls of
+    ``tokens`` tokens, and the job took the slowest rank's ``total_ms``."""
+    return ws * steps * tokens / (total_ms * 1e-3)
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
@@ -476,11 +495,7 @@ def main():
         torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
-    total_ms = e_start.elapsed_time(e_stop)
-    if ws > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(e_start.elapsed_time(e_stop), ws, "cuda")
     status = handles[0].sync_status()
     if status != 0:
         raise RuntimeError(f"device status {salr.status_string(status)}")
@@ -524,11 +539,7 @@ def main():
         launch_host(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if ws > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws, "cuda")
 
     peaks, peak_src = measured_peaks()
     kern_ms = total_ms / args.steps  # mean launch duration over the back-to-back region
@@ -558,7 +569,7 @@ def main():
     roof["algorithmic_bytes"] = abytes
     roof["algorithmic_flops"] = aflops
 
-    value = ws * args.steps * M / (total_ms * 1e-3)
+    value = whole_job_rate(ws, args.steps, M, total_ms)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -572,7 +583,7 @@ def main():
                              f"({ncopies * per_copy / 2**20:.0f} MiB"
                              f"{' > 2x L2' if ncopies * per_copy > 2 * L2_BYTES else ', smaller than L2'})"},
             "roofline": roof,
-            "e2e": {"value": ws * e2e_steps * M / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": whole_job_rate(ws, e2e_steps, M, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N},
             "gpu_launches": args.steps * launches_per_call,
             "clocks": clocks.summary(),
