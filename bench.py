@@ -106,6 +106,42 @@ def whole_job_rate(ws, steps, tokens, total_ms):
     return ws * steps * tokens / (total_ms * 1e-3)
 
 
+def dense_lora_context(w_bits, x_bits, a_cat, b_cat, wl, M, steps, salr_total_ms):
+    """Time the unpruned layer, Y = X W^T + (X A_cat) B_cat, with dense bf16 W through
+    torch (cuBLAS), back to back over enough dense copies to exceed twice the L2.  Context
+    for the pages' speedup-over-dense-LoRA claim; not part of the library."""
+    import torch
+
+    def dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).cuda()
+
+    N, K = wl.N, wl.K
+    copies = max(1, min(16, int(np.ceil(2 * L2_BYTES / (2 * N * K)))))
+    Ws = [dev(w_bits) for _ in range(copies)]
+    A, B, X = dev(a_cat), dev(b_cat), dev(x_bits)
+
+    def step(i):
+        return torch.addmm((X @ A) @ B, X, Ws[i % copies].t())
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(2e9 * 40e-6 * steps) + 10_000_000)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del Ws
+    return {"ms_per_step": ms / steps, "tokens_per_s": steps * M / (ms * 1e-3),
+            "salr_speedup": ms / salr_total_ms, "dense_copies": copies,
+            "note": "torch bf16 (cuBLAS) X W^T + (X A_cat) B_cat with the unpruned W, "
+                    "same GPU and steps; context only"}
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     return ws, int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0"))
@@ -511,6 +547,10 @@ def main():
     torch.cuda.synchronize()
     per_launch_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
 
+    # ---------------- context only: the same layer with a dense bf16 W through cuBLAS
+    # (torch), Y = X W^T + (X A_cat) B_cat, the comparison the pages' speedup claim makes
+    dense_ctx = dense_lora_context(w_bits, x_bits, a_cat, b_cat, wl, M, args.steps, total_ms)
+
     # ---------------- end to end: host activations in, host outputs back, per step
     xh = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
@@ -588,7 +628,8 @@ def main():
             "gpu_launches": args.steps * launches_per_call,
             "clocks": clocks.summary(),
             "per_launch_event_ms_p10_p50_p90": [float(np.percentile(per_launch_ms, q))
-                                                for q in (10, 50, 90)]}
+                                                for q in (10, 50, 90)],
+            "dense_lora_context": dense_ctx}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         n, el = time_oracle(wl, M)
         line["cpu_baseline"] = {"value": n * M / el, "unit": "tokens/s", "cores": blas_threads(),

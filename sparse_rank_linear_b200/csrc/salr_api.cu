@@ -24,6 +24,9 @@ namespace {
 
 constexpr uint64_t kMagic = 0x53414c5257454754ull;  // "SALRWEGT"
 constexpr int kSmemLimit = 232448;  // B200 opt-in dynamic shared memory per CTA
+// token tiles from which salr_linear expands the weight once to a dense scratch instead
+// of once per token tile
+constexpr int kDenseMinTokenTiles = 2;
 
 // Split-K scratch of the prefill kernel: fp32 tile sums and arrival counts (grown on
 // demand, left zeroed by every call).
@@ -315,7 +318,8 @@ int launch_t(const TParams& p, const CUtensorMap& tx, const CUtensorMap& ta, int
 
 template <int BNT>
 int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb,
-                   const CUtensorMap& tt, int grid, bool after_t, cudaStream_t st) {
+                   const CUtensorMap& tt, const CUtensorMap& tw, int grid, bool after_t,
+                   cudaStream_t st) {
   using L = PrefillLayout<BNT>;
   // Ring sizes.  Among 5 or 4 decoded-tile slots and 4 to 2 X slots, take the layout
   // with the most compact-block slots (a multiple of the group count, at most kPreMaxC):
@@ -329,7 +333,16 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   // block it - 4, which saw block it - 4 - SA >= it - 2 SA consumed (the MMA consumes in
   // order), so the slot can never be two phases behind.
   int sa = 0, sx = 0, sc = 0;
-  for (int a = kPreGroups + 1; a >= kPreGroups; --a) {
+  if (p.dense) {
+    // dense weight tiles: no compact-block ring; the deepest decoded-tile ring, then
+    // as many X slots as fit
+    sa = kPreMaxA;
+    for (sx = kPreMaxX; sx >= 2; --sx)
+      if (L::smem_bytes(sa, sx, 0, p.cbuf) <= kSmemLimit) break;
+    if (sx < 2) return SALR_ERR_UNSUPPORTED;
+    sc = kPreGroups;  // placeholder so the check below passes; no slot is used
+  }
+  for (int a = kPreGroups + 1; a >= kPreGroups && !p.dense; --a) {
     for (int x = kPreMaxX; x >= 2; --x) {
       int c = (kSmemLimit - L::smem_bytes(a, x, 0, p.cbuf)) / p.cbuf;
       if (c > kPreMaxC) c = kPreMaxC;
@@ -344,7 +357,7 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   if (sc < kPreGroups) return SALR_ERR_UNSUPPORTED;
   p.sa = sa;
   p.sx = sx;
-  p.sc = sc;
+  p.sc = p.dense ? 0 : sc;
   const int smem = L::smem_bytes(p.sa, p.sx, p.sc, p.cbuf);
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -368,7 +381,7 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = after_t ? 1 : 0;
-  SALR_TRY(cudaLaunchKernelEx(&cfg, salr_prefill_kernel<BNT>, p, tx, tb, tt));
+  SALR_TRY(cudaLaunchKernelEx(&cfg, salr_prefill_kernel<BNT>, p, tx, tb, tt, tw));
   return SALR_OK;
 }
 
@@ -740,13 +753,37 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   // persistent: at most one CTA per SM, each taking units cta, cta + grid, ...
   pp.units = RT * TT * pp.splits;
   const int grid = std::min(pp.units, sms);
+  // With several token tiles, every weight block would be expanded once per token tile.
+  // Then the weight is expanded once into a dense scratch from the library pool (freed
+  // in stream order after the call), and the layer kernel takes its weight tiles from
+  // there by TMA.
+  CUtensorMap tw;
+  std::memset(&tw, 0, sizeof(tw));
+  uint8_t* wdense = nullptr;
+  pp.dense = TT >= kDenseMinTokenTiles ? 1 : 0;
+  if (pp.dense) {
+    const cudaError_t e =
+        dev_alloc_async(reinterpret_cast<void**>(&wdense), static_cast<size_t>(h->N) * h->K * 2, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    decode_kernel<<<static_cast<unsigned>(h->nblocks), kBlockRows, 0, st>>>(
+        h->blob, h->offsets, static_cast<int>(h->K), reinterpret_cast<uint16_t*>(wdense));
+    const cudaError_t le = cudaGetLastError();
+    if (le != cudaSuccess || !make_map(&tw, wdense, h->K, h->N, 64, 128)) {
+      cudaFreeAsync(wdense, st);
+      return le != cudaSuccess ? cuda_status(le) : SALR_ERR_CUDA;
+    }
+  }
+  auto release_dense = [&](int code) {
+    if (wdense) cudaFreeAsync(wdense, st);
+    return code;
+  };
   if (R > 0) {
     rc = ensure_tscratch(h, M, st);
-    if (rc != SALR_OK) return rc;
-    if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
+    if (rc != SALR_OK) return release_dense(rc);
+    if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return release_dense(SALR_ERR_CUDA);
     // B_cat^T in chunks of 64 ranks (ranks past R read as zero)
-    if (!make_map(&tb, B_cat, h->N, R, 64, 64)) return SALR_ERR_CUDA;
-    if (!make_map(&tt, h->tscr.T, 128, M, 64, bnt)) return SALR_ERR_CUDA;
+    if (!make_map(&tb, B_cat, h->N, R, 64, 64)) return release_dense(SALR_ERR_CUDA);
+    if (!make_map(&tt, h->tscr.T, 128, M, 64, bnt)) return release_dense(SALR_ERR_CUDA);
     TParams tp{};
     tp.T = h->tscr.T;
     tp.T32 = h->tscr.T32;
@@ -766,10 +803,11 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     tp.splits = std::max(1, std::min(KB / 4, free_sms / TT));
     rc = bnt == 128 ? launch_t<128>(tp, tx, ta, TT * tp.splits, st)
                     : launch_t<256>(tp, tx, ta, TT * tp.splits, st);
-    if (rc != SALR_OK) return rc;
+    if (rc != SALR_OK) return release_dense(rc);
   }
-  return bnt == 128 ? launch_prefill<128>(pp, tx, tb, tt, grid, R > 0, st)
-                    : launch_prefill<256>(pp, tx, tb, tt, grid, R > 0, st);
+  rc = bnt == 128 ? launch_prefill<128>(pp, tx, tb, tt, tw, grid, R > 0, st)
+                  : launch_prefill<256>(pp, tx, tb, tt, tw, grid, R > 0, st);
+  return release_dense(rc);
 }
 
 int salr_linear_host(const void* X_host, int64_t M, salr_handle h, const void* A_cat,

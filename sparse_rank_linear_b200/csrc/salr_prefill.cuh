@@ -53,6 +53,7 @@ struct PrefillParams {
   int TT;              // token tiles
   int splits;          // K splits per output tile
   int units;           // work units: weight row tiles x token tiles x K splits
+  int dense;           // 1: weight tiles come dense from tmW by TMA (no decoding)
   int cbuf;            // bytes of a compact-block slot, multiple of 1024
   int sc, sa, sx;      // ring depths: compact blocks, decoded tiles, X tiles
 };
@@ -136,7 +137,8 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     salr_prefill_kernel(const __grid_constant__ PrefillParams p,
                         const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmT) {
+                        const __grid_constant__ CUtensorMap tmT,
+                        const __grid_constant__ CUtensorMap tmW) {
   using L = PrefillLayout<BNT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(kPreThreads, 1)
       mbar_init(&ctrl->cempty[s], WPG);
     }
     for (int s = 0; s < SA; ++s) {
-      mbar_init(&ctrl->dec[s], WPG);
+      mbar_init(&ctrl->dec[s], p.dense ? 1 : WPG);  // dense: the producer's copy completes it
       mbar_init(&ctrl->aempty[s], 1);
     }
     for (int s = 0; s < SX; ++s) {
@@ -183,7 +185,43 @@ __global__ void __launch_bounds__(kPreThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem;
 
-  if (warp == 0) {
+  if (warp == 0 && p.dense) {
+    // ================================================================ dense weight-tile producer
+    // The weights were expanded to a dense [N x K] scratch before this kernel: each
+    // iteration's 128 x 64 tile (or adapter chunk of B_cat^T) goes by TMA straight into
+    // the decoded-tile slot, and its arrival completes the slot's barrier.
+    if (lane == 0) {
+      prefetch_tmap(&tmW);
+      if (p.R16 > 0) prefetch_tmap(&tmB);
+      RingCursor ac;
+      uint32_t g = 0, gi = 0;
+      bool ok = true;
+      for (int u = cta; u < p.units && ok; u += G) {
+        const PreUnit w = pre_unit(p, u);
+        for (int it = 0; it < w.nk + w.nad; ++it, ++g, ac.next(SA)) {
+          const uint32_t sa = ac.s;
+          if (!mbar_wait(&ctrl->aempty[sa], ac.ph ^ 1) || pre_aborted(ctrl)) {
+            pre_timeout(p.status, ctrl);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctrl->dec[sa], kPreTileBytes);
+          if (it < w.nk) {
+            tma_load_2d(abuf(sa), &tmW, (w.kb0 + it) * 64, w.i * 128, &ctrl->dec[sa]);
+          } else {
+            const int c = it - w.nk;
+            tma_load_2d(abuf(sa), &tmB, w.i * 128, c * 64, &ctrl->dec[sa]);
+            tma_load_2d(abuf(sa) + 8192, &tmB, w.i * 128 + 64, c * 64, &ctrl->dec[sa]);
+          }
+          gi = g + 1;
+        }
+      }
+      if (pre_aborted(ctrl)) {
+        for (uint32_t x = gi > static_cast<uint32_t>(SA) ? gi - SA : 0; x < gi; ++x)
+          mbar_wait(&ctrl->dec[x % SA], (x / SA) & 1);
+      }
+    }
+  } else if (warp == 0) {
     // ================================================================ compact-block producer
     // Each unit's block offsets sit in one of two shared buffers: the whole warp starts
     // the copy of the next unit's offsets (cp.async) before lane 0 issues this unit's
@@ -412,10 +450,10 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     const int dw = warp - 7;
     const int grp = dw / WPG, wg = dw % WPG;
     uint32_t* cs = reinterpret_cast<uint32_t*>(tables + grp * 4096);
-    if (p.R16 > 0 && wg == 0 && lane == 0) prefetch_tmap(&tmB);
+    if (p.R16 > 0 && wg == 0 && lane == 0 && !p.dense) prefetch_tmap(&tmB);
     uint32_t g = 0, adn = 0;
     RingCursor cc, ac;  // walked on every iteration, this group's or not
-    bool ok = true;
+    bool ok = !p.dense;  // dense weights need no decoding
     for (int u = cta; u < p.units && ok; u += G) {
       const PreUnit w = pre_unit(p, u);
       for (int it = 0; it < w.nk + w.nad; ++it, ++g, cc.next(SC), ac.next(SA)) {
