@@ -232,16 +232,20 @@ def test_linear_ragged_shapes(M, R):
     h.free()
 
 
-@pytest.mark.parametrize("R", [72, 128])
-def test_linear_several_units_per_cta_full_compare(R):
-    # 40 row tiles x 8 token tiles = 320 units on at most 148 persistent CTAs: every CTA
-    # runs two or three units back to back through the same rings, with both TMEM
-    # accumulators in use and two adapter chunks per unit (R = 72: the second partial)
-    wl = synth.Workload("multi", 5120, 256, (R,), (2048,))
-    w, x = synth.weight(wl), synth.activations(wl, 2048)
+@pytest.mark.parametrize("M", [2048, 1000])
+@pytest.mark.parametrize("R", [0, 72, 128])
+def test_linear_several_units_per_cta_full_compare(R, M):
+    # 40 row tiles x 8 (or 4) token tiles = 320 (160) units on at most 148 persistent CTAs:
+    # CTAs run two or three units back to back through the same rings, with both TMEM
+    # accumulators in use and two adapter chunks per unit (R = 72: the second partial).
+    # M = 2048 takes the dense-scratch weight path, M = 1000 the fused decode.
+    wl = synth.Workload("multi", 5120, 256, (R,) if R else (), (M,))
+    w, x = synth.weight(wl), synth.activations(wl, M)
     ad = synth.adapters(wl)
     h = salr.encode(to_dev(w), 0.5)
-    Y = salr.linear(to_dev(x), h, to_dev(ad[0][0]), to_dev(ad[0][1]))
+    A = to_dev(ad[0][0]) if R else None
+    B = to_dev(ad[0][1]) if R else None
+    Y = salr.linear(to_dev(x), h, A, B)
     assert h.sync_status() == 0
     wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
     assert_close(to_bits(Y), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad), f"multi R={R}")
