@@ -667,9 +667,9 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
 int salr_decode(salr_handle h, void* W_out, void* stream) {
   if (!valid_handle(h) || !W_out) return SALR_ERR_INVALID;
   if (!aligned16(W_out)) return SALR_ERR_UNSUPPORTED;
-  decode_kernel<<<static_cast<unsigned>(h->nblocks), kBlockRows, 0,
-                  static_cast<cudaStream_t>(stream)>>>(h->blob, h->offsets, static_cast<int>(h->K),
-                                                       static_cast<uint16_t*>(W_out));
+  expand_dense_kernel<<<static_cast<unsigned>(h->nblocks), 128, 0,
+                        static_cast<cudaStream_t>(stream)>>>(
+      h->blob, h->offsets, static_cast<int>(h->K), static_cast<uint16_t*>(W_out));
   SALR_TRY(cudaGetLastError());
   return SALR_OK;
 }
@@ -767,7 +767,7 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     const cudaError_t e =
         dev_alloc_async(reinterpret_cast<void**>(&wdense), static_cast<size_t>(h->N) * h->K * 2, st);
     if (e != cudaSuccess) return cuda_status(e);
-    decode_kernel<<<static_cast<unsigned>(h->nblocks), kBlockRows, 0, st>>>(
+    expand_dense_kernel<<<static_cast<unsigned>(h->nblocks), 128, 0, st>>>(
         h->blob, h->offsets, static_cast<int>(h->K), reinterpret_cast<uint16_t*>(wdense));
     const cudaError_t le = cudaGetLastError();
     if (le != cudaSuccess || !make_map(&tw, wdense, h->K, h->N, 64, 128)) {

@@ -1,10 +1,12 @@
-// salr_codec.cuh - GPU encoder and decoder of the SALR bitmap block format.
+// salr_codec.cuh - GPU encoder of the SALR bitmap block format, and the checks of a
+// serialised image.
 //
 // Encoding (SALR technical summary, Methodology 1 and 4): each row of W keeps its
 // `keep` entries of largest magnitude (ties to the lower column), the mask is stored as a
 // bitmap and the kept values as a compact array, both cut into 128 x 64 blocks that are
 // located through a per-block offset table.  The byte layout is the one written out in
-// include/salr.h.
+// include/salr.h.  The dense expansion (salr_decode) uses the layer kernels' expansion
+// functions and lives with them (expand_dense_kernel).
 #pragma once
 #include <cstdint>
 #include "sm100.cuh"
@@ -226,35 +228,6 @@ __global__ void __launch_bounds__(kBlockRows) encode_scatter_kernel(
   if (r == 0) {
     const uint32_t end = (offsets[b + 1] - offsets[b]) * 16;
     for (uint32_t p = kBitmapBytes + 2 * nnz; p < end; ++p) base[p] = 0;
-  }
-}
-
-// One CTA of 128 threads per block: expand to dense rows, pruned entries +0.0.
-__global__ void __launch_bounds__(kBlockRows) decode_kernel(const uint8_t* __restrict__ blob,
-                                                            const uint32_t* __restrict__ offsets,
-                                                            int K, uint16_t* __restrict__ out) {
-  __shared__ uint32_t sh[33];
-  const int b = blockIdx.x, nwords = K / 64;
-  const int i = b / nwords, j = b % nwords, r = threadIdx.x;
-  const uint8_t* base = blob + static_cast<size_t>(offsets[b]) * 16;
-  const uint64_t word = reinterpret_cast<const uint64_t*>(base)[r];
-  const uint32_t rstart = block_excl_scan(__popcll(word), sh, nullptr);
-  const uint16_t* vals = reinterpret_cast<const uint16_t*>(base + kBitmapBytes) + rstart;
-  uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(i * kBlockRows + r) * K +
-                                        j * kBlockCols);
-  int k = 0;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    uint32_t o[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int c = 8 * q + 2 * e;
-      uint32_t lo = 0, hi = 0;
-      if ((word >> c) & 1) lo = vals[k++];
-      if ((word >> (c + 1)) & 1) hi = vals[k++];
-      o[e] = lo | (hi << 16);
-    }
-    dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
