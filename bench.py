@@ -600,9 +600,9 @@ def main():
         launches_per_call = 1
     else:
         kname = f"salr_prefill_kernel<{128 if M <= 128 else 256}>"
-        # the layer kernel, the t = X A_cat kernel before it, and from five token tiles of
-        # 256 (M > 1024) the weight's expansion to a dense scratch before both
-        launches_per_call = 1 + (1 if R > 0 else 0) + (1 if M > 1024 else 0)
+        # the layer kernel, the t = X A_cat kernel before it, and from two token tiles of
+        # 256 (M > 256) the weight's expansion to a dense scratch before both
+        launches_per_call = 1 + (1 if R > 0 else 0) + (1 if M > 256 else 0)
     roof["traffic"] = traffic_for(kname, WORKLOAD if wl.sparsity == 0.5
                                   else f"{WORKLOAD} s={wl.sparsity:.6g}")
     roof["peak_source"] = peak_src

@@ -232,14 +232,14 @@ def test_linear_ragged_shapes(M, R):
     h.free()
 
 
-@pytest.mark.parametrize("M", [2048, 1000])
+@pytest.mark.parametrize("N,K,M", [(5120, 256, 2048), (20480, 128, 200)])
 @pytest.mark.parametrize("R", [0, 72, 128])
-def test_linear_several_units_per_cta_full_compare(R, M):
-    # 40 row tiles x 8 (or 4) token tiles = 320 (160) units on at most 148 persistent CTAs:
-    # CTAs run two or three units back to back through the same rings, with both TMEM
-    # accumulators in use and two adapter chunks per unit (R = 72: the second partial).
-    # M = 2048 takes the dense-scratch weight path, M = 1000 the fused decode.
-    wl = synth.Workload("multi", 5120, 256, (R,) if R else (), (M,))
+def test_linear_several_units_per_cta_full_compare(R, N, K, M):
+    # more units than the at most 148 persistent CTAs: 40 row tiles x 8 token tiles (the
+    # dense-scratch weight path) or 160 row tiles x 1 token tile (the fused decode).  CTAs
+    # run units back to back through the same rings, with both TMEM accumulators in use
+    # and two adapter chunks per unit (R = 72: the second partial)
+    wl = synth.Workload("multi", N, K, (R,) if R else (), (M,))
     w, x = synth.weight(wl), synth.activations(wl, M)
     ad = synth.adapters(wl)
     h = salr.encode(to_dev(w), 0.5)
