@@ -94,7 +94,7 @@ SALR_API int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, vo
 SALR_API int salr_decode(salr_handle h, void* W_out, void* stream);
 
 /*
- * salr_linear - Y = X (M (.) W)^T + (X A_cat) B_cat, one kernel launch.
+ * salr_linear - Y = X (M (.) W)^T + (X A_cat) B_cat.
  *
  * Defined by: technical summary, Methodology 3 (one concatenated adapter GEMM on the
  * shared input) and Methodology 4 (two-stage pipelined bitmap decoding + tensor-core
@@ -116,6 +116,13 @@ SALR_API int salr_decode(salr_handle h, void* W_out, void* stream);
  * The handle holds the split-K workspace used by this call; it is grown on demand
  * (a cudaMalloc) and is not safe to share between calls running concurrently on
  * different streams.
+ *
+ * Kernels: for M <= 64 one persistent kernel.  For larger M, a t = X A_cat kernel (when
+ * R > 0) and a persistent layer kernel that may start while t still runs.  From M > 256
+ * on, the weight is first expanded once to a dense bf16 scratch of N x K x 2 bytes, taken
+ * from the library's pool on `stream` and given back to it in stream order at the end
+ * of the call; the layer kernel then reads dense weight tiles instead of decoding them
+ * once per 256 tokens.
  *
  * For M <= 64 the call may start while the previous kernel on `stream` is still
  * running (programmatic dependent launch): before that kernel has completed it reads
