@@ -337,9 +337,11 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   // order), so the slot can never be two phases behind.
   int sa = 0, sx = 0, sc = 0;
   if (p.dense) {
-    // dense weight tiles: no compact-block ring; the deepest decoded-tile ring, then
-    // as many X slots as fit
-    sa = kPreMaxA;
+    // dense weight tiles: no compact-block ring.  Four weight-tile slots and as many X
+    // slots as fit (up to four): measured against 6 + 3 and 3 + 5 slots on B200, 4 + 4
+    // was the fastest (down_proj M = 4096: 380 against 404 and 393 us; up_proj M = 2048
+    // even)
+    sa = 4;
     for (sx = kPreMaxX; sx >= 2; --sx)
       if (L::smem_bytes(sa, sx, 0, p.cbuf) <= kSmemLimit) break;
     if (sx < 2) return SALR_ERR_UNSUPPORTED;
