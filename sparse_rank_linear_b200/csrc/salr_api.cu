@@ -301,6 +301,13 @@ int ensure_tscratch(salr_weight_s* h, int64_t M, cudaStream_t st) {
   return SALR_OK;
 }
 
+// CTAs of the dense expansion: five per SM (39 KB of shared memory each), each walking
+// several blocks so that staging the next one overlaps expanding this one.
+unsigned expand_grid(const salr_weight_s* h) {
+  const long long g = std::min<long long>(h->nblocks, 5ll * device_sms(h->device));
+  return static_cast<unsigned>(g < 1 ? 1 : g);
+}
+
 template <int BNT>
 int launch_t(const TParams& p, const CUtensorMap& tx, const CUtensorMap& ta, int grid,
              cudaStream_t st) {
@@ -670,9 +677,9 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
 int salr_decode(salr_handle h, void* W_out, void* stream) {
   if (!valid_handle(h) || !W_out) return SALR_ERR_INVALID;
   if (!aligned16(W_out)) return SALR_ERR_UNSUPPORTED;
-  expand_dense_kernel<<<static_cast<unsigned>(h->nblocks), 128, 0,
-                        static_cast<cudaStream_t>(stream)>>>(
-      h->blob, h->offsets, static_cast<int>(h->K), static_cast<uint16_t*>(W_out));
+  expand_dense_kernel<<<expand_grid(h), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      h->blob, h->offsets, static_cast<int>(h->K), static_cast<int>(h->nblocks),
+      static_cast<uint16_t*>(W_out));
   SALR_TRY(cudaGetLastError());
   return SALR_OK;
 }
@@ -770,8 +777,10 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     const cudaError_t e =
         dev_alloc_async(reinterpret_cast<void**>(&wdense), static_cast<size_t>(h->N) * h->K * 2, st);
     if (e != cudaSuccess) return cuda_status(e);
-    expand_dense_kernel<<<static_cast<unsigned>(h->nblocks), 128, 0, st>>>(
-        h->blob, h->offsets, static_cast<int>(h->K), reinterpret_cast<uint16_t*>(wdense));
+    expand_dense_kernel<<<expand_grid(h), 128, 0, st>>>(h->blob, h->offsets,
+                                                       static_cast<int>(h->K),
+                                                       static_cast<int>(h->nblocks),
+                                                       reinterpret_cast<uint16_t*>(wdense));
     const cudaError_t le = cudaGetLastError();
     if (le != cudaSuccess || !make_map(&tw, wdense, h->K, h->N, 64, 128)) {
       cudaFreeAsync(wdense, st);

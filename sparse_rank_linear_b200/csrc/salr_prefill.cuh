@@ -515,38 +515,55 @@ __global__ void __launch_bounds__(kPreThreads, 1)
 
 // ------------------------------------------------------------------------------------
 // Dense expansion of the whole encoded weight, [N x K] bf16 row-major with pruned entries
-// +0 (the layer's dense-scratch path and salr_decode).  One CTA of four warps per 128 x 64
-// block: the compact block is staged in shared memory with 16-byte loads, the warps build
+// +0 (the layer's dense-scratch path and salr_decode).  CTAs of four warps walk the
+// 128 x 64 blocks blockIdx.x, blockIdx.x + gridDim.x, ...: each block is staged in shared
+// memory by cp.async while the previous one is expanded (two buffers), the warps build
 // the chunk table and expand 32 rows each with the layer kernels' device functions, and
 // every 8-column chunk goes straight to global memory (8 lanes write one 128-byte row
-// segment).  About 21 KB of shared memory, so several blocks are in flight per SM.
+// segment).  About 39 KB of shared memory, so several CTAs share an SM.
 constexpr int kExpandMaxBlockBytes = kBitmapBytes + 2 * kBlockRows * kBlockCols;  // dense block
+constexpr int kExpandBuf = kExpandMaxBlockBytes + 32;
 __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __restrict__ blob,
                                                            const uint32_t* __restrict__ offsets,
-                                                           int K, uint16_t* __restrict__ out) {
-  __shared__ __align__(16) uint8_t cb[kExpandMaxBlockBytes + 32];
+                                                           int K, int nblocks,
+                                                           uint16_t* __restrict__ out) {
+  __shared__ __align__(16) uint8_t cb[2][kExpandBuf];
   __shared__ __align__(16) uint32_t cs[kBlockRows * 8];
   __shared__ uint2 nt[16];
-  const int b = blockIdx.x, nwords = K / 64;
-  const int i = b / nwords, j = b % nwords;
+  const int nwords = K / 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t o0 = offsets[b], n16 = offsets[b + 1] - o0;
-  const uint4* src = reinterpret_cast<const uint4*>(blob) + o0;
-  for (uint32_t k = threadIdx.x; k < n16; k += 128) reinterpret_cast<uint4*>(cb)[k] = src[k];
-  if (threadIdx.x < 2) reinterpret_cast<uint4*>(cb)[n16 + threadIdx.x] = make_uint4(0, 0, 0, 0);
   if (threadIdx.x < 16) nt[threadIdx.x] = nibble_entry(threadIdx.x);
-  __syncthreads();
-  build_chunk_table<32>(reinterpret_cast<const uint64_t*>(cb), cs, warp, lane);
-  __syncwarp();
-  const uint8_t* vals = cb + kBitmapBytes;
-  const int c = lane & 7;
-  uint16_t* dst = out + static_cast<size_t>(i) * kBlockRows * K + j * kBlockCols + c * 8;
+  auto stage = [&](int b, int buf) {
+    const uint32_t o0 = offsets[b], n16 = offsets[b + 1] - o0;
+    const uint4* src = reinterpret_cast<const uint4*>(blob) + o0;
+    for (uint32_t k = threadIdx.x; k < n16; k += 128)
+      cp_async16(reinterpret_cast<uint4*>(cb[buf]) + k, src + k);
+  };
+  int buf = 0;
+  if (static_cast<int>(blockIdx.x) < nblocks) stage(blockIdx.x, 0);
+  cp_async_commit();
+  for (int b = blockIdx.x; b < nblocks; b += gridDim.x, buf ^= 1) {
+    const int bn = b + gridDim.x;
+    if (bn < nblocks) stage(bn, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait_one();  // this block's copies (the older group) have landed
+    const uint32_t n16 = offsets[b + 1] - offsets[b];
+    if (threadIdx.x < 2) reinterpret_cast<uint4*>(cb[buf])[n16 + threadIdx.x] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+    const int i = b / nwords, j = b % nwords;
+    build_chunk_table<32>(reinterpret_cast<const uint64_t*>(cb[buf]), cs, warp, lane);
+    __syncwarp();
+    const uint8_t* vals = cb[buf] + kBitmapBytes;
+    const int c = lane & 7;
+    uint16_t* dst = out + static_cast<size_t>(i) * kBlockRows * K + j * kBlockCols + c * 8;
 #pragma unroll 2
-  for (int st = 0; st < 8; ++st) {
-    const int row = 32 * warp + 4 * st + (lane >> 3);
-    const uint32_t e = cs[row * 8 + c];
-    const ExpandIn in = expand_load(vals, e & 0xFFFFu, e >> 16, nt);
-    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(row) * K) = expand_compute(in);
+    for (int st = 0; st < 8; ++st) {
+      const int row = 32 * warp + 4 * st + (lane >> 3);
+      const uint32_t e = cs[row * 8 + c];
+      const ExpandIn in = expand_load(vals, e & 0xFFFFu, e >> 16, nt);
+      *reinterpret_cast<uint4*>(dst + static_cast<size_t>(row) * K) = expand_compute(in);
+    }
+    __syncthreads();  // this buffer and the chunk table are free for the next blocks
   }
 }
 
