@@ -326,6 +326,36 @@ int launch_t(const TParams& p, const CUtensorMap& tx, const CUtensorMap& ta, int
   return SALR_OK;
 }
 
+// Work split of the persistent layer kernel over `tiles` output tiles of `kb` K blocks
+// on `sms` CTAs.
+// * Fewer tiles than CTAs: every tile is split into as many K parts as fit in one round.
+// * Otherwise tiles are taken whole for as many full rounds as there are; the rem tiles
+//   of the last, partial round are each split into s K parts (s = 1 when that does not
+//   help), which takes ceil(rem s / sms) rounds of 1/s of a tile instead of one round of
+//   a whole tile.  s minimises that, ties going to fewer splits; a part keeps at least 4
+//   K blocks, and s stays at most 8, since each part adds an fp32 partial sum in L2.
+struct TileSplit {
+  int full, splits;
+};
+TileSplit tail_split(int tiles, int kb, int sms) {
+  if (tiles < sms) return TileSplit{0, std::max(1, std::min(kb, sms / tiles))};
+  const int full = tiles / sms * sms, rem = tiles - full;
+  TileSplit r{tiles, 1};
+  if (rem == 0) return r;
+  r.full = full;
+  const int smax = std::max(1, std::min(8, kb / 4));
+  long long best_num = (rem + sms - 1) / sms, best_den = 1;  // rounds / s, as a fraction
+  for (int s = 2; s <= smax; ++s) {
+    const long long rounds = (static_cast<long long>(rem) * s + sms - 1) / sms;
+    if (rounds * best_den < best_num * s) {
+      best_num = rounds;
+      best_den = s;
+      r.splits = s;
+    }
+  }
+  return r;
+}
+
 template <int BNT>
 int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb,
                    const CUtensorMap& tt, const CUtensorMap& tw, int grid, bool after_t,
@@ -734,7 +764,6 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   const int KB = static_cast<int>(h->K / 64);
   if (KB > kPreMaxKBlocks) return SALR_ERR_UNSUPPORTED;
   const int R16 = static_cast<int>((R + 15) / 16 * 16);
-  const int64_t Mp = (M + 3) / 4 * 4;  // row stride of the fp32 sums (16-byte rows)
   CUtensorMap tx, ta, tb, tt;
   std::memset(&ta, 0, sizeof(ta));
   std::memset(&tb, 0, sizeof(tb));
@@ -750,20 +779,22 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   pp.N = static_cast<int>(h->N);
   pp.K = static_cast<int>(h->K);
   pp.M = static_cast<int>(M);
-  pp.Mp = static_cast<int>(Mp);
   pp.R16 = R > 0 ? R16 : 0;
   pp.kblocks = KB;
   pp.TT = TT;
-  pp.splits = RT * TT < sms ? std::min(KB, sms / (RT * TT)) : 1;
   pp.cbuf = static_cast<int>((h->max16 * 16 + 32 + 1023) / 1024 * 1024);
+  const TileSplit ts = tail_split(RT * TT, KB, sms);
+  pp.full = ts.full;
+  pp.splits = ts.splits;
   if (pp.splits > 1) {
-    rc = ensure_workspace(h, static_cast<size_t>(h->N) * Mp, static_cast<size_t>(RT) * TT * 4, st);
+    const size_t ntail = static_cast<size_t>(RT) * TT - ts.full;
+    rc = ensure_workspace(h, ntail * 128 * bnt, ntail * 4, st);
     if (rc != SALR_OK) return rc;
     pp.acc = h->work.ws;
     pp.counters = h->work.counters;
   }
   // persistent: at most one CTA per SM, each taking units cta, cta + grid, ...
-  pp.units = RT * TT * pp.splits;
+  pp.units = ts.full + (RT * TT - ts.full) * ts.splits;
   const int grid = std::min(pp.units, sms);
   // With several token tiles, every weight block would be expanded once per token tile.
   // Then the weight is expanded once into a dense scratch from the library pool (freed
@@ -804,7 +835,6 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     tp.counters = h->tscr.counters;
     tp.status = h->status;
     tp.M = static_cast<int>(M);
-    tp.Mp = static_cast<int>(Mp);
     tp.R16 = R16;
     tp.kblocks = KB;
     tp.TT = TT;

@@ -7,7 +7,8 @@
 //   several splits, each adds its fp32 part into a sum in L2 (vector reductions), and the
 //   last split of a token tile to count itself in converts the sum and clears it.
 // * salr_prefill_kernel: persistent, one CTA per SM over the work units (128-row weight
-//   tile, token tile, K split).  Each 128 x 64 bitmap block arrives by one bulk copy and
+//   tile, token tile, K split).  Tiles are whole while every CTA gets one; the tiles of a
+//   last, partial round are split along K so that their parts even out over the CTAs.  Each 128 x 64 bitmap block arrives by one bulk copy and
 //   the matching X tile by tensor TMA.  Decoder warps expand the block into the
 //   128-byte-swizzled tile (stage 1, Methodology 4) with the same device functions as
 //   the small-M kernel; tcgen05 MMAs multiply it (stage 2).  The adapter's up projection
@@ -44,15 +45,15 @@ struct PrefillParams {
   const uint8_t* blob;
   const uint32_t* offsets;
   uint16_t* Y;
-  float* acc;          // [N x Mp] fp32 sums of split-K tiles (token-contiguous), zero between calls
-  uint32_t* counters;  // [RT x TT x 4] split arrivals per tile and 32-row quarter, zero between calls
+  float* acc;          // [split tiles][128 rows][BNT tokens] fp32 sums, zero between calls
+  uint32_t* counters;  // [split tiles][4] split arrivals per 32-row quarter, zero between calls
   int* status;
   int N, K, M, R16;
-  int Mp;              // M rounded up to 4: row stride of the fp32 sums
   int kblocks;         // K / 64
   int TT;              // token tiles
-  int splits;          // K splits per output tile
-  int units;           // work units: weight row tiles x token tiles x K splits
+  int full;            // tiles 0 .. full - 1 are whole units
+  int splits;          // K splits of each tile from `full` on (the split tiles)
+  int units;           // split tiles x splits + full (split units first)
   int dense;           // 1: weight tiles come dense from tmW by TMA (no decoding)
   int cbuf;            // bytes of a compact-block slot, multiple of 1024
   int sc, sa, sx;      // ring depths: compact blocks, decoded tiles, X tiles
@@ -106,18 +107,30 @@ struct RingCursor {
   }
 };
 
-// One work unit: weight row tile i, token tile j, K split s, and its K-block range.
+// One work unit: output tile t = (weight row tile i, token tile j), K split sidx of ns,
+// and its K-block range.  Tiles below p.full are whole; each later tile is cut into
+// p.splits consecutive units (the parts of one tile go to neighbouring CTAs).  The split
+// units come first, so that their partial sums meet while the whole tiles that follow
+// keep the tensor cores busy.
 struct PreUnit {
-  int i, j, sidx, kb0, nk, nad;  // nad: adapter iterations (64 ranks each) after the K blocks
+  int t, i, j, sidx, ns, kb0, nk, nad;  // nad: adapter iterations (64 ranks each) after the K blocks
 };
 __device__ __forceinline__ PreUnit pre_unit(const PrefillParams& p, int u) {
   PreUnit w;
-  w.j = u % p.TT;
-  const int rest = u / p.TT;
-  w.sidx = rest % p.splits;
-  w.i = rest / p.splits;
-  w.kb0 = static_cast<int>(static_cast<long long>(w.sidx) * p.kblocks / p.splits);
-  const int kb1 = static_cast<int>(static_cast<long long>(w.sidx + 1) * p.kblocks / p.splits);
+  const int nsu = p.units - p.full;  // split units
+  if (u >= nsu) {
+    w.t = u - nsu;
+    w.sidx = 0;
+    w.ns = 1;
+  } else {
+    w.t = p.full + u / p.splits;
+    w.sidx = u % p.splits;
+    w.ns = p.splits;
+  }
+  w.j = w.t % p.TT;
+  w.i = w.t / p.TT;
+  w.kb0 = static_cast<int>(static_cast<long long>(w.sidx) * p.kblocks / w.ns);
+  const int kb1 = static_cast<int>(static_cast<long long>(w.sidx + 1) * p.kblocks / w.ns);
   w.nk = kb1 - w.kb0;
   w.nad = (p.R16 > 0 && w.sidx == 0) ? (p.R16 + 63) / 64 : 0;
   return w;
@@ -382,7 +395,7 @@ __global__ void __launch_bounds__(kPreThreads, 1)
       const int mvalid = min(BNT, p.M - w.j * BNT);
       const size_t n = static_cast<size_t>(w.i) * 128 + r;
       const size_t row0 = static_cast<size_t>(w.j) * BNT;
-      if (p.splits == 1) {
+      if (w.ns == 1) {
         for (int c = 0; c < BNT; c += 16) {
           uint32_t v[16];
           tmem_ld16(acc + lane_base + c, v);
@@ -396,18 +409,19 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->accempty[b]);
       } else {
-        // split K: add into the tile's fp32 sum in L2 (row n, token-contiguous), count in
-        // per warp; the warp that arrives last for these 32 rows writes Y and clears both
-        float* sum = p.acc + n * p.Mp + row0;
+        // split K: add into the tile's fp32 sum in L2, count in per warp; the warp that
+        // arrives last for these 32 rows writes Y and clears both.  The sum is token-major
+        // ([token][128 rows]), so that every reduction, load and store of a warp covers
+        // one 128-byte line.
+        const size_t st = static_cast<size_t>(w.t - p.full);  // index among the split tiles
+        float* sum = p.acc + st * 128 * BNT + r;
         for (int c = 0; c < BNT; c += 16) {
           uint32_t v[16];
           tmem_ld16(acc + lane_base + c, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            if (c + e < mvalid)
-              red_add_v4f32(sum + c + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                            __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          for (int e = 0; e < 16; ++e)
+            if (c + e < mvalid) red_add_f32(sum + (c + e) * 128, __uint_as_float(v[e]));
         }
         tc_fence_before();
         __syncwarp();
@@ -415,28 +429,21 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         __threadfence();
         __syncwarp();
         uint32_t last = 0;
-        const size_t cidx = (static_cast<size_t>(w.i) * p.TT + w.j) * 4 + q;
-        if (lane == 0) last = atomicAdd(p.counters + cidx, 1u) == static_cast<uint32_t>(p.splits - 1);
+        const size_t cidx = st * 4 + q;
+        if (lane == 0) last = atomicAdd(p.counters + cidx, 1u) == static_cast<uint32_t>(w.ns - 1);
         if (__shfl_sync(0xffffffffu, last, 0)) {
           __threadfence();
           // 32 tokens per L2 round trip: a chunk's loads all go out before its stores
           for (int c0 = 0; c0 < mvalid; c0 += 32) {
-            float4 t4[8];
+            float tv[32];
 #pragma unroll
-            for (int gq = 0; gq < 8; ++gq)
-              t4[gq] = c0 + 4 * gq < mvalid
-                           ? __ldcg(reinterpret_cast<const float4*>(sum + c0 + 4 * gq))
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int e = 0; e < 32; ++e) tv[e] = c0 + e < mvalid ? __ldcg(sum + (c0 + e) * 128) : 0.f;
 #pragma unroll
-            for (int gq = 0; gq < 8; ++gq) {
-              const int c = c0 + 4 * gq;
-              if (c >= mvalid) continue;
-              const float tv[4] = {t4[gq].x, t4[gq].y, t4[gq].z, t4[gq].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                if (c + e < mvalid) Y[(row0 + c + e) * p.N + n] = __float2bfloat16_rn(tv[e]);
-              __stcg(reinterpret_cast<float4*>(sum + c), make_float4(0.f, 0.f, 0.f, 0.f));
-            }
+            for (int e = 0; e < 32; ++e)
+              if (c0 + e < mvalid) {
+                Y[(row0 + c0 + e) * p.N + n] = __float2bfloat16_rn(tv[e]);
+                __stcg(sum + (c0 + e) * 128, 0.f);
+              }
           }
           if (lane == 0) p.counters[cidx] = 0u;
         }
@@ -576,10 +583,10 @@ constexpr int kTStages = 4;
 
 struct TParams {
   uint16_t* T;         // [M x 128] bf16
-  float* T32;          // [128 x Mp] fp32 sums of K splits (token-contiguous), zero between calls
+  float* T32;          // [tokens x 128 ranks] fp32 sums of K splits (token-major), zero between calls
   uint32_t* counters;  // [TT x 4] split arrivals per token tile and 32-rank quarter
   int* status;
-  int M, Mp, R16, kblocks, TT, splits;
+  int M, R16, kblocks, TT, splits;
 };
 
 struct TCtrl {
@@ -700,17 +707,17 @@ __global__ void __launch_bounds__(kTThreads, 1)
           }
         }
       } else {
-        float* sum = p.T32 + static_cast<size_t>(r) * p.Mp + row0;
+        // token-major sums ([token][128 ranks]): a warp's 32 ranks of one token are one
+        // 128-byte line for every reduction, load and store
+        float* sum = p.T32 + row0 * 128 + r;
         for (int c = 0; c < BNT; c += 16) {
           uint32_t v[16];
           tmem_ld16(tmem + lane_base + c, v);
           tmem_ld_wait();
           if (r < p.R16) {
 #pragma unroll
-            for (int e = 0; e < 16; e += 4)
-              if (c + e < mvalid)
-                red_add_v4f32(sum + c + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                              __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+            for (int e = 0; e < 16; ++e)
+              if (c + e < mvalid) red_add_f32(sum + (c + e) * 128, __uint_as_float(v[e]));
           }
         }
         __threadfence();
@@ -722,22 +729,15 @@ __global__ void __launch_bounds__(kTThreads, 1)
           if (r < p.R16) {
             // 32 tokens per L2 round trip: a chunk's loads all go out before its stores
             for (int c0 = 0; c0 < mvalid; c0 += 32) {
-              float4 t4[8];
+              float tv[32];
 #pragma unroll
-              for (int g = 0; g < 8; ++g)
-                t4[g] = c0 + 4 * g < mvalid
-                            ? __ldcg(reinterpret_cast<const float4*>(sum + c0 + 4 * g))
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+              for (int e = 0; e < 32; ++e) tv[e] = c0 + e < mvalid ? __ldcg(sum + (c0 + e) * 128) : 0.f;
 #pragma unroll
-              for (int g = 0; g < 8; ++g) {
-                const int c = c0 + 4 * g;
-                if (c >= mvalid) continue;
-                const float tv[4] = {t4[g].x, t4[g].y, t4[g].z, t4[g].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  if (c + e < mvalid) T[(row0 + c + e) * 128 + r] = __float2bfloat16_rn(tv[e]);
-                __stcg(reinterpret_cast<float4*>(sum + c), make_float4(0.f, 0.f, 0.f, 0.f));
-              }
+              for (int e = 0; e < 32; ++e)
+                if (c0 + e < mvalid) {
+                  T[(row0 + c0 + e) * 128 + r] = __float2bfloat16_rn(tv[e]);
+                  __stcg(sum + (c0 + e) * 128, 0.f);
+                }
             }
           }
           if (lane == 0) p.counters[j * 4 + q] = 0u;

@@ -88,6 +88,9 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 
 // Add four fp32 values into 16-byte aligned global memory; the addition is performed in
 // L2 (no return value, relaxed, gpu scope).
+__device__ __forceinline__ void red_add_f32(float* p, float a) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
+}
 __device__ __forceinline__ void red_add_v4f32(float* p, float a, float b, float c, float d) {
   asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b),
                "f"(c), "f"(d)

@@ -252,6 +252,32 @@ def test_linear_several_units_per_cta_full_compare(R, N, K, M):
     h.free()
 
 
+@pytest.mark.parametrize("N,K,M", [(5120, 1024, 2048), (20480, 1024, 200)])
+@pytest.mark.parametrize("R", [0, 72])
+def test_linear_split_tail_tiles_full_compare(R, N, K, M):
+    # 320 tiles (dense-scratch path) or 160 tiles (fused decode) of 16 K blocks on 148
+    # SMs: the tiles of the last, partial round are split in four along K, their parts
+    # summed in the fp32 workspace, with the adapter on each tile's first part.  A second
+    # call, and a call with another token count, reuse the self-clearing workspace.
+    wl = synth.Workload("tail", N, K, (R,) if R else (), (M,))
+    w, x = synth.weight(wl), synth.activations(wl, M)
+    ad = synth.adapters(wl)
+    h = salr.encode(to_dev(w), 0.5)
+    A = to_dev(ad[0][0]) if R else None
+    B = to_dev(ad[0][1]) if R else None
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    expect, bound = oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad)
+    for call in range(2):
+        Y = salr.linear(to_dev(x), h, A, B)
+        assert h.sync_status() == 0
+        assert_close(to_bits(Y), expect, bound, f"tail R={R} call {call}")
+    m2 = M // 2 + 3
+    Y = salr.linear(to_dev(x[:m2]), h, A, B)
+    assert h.sync_status() == 0
+    assert_close(to_bits(Y), expect[:m2], bound[:m2], f"tail R={R} M={m2}")
+    h.free()
+
+
 @pytest.mark.parametrize("M", [256, 64])
 def test_identity_rows_reproduce_decoded_columns_bitexact(M):
     # X = rows of the identity, no adapter: every output is a single product
