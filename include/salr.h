@@ -115,7 +115,9 @@ SALR_API int salr_decode(salr_handle h, void* W_out, void* stream);
  *
  * The handle holds the split-K workspace used by this call; it is grown on demand
  * (a cudaMalloc) and is not safe to share between calls running concurrently on
- * different streams.
+ * different streams.  For M > 64 it holds one fp32 sum of 128 rows x 128 or 256 tokens
+ * per output tile that the layer kernel splits along K.  Those are the tiles of its
+ * last, partial round over the SMs, or every tile when there are fewer tiles than SMs.
  *
  * Kernels: for M <= 64 one persistent kernel.  For larger M, a t = X A_cat kernel (when
  * R > 0) and a persistent layer kernel that may start while t still runs.  From M > 256
