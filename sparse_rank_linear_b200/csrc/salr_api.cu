@@ -26,9 +26,10 @@ constexpr uint64_t kMagic = 0x53414c5257454754ull;  // "SALRWEGT"
 constexpr int kSmemLimit = 232448;  // B200 opt-in dynamic shared memory per CTA
 // Token tiles (of 256) from which salr_linear expands the weight once to a dense scratch
 // instead of once per token tile.  Measured on B200 with both paths built: with one token
-// tile the fused decode is faster (down_proj M = 128: 55 against 70 us; up_proj M = 256:
-// 72 against 76 us); from two the dense scratch wins (up_proj M = 512: 104 against 128 us;
-// down_proj M = 512: 107 against 110 us; up_proj M = 1024: 134 against 183 us).
+// tile the fused decode is faster (down_proj M = 128: 51.7 against 68.0 us; up_proj
+// M = 256: 70.7 against 74.1 us; large M = 128: 167 against 258 us); from two the dense
+// scratch wins (up_proj M = 512: 104 against 128 us; down_proj M = 512: 107 against
+// 110 us; up_proj M = 1024: 134 against 183 us).
 constexpr int kDenseMinTokenTiles = 2;
 
 // Split-K scratch of the prefill kernel: fp32 tile sums and arrival counts (grown on
