@@ -4,8 +4,9 @@
 // * salr_t_kernel: t = X A_cat, the concatenated adapter's down projection (SALR
 //   technical summary, Methodology 3), computed once per call on the tensor cores and
 //   rounded once to bf16 into a [M x 128] scratch.  Grid: token tiles x K splits.  With
-//   several splits, each adds its fp32 part into a sum in L2 (vector reductions), and the
-//   last split of a token tile to count itself in converts the sum and clears it.
+//   several splits, each adds its fp32 part into a token-major sum in L2 (coalesced
+//   reductions), and the last split of a token tile to count itself in converts the sum
+//   and clears it.
 // * salr_prefill_kernel: persistent, one CTA per SM over the work units (128-row weight
 //   tile, token tile, K split).  Tiles are whole while every CTA gets one; the tiles of a
 //   last, partial round are split along K so that their parts even out over the CTAs.  Each 128 x 64 bitmap block arrives by one bulk copy and
