@@ -173,6 +173,42 @@ SALR_API int salr_linear_host(const void* X_host, int64_t M, salr_handle h, cons
 SALR_API int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, const void* A_cat,
                                  const void* B_cat, int64_t R, void* Y, void* stream);
 
+/*
+ * salr_linear_plan - how salr_linear runs a call, without running it.
+ *
+ * No counterpart in the SALR paper: a planning query of this library.  It reports the
+ * kernels, tiles and work split salr_linear chooses for M tokens and R adapter ranks on
+ * an N x K weight.  It also reports the device memory that call needs beyond its
+ * arguments: the transient dense weight scratch and the fp32 split sums held in the
+ * handle's workspace.
+ *
+ * N, K   the weight's shape, with the rules of salr_encode.
+ * M, R   as for salr_linear.
+ * sms    the device's SM count (> 0).  With 0, the current CUDA device's count is used.
+ * out    filled on success.
+ *
+ * Host logic only: nothing is allocated or launched, so with sms > 0 it needs no GPU.
+ * Returns SALR_ERR_INVALID for a NULL `out`, M < 1, R < 0 or sms < 0.  Returns
+ * SALR_ERR_UNSUPPORTED for shapes, M or R that salr_linear rejects, and SALR_ERR_CUDA
+ * when sms == 0 and there is no device.
+ */
+typedef struct {
+  int32_t path;        /* 0: one persistent kernel (M <= 64); 1: t kernel + fused decode and
+                          GEMM; 2: weight expansion + t kernel + GEMM on dense weight tiles */
+  int32_t kernels;     /* kernel launches per call */
+  int32_t token_tile;  /* tokens per MMA tile: 16, 32, 64, 128 or 256 */
+  int32_t grid;        /* CTAs of the layer kernel, at most one per SM */
+  int32_t units;       /* work units of the layer kernel: 128 x 64 weight blocks (path 0),
+                          else whole tiles plus the K parts of split tiles */
+  int32_t tiles;       /* output tiles of 128 weight rows x token_tile (paths 1, 2) */
+  int32_t whole_tiles; /* tiles computed whole (paths 1, 2) */
+  int32_t splits;      /* K parts of each remaining tile (paths 1, 2; 1 = none) */
+  int64_t split_sum_bytes;     /* fp32 sums of the split tiles in the handle's workspace */
+  int64_t dense_scratch_bytes; /* transient dense bf16 weight (path 2), else 0 */
+} salr_plan;
+SALR_API int salr_linear_plan(int64_t N, int64_t K, int64_t M, int64_t R, int32_t sms,
+                              salr_plan* out);
+
 /* salr_free - release a handle and every device buffer it owns.  Freeing an unknown or
  * already freed handle returns SALR_ERR_INVALID and touches nothing. */
 SALR_API int salr_free(salr_handle h);

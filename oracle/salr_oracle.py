@@ -10,11 +10,11 @@ Representation for Efficient Fine-Tuning of Large Language Models", gist.science
 technical summary, and the authors' abstract on the scholarfeed author page):
 
 * ``magnitude_mask`` / ``prune``: static magnitude pruning of the frozen base weight
-  W0 to a given sparsity, A and B left dense (Technical Summary, Methodology 1; abstract
-  "50% sparsity").  Granularity per output row, ties to the lower column index.
+  W0 to a given sparsity, A and B left dense (Technical Summary, Methodology 1; the
+  abstract's sparsity of one half).  Granularity per output row, ties to the lower column index.
 * ``encode_format`` / ``decode_format``: the bitmap-plus-compact-values storage with a
-  per-block offset table (Methodology 4, "Bitmap Encoding" and "Stage 1 ... lookup
-  tables").  The on-device block layout is this library's own definition and is
+  per-block offset table (Methodology 4, "Bitmap Encoding", and its first pipeline stage,
+  which reads the bitmaps through lookup tables).  The on-device block layout is this library's own definition and is
   written out in ``include/salr.h``; the oracle follows that definition literally.
 * ``linear``: Y = X (M (.) W)^T + sum_i (X A_i) B_i, the layer a SALR model runs at
   inference (Methodology 3, "Adapter Concatenation", with the pruned base of

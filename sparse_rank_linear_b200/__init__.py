@@ -5,8 +5,8 @@ bitmap plus compact values; one hand-written CUDA kernel per call.  The Python l
 a ctypes binding of the C ABI in ``include/salr.h``; importing it does not load the
 library, the first call does (and fails loudly if it has not been built).
 """
-from .binding import (SIGNATURES, SalrError, Weight, encode, linear, linear_host, load,
-                      load_library, residual_adapter, status_string)
+from .binding import (SIGNATURES, SalrError, SalrPlan, Weight, encode, linear, linear_host,
+                      load, load_library, plan, residual_adapter, status_string)
 
-__all__ = ["SIGNATURES", "SalrError", "Weight", "encode", "linear", "linear_host", "load",
-           "load_library", "residual_adapter", "status_string"]
+__all__ = ["SIGNATURES", "SalrError", "SalrPlan", "Weight", "encode", "linear", "linear_host",
+           "load", "load_library", "plan", "residual_adapter", "status_string"]

@@ -21,6 +21,15 @@ SALR_ERR_TIMEOUT = 5
 
 # name -> (restype, argtypes) for every entry point declared in include/salr.h
 _P, _I64, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
+
+
+class SalrPlan(ctypes.Structure):
+    """salr_plan of include/salr.h (field order and types as declared there)."""
+    _fields_ = [("path", ctypes.c_int32), ("kernels", ctypes.c_int32),
+                ("token_tile", ctypes.c_int32), ("grid", ctypes.c_int32),
+                ("units", ctypes.c_int32), ("tiles", ctypes.c_int32),
+                ("whole_tiles", ctypes.c_int32), ("splits", ctypes.c_int32),
+                ("split_sum_bytes", ctypes.c_int64), ("dense_scratch_bytes", ctypes.c_int64)]
 SIGNATURES = {
     "salr_encode": (_I, [_P, _I64, _I64, _F, _P, ctypes.POINTER(_P)]),
     "salr_decode": (_I, [_P, _P, _P]),
@@ -36,6 +45,7 @@ SIGNATURES = {
     "salr_save": (_I, [_P, _P, _I64, _P]),
     "salr_load": (_I, [_P, _I64, _P, ctypes.POINTER(_P)]),
     "salr_residual_adapter": (_I, [_P, _P, _I64, _P, _I64, _I, _P, _P, _P, _P]),
+    "salr_linear_plan": (_I, [_I64, _I64, _I64, _I64, ctypes.c_int32, ctypes.POINTER(SalrPlan)]),
     "salr_sync_status": (_I, [_P, _P]),
     "salr_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -254,3 +264,11 @@ def linear_host(X_host, weight: Weight, A_cat, B_cat, Y_host, stream=None):
         _ptr(X_host), X_host.shape[0], weight.handle, _ptr(A_cat), _ptr(B_cat), R, _ptr(Y_host),
         _stream_ptr(stream)))
     return Y_host
+
+
+def plan(N: int, K: int, M: int, R: int = 0, sms: int = 0) -> dict:
+    """salr_linear_plan: the kernels, tiles, work split and extra device memory that
+    salr_linear uses for M tokens on an N x K weight (sms = 0: the current device's)."""
+    out = SalrPlan()
+    _check("salr_linear_plan", load_library().salr_linear_plan(N, K, M, R, sms, ctypes.byref(out)))
+    return {name: getattr(out, name) for name, _ in SalrPlan._fields_}

@@ -329,12 +329,15 @@ int launch_t(const TParams& p, const CUtensorMap& tx, const CUtensorMap& ta, int
 
 // Work split of the persistent layer kernel over `tiles` output tiles of `kb` K blocks
 // on `sms` CTAs.
-// * Fewer tiles than CTAs: every tile is split into as many K parts as fit in one round.
-// * Otherwise tiles are taken whole for as many full rounds as there are; the rem tiles
-//   of the last, partial round are each split into s K parts (s = 1 when that does not
-//   help), which takes ceil(rem s / sms) rounds of 1/s of a tile instead of one round of
-//   a whole tile.  s minimises that, ties going to fewer splits; a part keeps at least 4
-//   K blocks, and s stays at most 8, since each part adds an fp32 partial sum in L2.
+// * Fewer tiles than CTAs: every tile is split along K into as many parts as fit in one
+//   round.
+// * Otherwise the tiles of the full rounds stay whole, and each CTA takes the same number
+//   of them.  The rem tiles of the last, partial round are split into s parts of at most
+//   ceil(kb / s) blocks.  The parts run first, so a CTA takes at most ceil(rem s / sms)
+//   of them.  s minimises that bound on a CTA's extra blocks, ceil(rem s / sms)
+//   ceil(kb / s), against kb for one whole tile; ties go to fewer splits.  A part keeps
+//   at least 4 K blocks, and s stays at most 8, since each part adds an fp32 partial sum
+//   in L2.
 struct TileSplit {
   int full, splits;
 };
@@ -345,16 +348,56 @@ TileSplit tail_split(int tiles, int kb, int sms) {
   if (rem == 0) return r;
   r.full = full;
   const int smax = std::max(1, std::min(8, kb / 4));
-  long long best_num = (rem + sms - 1) / sms, best_den = 1;  // rounds / s, as a fraction
+  long long best = kb;  // one whole tile
   for (int s = 2; s <= smax; ++s) {
-    const long long rounds = (static_cast<long long>(rem) * s + sms - 1) / sms;
-    if (rounds * best_den < best_num * s) {
-      best_num = rounds;
-      best_den = s;
+    const long long parts = (static_cast<long long>(rem) * s + sms - 1) / sms;
+    const long long cost = parts * ((kb + s - 1) / s);
+    if (cost < best) {
+      best = cost;
       r.splits = s;
     }
   }
   return r;
+}
+
+// The launch plan of salr_linear for M tokens on `sms` SMs: the call itself and
+// salr_linear_plan both take their decisions from here.  N and K are valid shapes
+// (check_shape); for M > 64, K stays within kPreMaxKBlocks blocks of 64.
+struct LinearPlan {
+  int path;     // 0 small-M kernel, 1 t + fused decode/GEMM, 2 expansion + t + dense GEMM
+  int kernels;  // launches per call
+  int bnt;      // tokens per MMA tile
+  int RT, KB, TT, tiles;
+  int full, splits;  // whole tiles; K parts of each later tile
+  int units, grid;
+  int64_t sum_bytes, dense_bytes;
+};
+LinearPlan plan_linear(int64_t N, int64_t K, int64_t M, int64_t R, int sms) {
+  LinearPlan p{};
+  p.RT = static_cast<int>(N / 128);
+  p.KB = static_cast<int>(K / 64);
+  if (M <= 64) {
+    p.path = 0;
+    p.kernels = 1;
+    p.bnt = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+    p.units = p.RT * p.KB;  // 128 x 64 blocks, split evenly over the CTAs
+    p.grid = std::min(p.units, sms);
+    return p;
+  }
+  p.bnt = M <= 128 ? 128 : 256;
+  p.TT = static_cast<int>((M + p.bnt - 1) / p.bnt);
+  p.tiles = p.RT * p.TT;
+  const TileSplit ts = tail_split(p.tiles, p.KB, sms);
+  p.full = ts.full;
+  p.splits = ts.splits;
+  p.units = ts.full + (p.tiles - ts.full) * ts.splits;
+  p.grid = std::min(p.units, sms);
+  const bool dense = p.TT >= kDenseMinTokenTiles;
+  p.path = dense ? 2 : 1;
+  p.kernels = 1 + (R > 0 ? 1 : 0) + (dense ? 1 : 0);
+  p.sum_bytes = p.splits > 1 ? static_cast<int64_t>(p.tiles - p.full) * 128 * p.bnt * 4 : 0;
+  p.dense_bytes = dense ? N * K * 2 : 0;
+  return p;
 }
 
 template <int BNT>
@@ -715,6 +758,34 @@ int salr_decode(salr_handle h, void* W_out, void* stream) {
   return SALR_OK;
 }
 
+int salr_linear_plan(int64_t N, int64_t K, int64_t M, int64_t R, int32_t sms, salr_plan* out) {
+  if (!out || M < 1 || R < 0 || sms < 0) return SALR_ERR_INVALID;
+  const int shape = check_shape(N, K);
+  if (shape != SALR_OK) return shape;
+  if (R % 8 != 0 || R > 128 || M > (1ll << 24)) return SALR_ERR_UNSUPPORTED;
+  if (sms == 0) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      return SALR_ERR_CUDA;
+    }
+    sms = n;
+  }
+  const LinearPlan p = plan_linear(N, K, M, R, sms);
+  out->path = p.path;
+  out->kernels = p.kernels;
+  out->token_tile = p.bnt;
+  out->grid = p.grid;
+  out->units = p.units;
+  out->tiles = p.tiles;
+  out->whole_tiles = p.path == 0 ? 0 : p.splits == 1 ? p.tiles : p.full;
+  out->splits = p.path == 0 ? 1 : p.splits;
+  out->split_sum_bytes = p.sum_bytes;
+  out->dense_scratch_bytes = p.dense_bytes;
+  return SALR_OK;
+}
+
 int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, const void* B_cat,
                 int64_t R, void* Y, void* stream) {
   int rc = check_linear_args(X, M, h, A_cat, B_cat, R, Y);
@@ -758,12 +829,10 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     return rc;
   }
   // prefill shapes: t = X A_cat once (own kernel), then the fused decode + GEMM
-  const int bnt = M <= 128 ? 128 : 256;
   const int sms = device_sms(h->device);
-  const int TT = static_cast<int>((M + bnt - 1) / bnt);
-  const int RT = static_cast<int>(h->N / 128);
-  const int KB = static_cast<int>(h->K / 64);
-  if (KB > kPreMaxKBlocks) return SALR_ERR_UNSUPPORTED;
+  if (h->K / 64 > kPreMaxKBlocks) return SALR_ERR_UNSUPPORTED;
+  const LinearPlan pl = plan_linear(h->N, h->K, M, R, sms);
+  const int bnt = pl.bnt, TT = pl.TT, KB = pl.KB;
   const int R16 = static_cast<int>((R + 15) / 16 * 16);
   CUtensorMap tx, ta, tb, tt;
   std::memset(&ta, 0, sizeof(ta));
@@ -784,19 +853,18 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   pp.kblocks = KB;
   pp.TT = TT;
   pp.cbuf = static_cast<int>((h->max16 * 16 + 32 + 1023) / 1024 * 1024);
-  const TileSplit ts = tail_split(RT * TT, KB, sms);
-  pp.full = ts.full;
-  pp.splits = ts.splits;
+  pp.full = pl.full;
+  pp.splits = pl.splits;
   if (pp.splits > 1) {
-    const size_t ntail = static_cast<size_t>(RT) * TT - ts.full;
+    const size_t ntail = static_cast<size_t>(pl.tiles - pl.full);
     rc = ensure_workspace(h, ntail * 128 * bnt, ntail * 4, st);
     if (rc != SALR_OK) return rc;
     pp.acc = h->work.ws;
     pp.counters = h->work.counters;
   }
   // persistent: at most one CTA per SM, each taking units cta, cta + grid, ...
-  pp.units = ts.full + (RT * TT - ts.full) * ts.splits;
-  const int grid = std::min(pp.units, sms);
+  pp.units = pl.units;
+  const int grid = pl.grid;
   // With several token tiles, every weight block would be expanded once per token tile.
   // Then the weight is expanded once into a dense scratch from the library pool (freed
   // in stream order after the call), and the layer kernel takes its weight tiles from
@@ -804,7 +872,7 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   CUtensorMap tw;
   std::memset(&tw, 0, sizeof(tw));
   uint8_t* wdense = nullptr;
-  pp.dense = TT >= kDenseMinTokenTiles ? 1 : 0;
+  pp.dense = pl.path == 2 ? 1 : 0;
   if (pp.dense) {
     const cudaError_t e =
         dev_alloc_async(reinterpret_cast<void**>(&wdense), static_cast<size_t>(h->N) * h->K * 2, st);

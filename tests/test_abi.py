@@ -150,3 +150,109 @@ def test_load_rejects_bad_images_on_host(lib):
     # shapes outside the rules are unsupported, as for salr_encode
     assert load(pk(n=100)) == 2
     assert load(pk(k=96)) == 2
+
+
+# ---------------------------------------------------------------- launch plan (host logic)
+def _plan(N, K, M, R=0, sms=148):
+    return binding.plan(N, K, M, R, sms)
+
+
+def test_linear_plan_of_the_workloads(lib):
+    # hand-derived: tiles = N/128 x ceil(M / token tile); with at least as many tiles as
+    # SMs the full rounds stay whole and the rem left over are split in s parts, s
+    # minimising ceil(rem s / 148) / s
+    q16 = _plan(4096, 4096, 16, 80)
+    assert (q16["path"], q16["kernels"], q16["token_tile"], q16["units"], q16["grid"]) == \
+        (0, 1, 16, 32 * 64, 148)
+    assert _plan(256, 256, 16, 8)["grid"] == 8  # tiny: 2 x 4 blocks
+    d128 = _plan(4096, 11008, 128, 128)  # 32 tiles < 148 SMs: each split in 148 // 32 = 4
+    assert (d128["path"], d128["kernels"], d128["tiles"], d128["whole_tiles"], d128["splits"],
+            d128["units"], d128["grid"]) == (1, 2, 32, 0, 4, 128, 128)
+    assert d128["split_sum_bytes"] == 32 * 128 * 128 * 4
+    assert d128["dense_scratch_bytes"] == 0
+    up = _plan(11008, 4096, 2048, 96)  # 688 tiles = 4 x 148 + 96; 96 x 3 = 288 -> 2 rounds of 1/3
+    assert (up["path"], up["kernels"], up["token_tile"], up["tiles"], up["whole_tiles"],
+            up["splits"], up["units"]) == (2, 3, 256, 688, 592, 3, 592 + 288)
+    assert up["split_sum_bytes"] == 96 * 128 * 256 * 4
+    assert up["dense_scratch_bytes"] == 11008 * 4096 * 2
+    dn = _plan(4096, 11008, 4096, 128)  # 512 = 3 x 148 + 68; 68 x 2 = 136 -> 1 round of 1/2
+    assert (dn["tiles"], dn["whole_tiles"], dn["splits"], dn["units"]) == (512, 444, 2, 580)
+    lg = _plan(28672, 8192, 8192, 96)  # 7168 = 48 x 148 + 64
+    assert (lg["tiles"], lg["whole_tiles"], lg["splits"]) == (7168, 7104, 2)
+    l128 = _plan(28672, 8192, 128, 96)  # 224 = 148 + 76; 76 x 7 = 532 -> 4 rounds of 1/7
+    assert (l128["path"], l128["whole_tiles"], l128["splits"], l128["units"]) == (1, 148, 7, 680)
+    u256 = _plan(11008, 4096, 256, 96)  # 86 tiles, 148 // 86 = 1: nothing split
+    assert (u256["tiles"], u256["whole_tiles"], u256["splits"], u256["grid"]) == (86, 86, 1, 86)
+    assert u256["split_sum_bytes"] == 0
+    # no adapter: no t kernel
+    assert _plan(11008, 4096, 2048, 0)["kernels"] == 2
+    assert _plan(4096, 11008, 128, 0)["kernels"] == 1
+    # whole rounds only: nothing split
+    full = _plan(128 * 148, 4096, 256)
+    assert (full["tiles"], full["whole_tiles"], full["splits"]) == (148, 148, 1)
+
+
+def _makespan(p, KB):
+    """Largest number of K blocks one CTA of the persistent layer kernel multiplies, with
+    CTA c taking units c, c + grid, ... and the split units first."""
+    s, tiles, whole = p["splits"], p["tiles"], p["whole_tiles"]
+    nsu = (tiles - whole) * s if s > 1 else 0
+    load = [0] * p["grid"]
+    for u in range(p["units"]):
+        if u < nsu:
+            i = u % s
+            blocks = (i + 1) * KB // s - i * KB // s
+        else:
+            blocks = KB
+        load[u % p["grid"]] += blocks
+    return max(load)
+
+
+@pytest.mark.parametrize("sms", [148, 132, 64])
+def test_linear_plan_split_never_lengthens_a_cta(lib, sms):
+    rng = np.random.default_rng(7)
+    for _ in range(150):
+        RT = int(rng.integers(1, 400))
+        KB = int(rng.integers(1, 200))
+        M = int(rng.integers(65, 20000))
+        p = _plan(128 * RT, 64 * KB, M, 0, sms)
+        tiles = p["tiles"]
+        assert tiles == RT * -(-M // p["token_tile"])
+        s = p["splits"]
+        assert p["units"] == p["whole_tiles"] + (tiles - p["whole_tiles"]) * s
+        assert p["grid"] == min(p["units"], sms)
+        if s > 1:
+            if tiles >= sms:
+                # only the last, partial round is split, into at most 8 parts of >= 4 blocks
+                assert p["whole_tiles"] == tiles // sms * sms < tiles
+                assert s <= 8 and KB // s >= 4
+            else:
+                assert p["whole_tiles"] == 0 and s == min(KB, sms // tiles)
+        else:
+            assert p["whole_tiles"] == tiles
+        # against taking every tile whole: never longer, and shorter when s > 1
+        whole = {"splits": 1, "tiles": tiles, "whole_tiles": tiles, "units": tiles,
+                 "grid": min(tiles, sms)}
+        assert _makespan(p, KB) <= _makespan(whole, KB)
+        # a CTA takes tiles // sms whole tiles and at most ceil(rem s / sms) parts of at
+        # most ceil(KB / s) blocks
+        if s > 1 and tiles >= sms:
+            rem = tiles - p["whole_tiles"]
+            assert _makespan(p, KB) <= tiles // sms * KB + -(-rem * s // sms) * -(-KB // s)
+        if s > 1:
+            assert _makespan(p, KB) < _makespan(whole, KB)
+
+
+def test_linear_plan_rejects_bad_arguments(lib):
+    out = binding.SalrPlan()
+    f = lib.salr_linear_plan
+    assert f(4096, 4096, 0, 0, 148, ctypes.byref(out)) == 1      # M < 1
+    assert f(4096, 4096, 16, -8, 148, ctypes.byref(out)) == 1    # R < 0
+    assert f(4096, 4096, 16, 0, -1, ctypes.byref(out)) == 1      # sms < 0
+    assert f(4096, 4096, 16, 0, 148, None) == 1                  # no output
+    assert f(4096, 4096, 16, 12, 148, ctypes.byref(out)) == 2    # R % 8
+    assert f(4096, 4096, 16, 136, 148, ctypes.byref(out)) == 2   # R > 128
+    assert f(4000, 4096, 16, 0, 148, ctypes.byref(out)) == 2     # N % 128
+    assert f(4096, 4000, 16, 0, 148, ctypes.byref(out)) == 2     # K % 64
+    assert f(4096, 64 * 513, 512, 0, 148, ctypes.byref(out)) == 2  # K past the layer kernels
+    assert f(4096, 4096, (1 << 24) + 1, 0, 148, ctypes.byref(out)) == 2
