@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -181,7 +182,7 @@ cudaError_t alloc_handle_memory(salr_weight_s* h, int64_t blob_capacity, cudaStr
 }
 
 int device_sms(int dev) {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];  // zero-initialised: not looked up yet
   if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
   int n = 0;
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -313,7 +314,7 @@ template <int BNT>
 int launch_t(const TParams& p, const CUtensorMap& tx, const CUtensorMap& ta, int grid,
              cudaStream_t st) {
   constexpr int smem = TLayout<BNT>::kSmemBytes;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
@@ -445,7 +446,7 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   p.sx = sx;
   p.sc = p.dense ? 0 : sc;
   const int smem = L::smem_bytes(p.sa, p.sx, p.sc, p.cbuf);
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
@@ -540,7 +541,7 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   if (sc < kStreamGroups) return SALR_ERR_UNSUPPORTED;
   p.sc = sc;
   const int smem = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, p.sc, kStreamGroups);
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
@@ -703,7 +704,7 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
 
   const int mask_smem = static_cast<int>(K * sizeof(uint16_t));
   if (mask_smem > 48 * 1024) {
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];  // zero-initialised: false
     if (h->device < 0 || h->device >= 64) return fail(SALR_ERR_UNSUPPORTED);
     if (!attr_set[h->device]) {
       if ((e = cudaFuncSetAttribute(encode_mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1168,7 +1169,7 @@ cudaError_t orthonormalise(float*& Y, int rows, int l, int lp, int passes, SvdSc
 }
 
 int svd_kernel_attributes(int dev) {
-  static bool set[64] = {false};
+  static std::atomic<bool> set[64];  // zero-initialised: false
   if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
   if (set[dev]) return SALR_OK;
   const int big = kSvdMaxL * (kSvdMaxL + 1) * static_cast<int>(sizeof(double));
