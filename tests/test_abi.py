@@ -256,3 +256,35 @@ def test_linear_plan_rejects_bad_arguments(lib):
     assert f(4096, 4000, 16, 0, 148, ctypes.byref(out)) == 2     # K % 64
     assert f(4096, 64 * 513, 512, 0, 148, ctypes.byref(out)) == 2  # K past the layer kernels
     assert f(4096, 4096, (1 << 24) + 1, 0, 148, ctypes.byref(out)) == 2
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "salr.h"
+
+int main(void) {
+  salr_plan p;
+  int rc = salr_linear_plan(11008, 4096, 2048, 96, 148, &p);
+  if (rc != SALR_OK) { printf("plan %d\n", rc); return 1; }
+  printf("%d %d %d %d %d %d %lld\n", p.path, p.kernels, p.tiles, p.whole_tiles, p.splits,
+         p.units, (long long)p.dense_scratch_bytes);
+  if (strcmp(salr_status_string(SALR_ERR_UNSUPPORTED), "SALR_ERR_UNSUPPORTED") != 0) return 2;
+  if (salr_free(NULL) != SALR_ERR_INVALID) return 3;
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links_from_a_c_program(lib, tmp_path):
+    # the boundary is a C ABI: the header compiles as C99 and a C program links the
+    # library and calls the host-only entry points (no GPU needed)
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER),
+                    str(src), "-o", str(exe), LIB, f"-Wl,-rpath,{os.path.dirname(LIB)}"],
+                   check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout + out.stderr
+    assert out.stdout.split() == ["2", "3", "688", "592", "3", "880", str(11008 * 4096 * 2)]
