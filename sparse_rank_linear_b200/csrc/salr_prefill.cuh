@@ -1,6 +1,10 @@
 // salr_prefill.cuh - the SALR layer for token counts above 64 (prefill shapes), where the
-// tensor-core contraction dominates.  Two kernels per call:
+// tensor-core contraction dominates.  Up to three kernels per call:
 //
+// * expand_dense_kernel (from two token tiles on): the weight expanded once into a dense
+//   bf16 N x K scratch, so that the layer kernel need not decode every block once per
+//   token tile.  Persistent CTAs walk the blocks, staging the next by cp.async while
+//   expanding the current.
 // * salr_t_kernel: t = X A_cat, the concatenated adapter's down projection (SALR
 //   technical summary, Methodology 3), computed once per call on the tensor cores and
 //   rounded once to bf16 into a [M x 128] scratch.  Grid: token tiles x K splits.  With
@@ -9,21 +13,24 @@
 //   and clears it.
 // * salr_prefill_kernel: persistent, one CTA per SM over the work units (128-row weight
 //   tile, token tile, K split).  Tiles are whole while every CTA gets one; the tiles of a
-//   last, partial round are split along K so that their parts even out over the CTAs.  Each 128 x 64 bitmap block arrives by one bulk copy and
-//   the matching X tile by tensor TMA.  Decoder warps expand the block into the
-//   128-byte-swizzled tile (stage 1, Methodology 4) with the same device functions as
-//   the small-M kernel; tcgen05 MMAs multiply it (stage 2).  The adapter's up projection
-//   B_cat^T t^T runs as extra iterations of the same pipeline after a unit's K blocks (on
-//   split 0).  The epilogue writes Y; with several K splits, each adds into an fp32 sum in
-//   L2 whose last contributor writes Y.
+//   last, partial round are split along K so that their parts even out over the CTAs.
+//   Fused mode: each 128 x 64 bitmap block arrives by one bulk copy and the matching X
+//   tile by tensor TMA; decoder warps expand the block into the 128-byte-swizzled tile
+//   (stage 1, Methodology 4) with the same device functions as the small-M kernel, and
+//   tcgen05 MMAs multiply it (stage 2).  Dense mode: warp 0 copies the weight tiles from
+//   the dense scratch by TMA into the same slots, and the decoders stay idle.  The
+//   adapter's up projection B_cat^T t^T runs as extra iterations of the same pipeline
+//   after a unit's K blocks (on split 0).  The epilogue writes Y; a split unit adds into
+//   a token-major fp32 sum in L2 whose last contributor writes Y.
 //
 // Orientation as in the small-M kernel: D[128 weight rows x BNT tokens] in TMEM, two
 // accumulators used by alternate units.  Rings: compact blocks (producer -> decoders),
-// decoded tiles (decoders -> MMA) and X tiles (X loader -> MMA), so that the copy latency
-// and the decode of a block overlap the MMAs of earlier blocks; four decoder groups each
-// work on a different block.  Warp roles (736 threads): 0 compact-block producer, 1 TMEM
-// allocator + MMA issuer, 2-5 epilogue, 6 X-tile producer, 7-22 decoders.  Every wait is
-// bounded; a timeout is recorded in the status word.
+// decoded tiles (decoders or the dense loads -> MMA) and X tiles (X loader -> MMA), so
+// that the copy latency and the decode of a block overlap the MMAs of earlier blocks;
+// four decoder groups each work on a different block.  Warp roles (736 threads): 0
+// compact-block or dense-tile producer, 1 TMEM allocator + MMA issuer, 2-5 epilogue, 6
+// X-tile producer, 7-22 decoders.  Every wait is bounded; a timeout is recorded in the
+// status word.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
