@@ -1,7 +1,7 @@
 // salr_stream.cuh - persistent SALR layer kernel for small token counts (decode shapes).
 //
-// Same layer as salr_linear_kernel, Y = X (M (.) W)^T + (X A_cat) B_cat, organised for
-// the HBM-bound regime (M <= 64) where decoding the bitmap blocks is the whole cost:
+// The layer salr_linear computes, Y = X (M (.) W)^T + (X A_cat) B_cat, organised for the
+// HBM-bound regime (M <= 64) where decoding the bitmap blocks is the whole cost:
 //
 // * Work split: the weight's 128 x 64 blocks, in storage order, are cut into one
 //   contiguous range per CTA (one CTA per SM, every SM the same number of blocks).  A
