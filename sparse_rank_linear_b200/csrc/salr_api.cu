@@ -580,6 +580,11 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   return SALR_OK;
 }
 
+// Output tiles of 128 x 128 beyond 2^27 would let the layer kernel's work units (up to 8
+// parts per tile) overflow its 32-bit counts; such an output (M x N) is far beyond any
+// GPU's memory anyway.
+bool too_many_tiles(int64_t N, int64_t M) { return (N / 128) * ((M + 127) / 128) > (1ll << 27); }
+
 int check_linear_args(const void* X, int64_t M, salr_handle h, const void* A, const void* B,
                       int64_t R, const void* Y) {
   if (!valid_handle(h)) return SALR_ERR_INVALID;
@@ -588,6 +593,7 @@ int check_linear_args(const void* X, int64_t M, salr_handle h, const void* A, co
   if (R > 0 && (!A || !B)) return SALR_ERR_INVALID;
   if (R % 8 != 0 || R > 128) return SALR_ERR_UNSUPPORTED;
   if (M > (1ll << 24)) return SALR_ERR_UNSUPPORTED;
+  if (too_many_tiles(h->N, M)) return SALR_ERR_UNSUPPORTED;
   if (!aligned16(X) || !aligned16(Y) || (R > 0 && (!aligned16(A) || !aligned16(B))))
     return SALR_ERR_UNSUPPORTED;
   return SALR_OK;
@@ -763,7 +769,7 @@ int salr_linear_plan(int64_t N, int64_t K, int64_t M, int64_t R, int32_t sms, sa
   if (!out || M < 1 || R < 0 || sms < 0) return SALR_ERR_INVALID;
   const int shape = check_shape(N, K);
   if (shape != SALR_OK) return shape;
-  if (R % 8 != 0 || R > 128 || M > (1ll << 24)) return SALR_ERR_UNSUPPORTED;
+  if (R % 8 != 0 || R > 128 || M > (1ll << 24) || too_many_tiles(N, M)) return SALR_ERR_UNSUPPORTED;
   if (sms == 0) {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||

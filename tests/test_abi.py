@@ -256,6 +256,9 @@ def test_linear_plan_rejects_bad_arguments(lib):
     assert f(4096, 4000, 16, 0, 148, ctypes.byref(out)) == 2     # K % 64
     assert f(4096, 64 * 513, 512, 0, 148, ctypes.byref(out)) == 2  # K past the layer kernels
     assert f(4096, 4096, (1 << 24) + 1, 0, 148, ctypes.byref(out)) == 2
+    # an output of more than 2^27 tiles of 128 x 128 (work-unit counts stay 32-bit)
+    assert f(1 << 22, 64, 1 << 24, 0, 148, ctypes.byref(out)) == 2
+    assert f(1 << 16, 64, 1 << 24, 0, 148, ctypes.byref(out)) == 0
 
 
 C_CLIENT = r"""
