@@ -30,8 +30,9 @@
  *     device (a NaN in W, a pipeline wait that ran out of time) are recorded in the
  *     handle's status word; salr_encode reports them itself, salr_sync_status reads them.
  *
- * Shape rules (v1): N % 128 == 0, K % 64 == 0, 64 <= K <= 32768, R % 8 == 0, R <= 128,
- * M >= 1, all pointers 16-byte aligned.
+ * Shape rules (v1): N % 128 == 0, 128 <= N <= 2^22, K % 64 == 0, 64 <= K <= 32768,
+ * R % 8 == 0, R <= 128, 1 <= M <= 2^24, at most 2^27 output tiles of 128 x 128
+ * ((N / 128) * ceil(M / 128)), all pointers 16-byte aligned.
  */
 #ifndef SALR_H_
 #define SALR_H_
