@@ -1,10 +1,13 @@
 #!/usr/bin/env python
 """Benchmark of the SALR linear layer Y = X (M.W)^T + (X A_cat) B_cat on B200.
 
-One step is one salr_linear call on the decode q_proj workload (W 4096 x 4096 bf16, 50%
-per-row magnitude pruned and bitmap-encoded, adapters 64 + 16 stacked to R = 80,
-X 16 x 4096).  --workload/--tokens time another configuration of salr_synth.WORKLOADS the
-same way (the default is the headline line).  Prints one JSON line (see --help).
+One step is one salr_linear call.  The headline line is the largest single-GPU workload
+of the configurations: W 28672 x 8192 bf16 (heavy-tailed), 50% per-row magnitude pruned
+and bitmap-encoded, adapters 64 + 32 stacked to R = 96, X 8192 x 8192.
+--workload/--tokens time another point of salr_synth.WORKLOADS as the headline instead.
+Every configuration point (tiny 16; q_proj 1, 16; up_proj 2048; down_proj 1, 128, 4096;
+large 16, 8192) is also timed the same way and reported under "per_config".  Prints one
+JSON line (see --help).
 
 Timing: W warm-up steps, then K steps queued back to back behind a short GPU sleep (so
 that host launch overhead leaves no gaps), with CUDA events on the launching stream at the
@@ -13,9 +16,10 @@ consecutive layers would.  A second pass puts an event pair around every call an
 their percentiles.  The weight/adapter set rotates over enough copies that the working set
 exceeds twice the L2 (no step finds its weights in L2).
 
---impl reference times the fp64 CPU oracle on the same workload instead (one full layer
-per step on the host cores).  Under torchrun every rank runs an independent replica
-(the layer has no data-path exchange); time is the max over ranks.
+--impl reference times the fp64 CPU oracle on a bounded sample of the same workload
+instead (each step: up to 64 tokens against up to 1024 output rows, on the host cores;
+tokens/s counts full-layer tokens).  Under torchrun every rank runs an independent
+replica (the layer has no data-path exchange); time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -39,15 +43,17 @@ if ROOT not in sys.path:
 import salr_synth as synth  # noqa: E402
 
 METRIC = "SALR linear tokens/s + achieved fraction of HBM/tensor roofline on 1 B200"
-WORKLOAD = "q_proj"
-M_TOKENS = 16
+WORKLOAD = "large"
+M_TOKENS = 8192
 SPARSITY = None  # None: the workload's own (0.5)
 L2_BYTES = 126 * 1024 * 1024
 # the headers each layer kernel is compiled from: a recorded DRAM-traffic figure stays
 # valid while these are unchanged
 KERNEL_SOURCES = {
-    "salr_stream_kernel": ["sm100.cuh", "salr_codec.cuh", "salr_stream.cuh"],
-    "salr_prefill_kernel": ["sm100.cuh", "salr_codec.cuh", "salr_stream.cuh", "salr_prefill.cuh"],
+    "salr_stream_kernel": ["sm100.cuh", "salr_block.cuh", "salr_decode.cuh", "salr_codec.cuh",
+                           "salr_stream.cuh"],
+    "salr_prefill_kernel": ["sm100.cuh", "salr_block.cuh", "salr_decode.cuh", "salr_codec.cuh",
+                            "salr_stream.cuh", "salr_prefill.cuh"],
 }
 
 
@@ -212,13 +218,15 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def oracle_step_fn(wl, M):
-    """The fp64 oracle on one full step of the workload (inputs prepared untimed)."""
+def oracle_sample_fn(wl, M, rows):
+    """The fp64 oracle on a bounded sample of one step: ``M`` tokens against the first
+    ``rows`` output rows of W (mask, pruned weight and adapters' columns prepared
+    untimed).  The work per (token, output row) is that of the full layer."""
     import oracle
-    w = synth.weight(wl)
+    w = synth.weight(wl, rows=np.arange(rows))
     wp = oracle.prune(w, oracle.magnitude_mask(w, wl.sparsity))
     x = synth.activations(wl, M)
-    ad = synth.adapters(wl)
+    ad = [(a, b[:, :rows]) for a, b in synth.adapters(wl)]
     return lambda: oracle.linear(x, wp, ad)
 
 
@@ -231,10 +239,23 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+# bounded oracle sample: at most this many tokens and output rows per step
+ORACLE_TOKENS = 64
+ORACLE_ROWS = 1024
+
+
+def oracle_sample(wl, M):
+    """(tokens, rows) of one oracle step and the factor that turns its tokens into
+    full-layer tokens (a sampled step covers rows / N of each token's outputs)."""
+    mo, ro = min(M, ORACLE_TOKENS), min(wl.N, ORACLE_ROWS)
+    return mo, ro, ro / wl.N
+
+
 def time_oracle(wl, M, steps=None, budget_s=10.0):
-    """Oracle steps in a bounded time; above 64 tokens each step is a fixed 64-token slice
-    of X (the work per token is the same, so tokens/s carries over)."""
-    step = oracle_step_fn(wl, min(M, 64))
+    """Oracle steps in a bounded time (or a fixed count); returns (steps, seconds,
+    full-layer tokens per second, sample description)."""
+    mo, ro, frac = oracle_sample(wl, M)
+    step = oracle_sample_fn(wl, mo, ro)
     step()  # warm
     t0 = time.perf_counter()
     n = 0
@@ -244,7 +265,41 @@ def time_oracle(wl, M, steps=None, budget_s=10.0):
         el = time.perf_counter() - t0
         if (steps is not None and n >= steps) or (steps is None and el >= budget_s):
             break
-    return n, el
+    sample = (f"{n} steps of {mo} of the {M} tokens x {ro} of the {wl.N} output rows "
+              f"({wl.name}, K={wl.K}, R={wl.R}) in {el:.2f} s, fp64 numpy oracle; tokens/s "
+              f"counts full-layer tokens ({mo} x {ro}/{wl.N} per step)")
+    return n, el, n * mo * frac / el, sample
+
+
+def format_bytes(N, K, keep):
+    """Encoded size of a weight: bitmap, kept values and offset table (the 16-byte
+    padding of each block, at most 14 bytes, left out)."""
+    nb = (N // 128) * (K // 64)
+    return N * K // 8 + 2 * N * keep + 4 * (nb + 1)
+
+
+def l2_plan(wl):
+    """Weight + adapter copies the timed loop rotates over so that no step finds its
+    weights in L2: enough for twice the L2, at least 2, at most 64 (the smallest layer
+    cannot outgrow the L2 this way; the config says so)."""
+    keep = wl.K - int(np.floor(wl.sparsity * wl.K))
+    per_copy = format_bytes(wl.N, wl.K, keep) + 2 * wl.R * (wl.K + wl.N)
+    ncopies = min(64, max(2, int(np.ceil(2 * L2_BYTES / per_copy))))
+    return ncopies, per_copy
+
+
+def config_for(wl, M, ws):
+    """The config block of the JSON line: the same for the CUDA arm and the reference arm."""
+    ncopies, per_copy = l2_plan(wl)
+    big = ncopies * per_copy > 2 * L2_BYTES
+    return {"workload": f"{wl.name} N={wl.N} K={wl.K} R={wl.R} "
+                        f"({'+'.join(str(r) for r in wl.ranks)}) M={M} sparsity={wl.sparsity:.6g}",
+            "model": f"SALR linear layer ({wl.name} shape)", "global_batch": M * ws,
+            "parallelism": f"replicas x{ws}",
+            "l2": (f"inputs larger than L2: rotating {ncopies} weight+adapter copies "
+                   f"({ncopies * per_copy / 2**20:.0f} MiB > 2x L2)" if big else
+                   f"layer smaller than L2: rotating {ncopies} weight+adapter copies "
+                   f"({ncopies * per_copy / 2**20:.0f} MiB, partly L2-resident)")}
 
 
 def run_reference(args):
@@ -252,23 +307,24 @@ def run_reference(args):
     if rank != 0:
         return
     wl = workload()
-    step = oracle_step_fn(wl, min(M_TOKENS, 64))
+    M = M_TOKENS
+    mo, ro, frac = oracle_sample(wl, M)
+    step = oracle_sample_fn(wl, mo, ro)
     for _ in range(args.warmup):
         step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         step()
     el = time.perf_counter() - t0
-    mo = min(M_TOKENS, 64)
-    value = args.steps * mo / el
+    value = args.steps * mo * frac / el
     cores = blas_threads()
-    sample = f"full {WORKLOAD} layer (M={mo} of {M_TOKENS} tokens) per step, fp64 numpy oracle"
+    sample = (f"each step: {mo} of the {M} tokens x {ro} of the {wl.N} output rows, fp64 "
+              f"numpy oracle; tokens/s counts full-layer tokens ({mo} x {ro}/{wl.N} per step)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD} N={wl.N} K={wl.K} R={wl.R} M={M_TOKENS} "
-                                   f"sparsity={wl.sparsity:.6g}"},
+            "config": config_for(wl, M, ws),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -421,18 +477,197 @@ def traffic_for(kname, workload):
     return e.get("bytes_per_launch")
 
 
+# The (workload, tokens) points of the configurations; the headline line is the largest
+# single-GPU one (large, 8192 tokens), the others are reported under "per_config".
+POINTS = (("tiny", 16), ("q_proj", 1), ("q_proj", 16), ("up_proj", 2048), ("down_proj", 1),
+          ("down_proj", 128), ("down_proj", 4096), ("large", 16), ("large", 8192))
+# A timed region at least this long runs under the power cap: its tensor roofline is the
+# sustained GEMM peak (a shorter region takes the burst peak).
+LONG_REGION_MS = 500.0
+
+
+class Layer:
+    """One workload on the device: rotating encoded copies of W and adapter copies."""
+
+    def __init__(self, salr, wl, dev):
+        self.wl = wl
+        self.w_bits = synth.weight(wl)
+        ad = synth.adapters(wl)
+        self.a_cat = np.concatenate([a for a, _ in ad], axis=1)
+        self.b_cat = np.concatenate([b for _, b in ad], axis=0)
+        W = dev(self.w_bits)
+        self.ncopies, self.per_copy = l2_plan(wl)
+        self.handles = [salr.encode(W, wl.sparsity) for _ in range(self.ncopies)]
+        self.A = [dev(self.a_cat) for _ in range(self.ncopies)]
+        self.B = [dev(self.b_cat) for _ in range(self.ncopies)]
+        del W
+        self.keep = wl.K - int(np.floor(wl.sparsity * wl.K))
+
+    def free(self):
+        for h in self.handles:
+            h.free()
+        self.handles, self.A, self.B = [], [], []
+
+
+def roofline_of(wl, M, keep, kern_ms, region_ms, peaks, peak_src, traffic_key, plan):
+    """The roofline block of one point: the bound (HBM bytes or tensor FLOPs, whichever
+    takes longer at the measured peaks), achieved rate, fraction."""
+    N, K, R = wl.N, wl.K, wl.R
+    abytes = algorithmic_bytes(N, K, R, M, keep)
+    aflops = algorithmic_flops(N, K, R, M)
+    long_region = region_ms >= LONG_REGION_MS
+    tpeak = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops",
+                      peaks["bf16_tflops"])
+    t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = aflops / (tpeak * 1e12)
+    if t_hbm >= t_tc:
+        achieved = abytes / (kern_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+        roof["peak_source"] = f"{peak_src} hbm_gbs"
+    else:
+        achieved = aflops / (kern_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tpeak, "unit": "TFLOP/s",
+                "frac": achieved / tpeak}
+        roof["peak_source"] = (f"{peak_src} "
+                               f"{'bf16_tflops_sustained' if long_region else 'bf16_tflops'}"
+                               f" ({'timed region of %.0f ms, under the power cap' % region_ms if long_region else 'short timed region: burst'})")
+        roof["frac_of_burst_peak"] = achieved / peaks["bf16_tflops"]
+    if M <= 64:
+        kname = f"salr_stream_kernel<{16 if M <= 16 else 32 if M <= 32 else 64},16>"
+    else:
+        kname = f"salr_prefill_kernel<{128 if M <= 128 else 256}>"
+    roof["traffic"] = traffic_for(kname, traffic_key)
+    roof["kernel"] = kname
+    roof["kernels_per_call"] = plan["kernels"]
+    roof["kernel_ms"] = kern_ms
+    roof["algorithmic_bytes"] = abytes
+    roof["algorithmic_flops"] = aflops
+    return roof
+
+
+def time_point(lib, salr, layer, M, steps, warmup, stream, ws, local):
+    """K calls of the layer on device-resident inputs, back to back behind a GPU sleep
+    (CUDA events at the two ends), then a diagnostic pass with an event pair around every
+    call.  Returns the region's time (max over ranks), the per-call percentiles and the
+    clocks seen."""
+    import ctypes
+    import torch
+    import torch.distributed as dist
+
+    wl = layer.wl
+    X = torch.from_numpy(np.ascontiguousarray(synth.activations(wl, M)).view(np.int16)).view(
+        torch.bfloat16).cuda()
+    Y = torch.empty(M, wl.N, dtype=torch.bfloat16, device="cuda")
+    sp = salr.binding._stream_ptr(stream)
+
+    def launch(i):
+        c = i % layer.ncopies
+        rc = lib.salr_linear(ctypes.c_void_p(X.data_ptr()), M, layer.handles[c].handle,
+                             ctypes.c_void_p(layer.A[c].data_ptr()),
+                             ctypes.c_void_p(layer.B[c].data_ptr()), wl.R,
+                             ctypes.c_void_p(Y.data_ptr()), sp)
+        if rc:
+            raise RuntimeError(salr.status_string(rc))
+
+    # every copy is used once before timing (a handle allocates its scratch on first use)
+    for i in range(max(warmup, layer.ncopies)):
+        launch(i)
+    torch.cuda.synchronize()
+    if layer.handles[0].sync_status() != 0:
+        raise RuntimeError("device status after warm-up")
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_stop = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        torch.cuda._sleep(int(2e9 * 40e-6 * steps) + 10_000_000)
+        e_start.record(stream)
+        for i in range(steps):
+            launch(i)
+        e_stop.record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    total_ms = max_over_ranks(e_start.elapsed_time(e_stop), ws, "cuda")
+    for h in layer.handles:
+        status = h.sync_status()
+        if status != 0:
+            raise RuntimeError(f"device status {salr.status_string(status)}")
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e9 * 40e-6 * steps) + 10_000_000)
+    for i in range(steps):
+        ev_s[i].record(stream)
+        launch(i)
+        ev_e[i].record(stream)
+    torch.cuda.synchronize()
+    per_launch = [ev_s[i].elapsed_time(ev_e[i]) for i in range(steps)]
+    del X, Y
+    return total_ms, per_launch, clocks.summary()
+
+
+def time_e2e(lib, salr, layer, M, steps, warmup, stream, ws):
+    """The same calls through salr_linear_host: pinned host activations in and host
+    outputs back, the copies inside the timed region."""
+    import ctypes
+    import torch
+
+    wl = layer.wl
+    xh = torch.from_numpy(synth.activations(wl, M).view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty(M, wl.N, dtype=torch.bfloat16).pin_memory()
+    sp = salr.binding._stream_ptr(stream)
+    # bounded so that the host copies of a prefill-sized step stay within a few seconds
+    n = max(3, min(steps, int(4e9 // (2 * M * (wl.K + wl.N)))))
+
+    def launch_host(i):
+        c = i % layer.ncopies
+        rc = lib.salr_linear_host(ctypes.c_void_p(xh.data_ptr()), M, layer.handles[c].handle,
+                                  ctypes.c_void_p(layer.A[c].data_ptr()),
+                                  ctypes.c_void_p(layer.B[c].data_ptr()), wl.R,
+                                  ctypes.c_void_p(yh.data_ptr()), sp)
+        if rc:
+            raise RuntimeError(salr.status_string(rc))
+
+    for i in range(warmup):
+        launch_host(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e9 * 60e-6 * n) + 10_000_000)
+    e0.record(stream)
+    for i in range(n):
+        launch_host(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), ws, "cuda")
+    return {"value": whole_job_rate(ws, n, M, ms), "unit": "tokens/s",
+            "h2d_bytes_per_step": 2 * M * wl.K, "d2h_bytes_per_step": 2 * M * wl.N,
+            "steps": n, "api": "salr_linear_host (pinned host X and Y)"}
+
+
 def main():
     global WORKLOAD, M_TOKENS, SPARSITY
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--tokens", type=int, default=M_TOKENS, help="M, tokens per call")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="M, tokens per call (default: the workload's largest)")
     ap.add_argument("--sparsity", type=float, default=None,
                     help="fraction of each row pruned (default: the workload's, 0.5)")
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["salr", "reference"], default="salr")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time the headline point only")
+    ap.add_argument("--per-config-steps", type=int, default=100)
     ap.add_argument("--adapter-report", action="store_true",
                     help="time salr_residual_adapter on the workload's weight")
     ap.add_argument("--encode-report", action="store_true",
@@ -440,7 +675,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    WORKLOAD, M_TOKENS, SPARSITY = args.workload, args.tokens, args.sparsity
+    WORKLOAD, SPARSITY = args.workload, args.sparsity
+    M_TOKENS = args.tokens if args.tokens is not None else max(synth.WORKLOADS[WORKLOAD].Ms)
     if SPARSITY is not None and not 0.0 <= SPARSITY < 1.0:
         ap.error("--sparsity must lie in [0, 1)")
     if args.impl == "reference":
@@ -466,182 +702,84 @@ def main():
     if ws > 1:
         dist.barrier()
     lib = salr.load_library()
-
-    wl = workload()
-    N, K, R, M = wl.N, wl.K, wl.R, M_TOKENS
-    keep = K - int(np.floor(wl.sparsity * K))
+    peaks, peak_src = measured_peaks()
+    stream = torch.cuda.current_stream()
 
     def dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
-    w_bits = synth.weight(wl)
-    W = dev(w_bits)
-    ad = synth.adapters(wl)
-    a_cat = np.concatenate([a for a, _ in ad], axis=1)
-    b_cat = np.concatenate([b for _, b in ad], axis=0)
-    x_bits = synth.activations(wl, M)
-    X = dev(x_bits)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    def traffic_key(wl):
+        return wl.name if wl.sparsity == 0.5 else f"{wl.name} s={wl.sparsity:.6g}"
 
-    # rotate over enough independent weight + adapter copies to exceed 2x L2
-    first = salr.encode(W, wl.sparsity)
-    per_copy = first.info()["bytes"] + 2 * R * (K + N)
-    # (at most 64 copies: the smallest layers cannot outgrow L2 this way; the line says so)
-    ncopies = min(64, max(2, int(np.ceil(2 * L2_BYTES / per_copy))))
-    handles = [first] + [salr.encode(W, wl.sparsity) for _ in range(ncopies - 1)]
-    A = [dev(a_cat) for _ in range(ncopies)]
-    B = [dev(b_cat) for _ in range(ncopies)]
-    del W
+    def point_entry(layer, M, steps, region_ms, per_launch, clocks):
+        wl = layer.wl
+        plan = salr.plan(wl.N, wl.K, M, wl.R)
+        kern_ms = region_ms / steps
+        return {"workload": config_for(wl, M, ws)["workload"], "value": whole_job_rate(ws, steps, M, region_ms),
+                "unit": "tokens/s", "steps": steps, "ms_per_step": kern_ms,
+                "roofline": roofline_of(wl, M, layer.keep, kern_ms, region_ms, peaks, peak_src,
+                                        traffic_key(wl), plan),
+                "gpu_launches": steps * plan["kernels"],
+                "per_launch_event_ms_p10_p50_p90": [float(np.percentile(per_launch, q))
+                                                    for q in (10, 50, 90)],
+                "clocks": clocks}
+
+    # ---------------- headline point
+    wl = workload()
+    M = M_TOKENS
+    layer = Layer(salr, wl, dev)
     torch.cuda.synchronize()
-
-    stream = torch.cuda.current_stream()
-    sp = salr.binding._stream_ptr(stream)
-    import ctypes
-
-    def launch(i):
-        c = i % ncopies
-        rc = lib.salr_linear(ctypes.c_void_p(X.data_ptr()), M, handles[c].handle,
-                             ctypes.c_void_p(A[c].data_ptr()), ctypes.c_void_p(B[c].data_ptr()),
-                             R, ctypes.c_void_p(Y.data_ptr()), sp)
-        if rc:
-            raise RuntimeError(salr.status_string(rc))
-
-    # every copy is used once before timing (a handle allocates its scratch on first use)
-    for i in range(max(args.warmup, ncopies)):
-        launch(i)
-    torch.cuda.synchronize()
-    for h in handles[:1]:
-        if h.sync_status() != 0:
-            raise RuntimeError("device status after warm-up")
-
-    # ---------------- device-resident timed region: K launches back to back, CUDA events
-    # at the two ends only (no event between launches), queued behind a GPU sleep so that
-    # host launch overhead leaves no gaps
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_stop = torch.cuda.Event(enable_timing=True)
-    if ws > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        torch.cuda._sleep(int(2e9 * 40e-6 * args.steps) + 10_000_000)
-        e_start.record(stream)
-        for i in range(args.steps):
-            launch(i)
-        e_stop.record(stream)
-        torch.cuda.synchronize()
-    if ws > 1:
-        dist.barrier()
-    total_ms = max_over_ranks(e_start.elapsed_time(e_stop), ws, "cuda")
-    status = handles[0].sync_status()
-    if status != 0:
-        raise RuntimeError(f"device status {salr.status_string(status)}")
-    # diagnostic pass: one event pair around every launch (adds the events' own cost)
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    torch.cuda._sleep(int(2e9 * 40e-6 * args.steps) + 10_000_000)
-    for i in range(args.steps):
-        ev_s[i].record(stream)
-        launch(i)
-        ev_e[i].record(stream)
-    torch.cuda.synchronize()
-    per_launch_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
-
-    # ---------------- context only: the same layer with a dense bf16 W through cuBLAS
-    # (torch), Y = X W^T + (X A_cat) B_cat, the comparison the pages' speedup claim makes
-    dense_ctx = dense_lora_context(w_bits, x_bits, a_cat, b_cat, wl, M, args.steps, total_ms)
-
-    # ---------------- end to end: host activations in, host outputs back, per step
-    xh = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
-    # bounded so that the host copies of a prefill-sized step stay within a few seconds
-    e2e_steps = max(3, min(args.steps, int(4e9 // (2 * M * (K + N)))))
-
-    def launch_host(i):
-        c = i % ncopies
-        rc = lib.salr_linear_host(ctypes.c_void_p(xh.data_ptr()), M, handles[c].handle,
-                                  ctypes.c_void_p(A[c].data_ptr()), ctypes.c_void_p(B[c].data_ptr()),
-                                  R, ctypes.c_void_p(yh.data_ptr()), sp)
-        if rc:
-            raise RuntimeError(salr.status_string(rc))
-
-    for i in range(args.warmup):
-        launch_host(i)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    if ws > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    torch.cuda._sleep(int(2e9 * 60e-6 * e2e_steps) + 10_000_000)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        launch_host(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws, "cuda")
-
-    peaks, peak_src = measured_peaks()
-    kern_ms = total_ms / args.steps  # mean launch duration over the back-to-back region
-    abytes = algorithmic_bytes(N, K, R, M, keep)
-    aflops = algorithmic_flops(N, K, R, M)
-    t_hbm = abytes / (peaks["hbm_gbs"] * 1e9)
-    t_tc = aflops / (peaks["bf16_tflops"] * 1e12)
-    if t_hbm >= t_tc:
-        achieved = abytes / (kern_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"]}
-    else:
-        achieved = aflops / (kern_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"]}
-    if M <= 64:
-        kname = f"salr_stream_kernel<{16 if M <= 16 else 32 if M <= 32 else 64},16>"
-        launches_per_call = 1
-    else:
-        kname = f"salr_prefill_kernel<{128 if M <= 128 else 256}>"
-        # the layer kernel, the t = X A_cat kernel before it, and from two token tiles of
-        # 256 (M > 256) the weight's expansion to a dense scratch before both
-        launches_per_call = 1 + (1 if R > 0 else 0) + (1 if M > 256 else 0)
-    roof["traffic"] = traffic_for(kname, WORKLOAD if wl.sparsity == 0.5
-                                  else f"{WORKLOAD} s={wl.sparsity:.6g}")
-    roof["peak_source"] = peak_src
-    roof["kernel"] = kname
-    roof["kernel_ms"] = kern_ms
-    roof["algorithmic_bytes"] = abytes
-    roof["algorithmic_flops"] = aflops
-
-    value = whole_job_rate(ws, args.steps, M, total_ms)
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+    total_ms, per_launch, clocks = time_point(lib, salr, layer, M, args.steps, args.warmup,
+                                              stream, ws, local)
+    head = point_entry(layer, M, args.steps, total_ms, per_launch, clocks)
+    # context only: the same layer with a dense bf16 W through cuBLAS (torch),
+    # Y = X W^T + (X A_cat) B_cat, the comparison the pages' speedup claim makes
+    dense_ctx = dense_lora_context(layer.w_bits, synth.activations(wl, M), layer.a_cat,
+                                   layer.b_cat, wl, M, args.steps, total_ms)
+    e2e = time_e2e(lib, salr, layer, M, args.steps, args.warmup, stream, ws)
+    line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD} N={N} K={K} R={R} "
-                                   f"({'+'.join(str(r) for r in wl.ranks)}) M={M} "
-                                   f"sparsity={wl.sparsity:.6g}",
-                       "model": f"SALR linear layer ({WORKLOAD} shape)", "global_batch": M * ws,
-                       "parallelism": f"replicas x{ws}",
-                       "l2": f"rotating {ncopies} weight+adapter copies "
-                             f"({ncopies * per_copy / 2**20:.0f} MiB"
-                             f"{' > 2x L2' if ncopies * per_copy > 2 * L2_BYTES else ', smaller than L2'})"},
-            "roofline": roof,
-            "e2e": {"value": whole_job_rate(ws, e2e_steps, M, e2e_ms), "unit": "tokens/s",
-                    "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N},
-            "gpu_launches": args.steps * launches_per_call,
-            "clocks": clocks.summary(),
-            "per_launch_event_ms_p10_p50_p90": [float(np.percentile(per_launch_ms, q))
-                                                for q in (10, 50, 90)],
+            "data": "synthetic", "config": config_for(wl, M, ws),
+            "roofline": head["roofline"], "e2e": e2e,
+            "gpu_launches": head["gpu_launches"], "clocks": clocks,
+            "per_launch_event_ms_p10_p50_p90": head["per_launch_event_ms_p10_p50_p90"],
             "dense_lora_context": dense_ctx}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        n, el = time_oracle(wl, M)
-        line["cpu_baseline"] = {"value": n * M / el, "unit": "tokens/s", "cores": blas_threads(),
-                                "kind": "oracle",
-                                "sample": f"{n} full {WORKLOAD} layers (M={M}) in {el:.1f} s, "
-                                          "fp64 numpy oracle"}
+        n, el, rate, sample = time_oracle(wl, M)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle", "sample": sample}
+
+    # ---------------- every configuration point, the same way (context for the headline)
+    if not args.no_per_config and SPARSITY is None:
+        per = []
+        steps = min(args.steps, args.per_config_steps)
+        cur = layer
+        for name, Mp in POINTS:
+            if cur is None or cur.wl.name != name:
+                if cur is not None:
+                    cur.free()
+                    torch.cuda.synchronize()
+                    torch.cuda.empty_cache()
+                cur = Layer(salr, synth.WORKLOADS[name], dev)
+                torch.cuda.synchronize()
+            if cur is layer and Mp == M:
+                e = dict(head)
+                e["steps"] = args.steps
+            else:
+                t_ms, pl, ck = time_point(lib, salr, cur, Mp, steps, args.warmup, stream, ws, local)
+                e = point_entry(cur, Mp, steps, t_ms, pl, ck)
+            d = dense_lora_context(cur.w_bits, synth.activations(cur.wl, Mp), cur.a_cat,
+                                   cur.b_cat, cur.wl, Mp, e["steps"], e["ms_per_step"] * e["steps"])
+            e["dense_lora_ms_per_step"] = d["ms_per_step"]
+            e["salr_speedup_vs_dense_lora"] = d["salr_speedup"]
+            per.append(e)
+        if cur is not None and cur is not layer:
+            cur.free()
+        line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
-    for h in handles:
-        h.free()
+    layer.free()
     if ws > 1:
         dist.destroy_process_group()
 
