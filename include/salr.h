@@ -79,9 +79,12 @@ typedef enum {
  * 128 rows x 64 columns; block b = i * (K/64) + j covers rows 128i..128i+127 and
  * columns 64j..64j+63 and starts at byte 16 * offsets[b] of the blob.  A block holds
  * 128 little-endian uint64 words (word r: bit c set when W[128i+r, 64j+c] is kept),
- * then the kept values as bf16 in row-major order (a kept -0 stays -0), then zero
- * bytes up to a multiple of 16.  offsets has nblocks + 1 uint32 entries; the last is
- * the blob size in 16-byte units.
+ * then the kept values as bf16 (a kept -0 stays -0), then zero bytes up to a multiple
+ * of 16.  Within a block the values are ordered by row quarter (block rows 32q..32q+31),
+ * then by 4-column group (block columns 4n..4n+3), then by row, then by column: a warp
+ * rebuilding one quarter, one row per thread, then finds each group's values of its 32
+ * rows side by side.  offsets has nblocks + 1 uint32 entries; the last is the blob size
+ * in 16-byte units.
  */
 SALR_API int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* stream,
                 salr_handle* out);
@@ -231,7 +234,7 @@ SALR_API int salr_format_view(salr_handle h, const void** blob, int64_t* blob_by
  *
  *   bytes [0, 64)   header
  *                     0  char[8] "SALRBLK1"       32  int64 keep (entries kept per row)
- *                     8  uint32 version = 1       40  int64 nnz = N * keep
+ *                     8  uint32 version = 2       40  int64 nnz = N * keep
  *                    12  uint32 header size = 64  48  float32 sparsity
  *                    16  int64 N                  52  uint32 0
  *                    24  int64 K                  56  int64 blob bytes (multiple of 16)

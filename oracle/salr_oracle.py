@@ -89,6 +89,12 @@ def prune(w_bits: np.ndarray, mask: np.ndarray) -> np.ndarray:
     return np.where(mask, w_bits, np.uint16(0)).astype(np.uint16)
 
 
+def _quarter_group_order(a: np.ndarray) -> np.ndarray:
+    """A 128 x 64 block viewed as [quarter][4-column group][row in quarter][column in
+    group] (4 x 16 x 32 x 4), the order of the format's value array."""
+    return a.reshape(4, ROWS_PER_BLOCK // 4, COLS_PER_BLOCK // 4, 4).transpose(0, 2, 1, 3)
+
+
 def encode_format(wp_bits: np.ndarray, mask: np.ndarray):
     """Byte image of the encoded weight, following the block layout of ``salr.h``.
 
@@ -96,8 +102,10 @@ def encode_format(wp_bits: np.ndarray, mask: np.ndarray):
     total) in 16-byte units, ``blob`` (uint8).  Block b = i * (K/64) + j covers rows
     128 i .. 128 i + 127 and columns 64 j .. 64 j + 63.  A block is: 128 little-endian
     uint64 bitmap words (word r, bit c set when W[128 i + r, 64 j + c] is kept), then
-    the kept values as little-endian bf16 in row-major order, then zero bytes up to a
-    multiple of 16.
+    the kept values as little-endian bf16, then zero bytes up to a multiple of 16.  The
+    values are ordered by row quarter (block rows 32q .. 32q + 31), then by 4-column
+    group (block columns 4n .. 4n + 3), then by row, then by column: the pages fix only
+    "a bitmap plus a compact array of the kept values"; this order is the library's.
     """
     n, k = wp_bits.shape
     if n % ROWS_PER_BLOCK or k % COLS_PER_BLOCK:
@@ -113,7 +121,10 @@ def encode_format(wp_bits: np.ndarray, mask: np.ndarray):
             cs = slice(j * COLS_PER_BLOCK, (j + 1) * COLS_PER_BLOCK)
             m = mask[rs, cs]
             words = (m.astype(np.uint64) * weights[None, :]).sum(axis=1, dtype=np.uint64)
-            vals = wp_bits[rs, cs][m]  # boolean indexing walks row-major
+            # (row, col) -> (quarter, group, row in quarter, col in group): boolean
+            # indexing then walks the values in the format's order
+            mq = _quarter_group_order(m)
+            vals = _quarter_group_order(wp_bits[rs, cs])[mq]
             body = words.astype("<u8").tobytes() + vals.astype("<u2").tobytes()
             pad = (-len(body)) % 16
             body += b"\x00" * pad
@@ -140,8 +151,9 @@ def decode_format(offsets: np.ndarray, blob: np.ndarray, n: int, k: int) -> np.n
                     & np.uint64(1)).astype(bool)
             nnz = int(bits.sum())
             vals = np.frombuffer(raw, dtype="<u2", count=nnz, offset=start + BITMAP_BYTES)
-            blk = np.zeros((ROWS_PER_BLOCK, COLS_PER_BLOCK), dtype=np.uint16)
-            blk[bits] = vals
+            blk_q = np.zeros((4, COLS_PER_BLOCK // 4, ROWS_PER_BLOCK // 4, 4), dtype=np.uint16)
+            blk_q[_quarter_group_order(bits)] = vals
+            blk = blk_q.transpose(0, 2, 1, 3).reshape(ROWS_PER_BLOCK, COLS_PER_BLOCK)
             out[i * ROWS_PER_BLOCK:(i + 1) * ROWS_PER_BLOCK,
                 j * COLS_PER_BLOCK:(j + 1) * COLS_PER_BLOCK] = blk
     return out

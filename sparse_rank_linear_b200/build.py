@@ -15,7 +15,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsalr.so")
 SOURCES = ["salr_api.cu"]
-HEADERS = ["sm100.cuh", "salr_codec.cuh", "salr_prefill.cuh", "salr_stream.cuh", "salr_svd.cuh"]
+HEADERS = ["sm100.cuh", "salr_block.cuh", "salr_decode.cuh", "salr_codec.cuh", "salr_prefill.cuh",
+           "salr_stream.cuh", "salr_svd.cuh"]
 
 
 def nvcc_path() -> str:

@@ -52,15 +52,14 @@ struct TScratch {
 };
 
 // Scratch of the persistent small-M kernel: fp32 sums of split row tiles [N x 64] and
-// their arrival counts [N/128 x 4 quarters] (left zeroed by every call), and two fp32 t = X A_cat
-// accumulators [64 x 128] with their arrival counts, used by alternate calls; each call
-// clears the buffer the next call will use.  `epoch` counts the calls.
+// their arrival counts [N/128 x 4 quarters], the fp32 t = X A_cat accumulator [64 x 128]
+// and its two counts (parts arrived, readers done).  Every call leaves all of it zero:
+// the last user of each piece clears it on the device.
 struct StreamScratch {
   float* acc = nullptr;
   uint32_t* counters = nullptr;
-  float* tacc = nullptr;       // 2 x kTBuf floats
+  float* tacc = nullptr;       // kTBuf floats
   uint32_t* tflags = nullptr;  // 2 counts
-  uint32_t epoch = 0;
 };
 constexpr int kTBuf = 64 * 128;
 
@@ -303,11 +302,24 @@ int ensure_tscratch(salr_weight_s* h, int64_t M, cudaStream_t st) {
   return SALR_OK;
 }
 
-// CTAs of the dense expansion: five per SM (39 KB of shared memory each), each walking
-// several blocks so that staging the next one overlaps expanding this one.
-unsigned expand_grid(const salr_weight_s* h) {
-  const long long g = std::min<long long>(h->nblocks, 5ll * device_sms(h->device));
-  return static_cast<unsigned>(g < 1 ? 1 : g);
+// The dense expansion: as many CTAs as share the SMs (about 51 KB of shared memory each),
+// each walking several blocks so that staging the next one overlaps expanding this one.
+cudaError_t launch_expand(const salr_weight_s* h, uint16_t* out, cudaStream_t st) {
+  static std::atomic<bool> attr_set[64];  // zero-initialised: false
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(expand_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kExpandSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const long long g = std::min<long long>(h->nblocks, 1ll * kExpandCtasPerSm * device_sms(h->device));
+  expand_dense_kernel<<<static_cast<unsigned>(g < 1 ? 1 : g), 128, kExpandSmemBytes, st>>>(
+      h->blob, h->offsets, static_cast<int>(h->K), static_cast<int>(h->nblocks), out);
+  return cudaGetLastError();
 }
 
 template <int BNT>
@@ -481,7 +493,7 @@ int ensure_stream_scratch(salr_weight_s* h, cudaStream_t st) {
   void *a = nullptr, *b = nullptr, *c = nullptr, *d = nullptr;
   const size_t ab = static_cast<size_t>(h->N) * 64 * sizeof(float);
   const size_t cb = static_cast<size_t>(h->N / 128) * 4 * sizeof(uint32_t);
-  const size_t tb = 2 * kTBuf * sizeof(float);
+  const size_t tb = kTBuf * sizeof(float);
   cudaError_t e;
   if ((e = dev_alloc(&a, ab)) != cudaSuccess || (e = dev_alloc(&b, cb)) != cudaSuccess ||
       (e = dev_alloc(&c, tb)) != cudaSuccess || (e = dev_alloc(&d, 2 * sizeof(uint32_t))) != cudaSuccess) {
@@ -495,7 +507,6 @@ int ensure_stream_scratch(salr_weight_s* h, cudaStream_t st) {
   h->sscr.counters = static_cast<uint32_t*>(b);
   h->sscr.tacc = static_cast<float*>(c);
   h->sscr.tflags = static_cast<uint32_t*>(d);
-  h->sscr.epoch = 0;
   SALR_TRY(cudaMemsetAsync(a, 0, ab, st));
   SALR_TRY(cudaMemsetAsync(b, 0, cb, st));
   SALR_TRY(cudaMemsetAsync(c, 0, tb, st));
@@ -503,23 +514,12 @@ int ensure_stream_scratch(salr_weight_s* h, cudaStream_t st) {
   return SALR_OK;
 }
 
-// Point the kernel at its scratch: this call's t buffer (by the parity of the call count
-// that follows `last`) and the other one, which the call clears for the next.  The caller
-// records the new count only once the launch has succeeded, so that a call that never
-// ran does not flip the parity.
-uint32_t bind_call(StreamParams& sp, float* acc, uint32_t* counters, float* tacc, uint32_t* tflags,
-                   int tbuf, uint32_t last) {
-  const uint32_t epoch = last + 1;
-  const int b = static_cast<int>(epoch & 1u);
+// Point the kernel at its scratch (all of it zero between calls).
+void bind_call(StreamParams& sp, float* acc, uint32_t* counters, float* tacc, uint32_t* tflags) {
   sp.acc = acc;
   sp.counters = counters;
-  sp.tacc = tacc + b * tbuf;
-  sp.tacc_next = tacc + (1 - b) * tbuf;
-  sp.tflag = tflags + b;
-  sp.tflag_next = tflags + (1 - b);
-  sp.tzero = tbuf;
-  sp.epoch = epoch;
-  return epoch;
+  sp.tacc = tacc;
+  sp.tflag = tflags;
 }
 
 template <int BNT>
@@ -531,7 +531,7 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   // decoded-tile ring: one entry per decoder group plus one; the rest of shared memory
   // becomes compact-block entries, which set how many blocks are in flight from HBM
   p.sa = kStreamGroups + 1;
-  const int fixed = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, 0, kStreamGroups);
+  const int fixed = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, 0);
   // The compact-block slots come in a multiple of the group count, so that slot s only
   // ever holds blocks of group s mod 4: a group never waits on a slot whose previous fill
   // it has not consumed itself, and a parity wait can never pass on a phase two fills old.
@@ -540,7 +540,7 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   sc -= sc % kStreamGroups;
   if (sc < kStreamGroups) return SALR_ERR_UNSUPPORTED;
   p.sc = sc;
-  const int smem = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, p.sc, kStreamGroups);
+  const int smem = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, p.sc);
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
@@ -553,6 +553,7 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   const long long units = p.units;
   const int grid = static_cast<int>(units < sms ? units : sms);
   p.tshare = grid < p.kblocks ? grid : p.kblocks;
+  p.treaders = stream_t_readers(units, grid, p.kblocks);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -606,7 +607,9 @@ int noalloc_reset(int dev);  // defined with salr_linear_noalloc below
 namespace {
 
 constexpr char kImageMagic[8] = {'S', 'A', 'L', 'R', 'B', 'L', 'K', '1'};
-constexpr uint32_t kImageVersion = 1;
+// Version 2: block values in quarter / 4-column group / row / column order (version 1 held
+// them row-major and is refused).
+constexpr uint32_t kImageVersion = 2;
 constexpr int64_t kImageHeader = 64;
 
 struct ImageHeader {
@@ -758,10 +761,7 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
 int salr_decode(salr_handle h, void* W_out, void* stream) {
   if (!valid_handle(h) || !W_out) return SALR_ERR_INVALID;
   if (!aligned16(W_out)) return SALR_ERR_UNSUPPORTED;
-  expand_dense_kernel<<<expand_grid(h), 128, 0, static_cast<cudaStream_t>(stream)>>>(
-      h->blob, h->offsets, static_cast<int>(h->K), static_cast<int>(h->nblocks),
-      static_cast<uint16_t*>(W_out));
-  SALR_TRY(cudaGetLastError());
+  SALR_TRY(launch_expand(h, static_cast<uint16_t*>(W_out), static_cast<cudaStream_t>(stream)));
   return SALR_OK;
 }
 
@@ -806,8 +806,7 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     sp.blob = h->blob;
     sp.offsets = h->offsets;
     sp.Y = static_cast<uint16_t*>(Y);
-    const uint32_t epoch = bind_call(sp, h->sscr.acc, h->sscr.counters, h->sscr.tacc,
-                                     h->sscr.tflags, kTBuf, h->sscr.epoch);
+    bind_call(sp, h->sscr.acc, h->sscr.counters, h->sscr.tacc, h->sscr.tflags);
     sp.status = h->status;
     sp.N = static_cast<int>(h->N);
     sp.K = static_cast<int>(h->K);
@@ -832,7 +831,6 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
       case 32: rc = launch_stream<32>(sp, tx, ta, tb, sms, st); break;
       default: rc = launch_stream<64>(sp, tx, ta, tb, sms, st);
     }
-    if (rc == SALR_OK) h->sscr.epoch = epoch;
     return rc;
   }
   // prefill shapes: t = X A_cat once (own kernel), then the fused decode + GEMM
@@ -884,11 +882,7 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     const cudaError_t e =
         dev_alloc_async(reinterpret_cast<void**>(&wdense), static_cast<size_t>(h->N) * h->K * 2, st);
     if (e != cudaSuccess) return cuda_status(e);
-    expand_dense_kernel<<<expand_grid(h), 128, 0, st>>>(h->blob, h->offsets,
-                                                       static_cast<int>(h->K),
-                                                       static_cast<int>(h->nblocks),
-                                                       reinterpret_cast<uint16_t*>(wdense));
-    const cudaError_t le = cudaGetLastError();
+    const cudaError_t le = launch_expand(h, reinterpret_cast<uint16_t*>(wdense), st);
     if (le != cudaSuccess || !make_map(&tw, wdense, h->K, h->N, 64, 128)) {
       cudaFreeAsync(wdense, st);
       return le != cudaSuccess ? cuda_status(le) : SALR_ERR_CUDA;
@@ -991,7 +985,7 @@ int salr_format_view(salr_handle h, const void** blob, int64_t* blob_bytes, cons
 // ------------------------------------------------------------------------------------
 // Serialised image of a handle: the byte form of the compressed weight.  Layout (all
 // little-endian; include/salr.h documents it for readers of the files):
-//   [0,64)   header: "SALRBLK1", u32 version 1, u32 header bytes 64, i64 N, i64 K,
+//   [0,64)   header: "SALRBLK1", u32 version 2, u32 header bytes 64, i64 N, i64 K,
 //            i64 keep, i64 nnz, f32 sparsity, u32 0, i64 blob bytes
 //   [64,..)  offset table, (nblocks + 1) x u32, zero padded to a multiple of 16 bytes
 //   then     the blob (bitmaps, kept values, zero padding), exactly as on the device
@@ -1340,7 +1334,7 @@ int salr_sync_status(salr_handle h, void* stream) {
   if (h->sscr.acc) {
     SALR_TRY(cudaMemset(h->sscr.acc, 0, static_cast<size_t>(h->N) * 64 * sizeof(float)));
     SALR_TRY(cudaMemset(h->sscr.counters, 0, static_cast<size_t>(h->N / 128) * 4 * sizeof(uint32_t)));
-    SALR_TRY(cudaMemset(h->sscr.tacc, 0, 2 * kTBuf * sizeof(float)));
+    SALR_TRY(cudaMemset(h->sscr.tacc, 0, kTBuf * sizeof(float)));
     SALR_TRY(cudaMemset(h->sscr.tflags, 0, 2 * sizeof(uint32_t)));
   }
   const int nrc = noalloc_reset(h->device);
@@ -1366,13 +1360,14 @@ namespace {
 
 constexpr int64_t kNoAllocMaxM = 16;     // tokens per call
 constexpr int64_t kNoAllocMaxN = 32768;  // output features
-constexpr int kNoAllocMaxSMs = 160;      // CTAs of the persistent kernel
-// layout: [t counts: 2 u32][t accumulators: 2 x 16 x 128 f32]
+// layout: [t counts: 2 u32][t accumulator: 16 x 128 f32]
 //         [split-tile arrival counts: N/128 x 4 u32][split-tile sums: N x 16 f32]
+// Nothing in it scales with the SM count: the kernel keeps every per-CTA quantity in
+// shared memory.
 constexpr int kNaTBuf = 16 * 128;
 constexpr size_t kNaFlags = 0;
 constexpr size_t kNaTacc = 256;
-constexpr size_t kNaCounters = kNaTacc + 2 * kNaTBuf * sizeof(float);
+constexpr size_t kNaCounters = kNaTacc + kNaTBuf * sizeof(float);
 constexpr size_t kNaAcc = kNaCounters + (kNoAllocMaxN / 128) * 4 * sizeof(uint32_t);
 constexpr size_t kNaBytes = kNaAcc + static_cast<size_t>(kNoAllocMaxN) * 16 * sizeof(float);
 
@@ -1380,11 +1375,11 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNaBytes];
 
 std::mutex g_na_mu;
 unsigned char* g_na_ptr[64] = {nullptr};
-uint32_t g_na_epoch[64] = {0};
 
 // Device address of the scratch array for the current device (looked up, and cleared on
-// the caller's stream, once per device) and the tag of this call.
-int noalloc_scratch(int dev, cudaStream_t st, unsigned char** out, uint32_t* epoch) {
+// the caller's stream, once per device).  Every call leaves the array zero again on the
+// device, so nothing about a call is kept on the host.
+int noalloc_scratch(int dev, cudaStream_t st, unsigned char** out) {
   if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> g(g_na_mu);
   if (!g_na_ptr[dev]) {
@@ -1395,13 +1390,7 @@ int noalloc_scratch(int dev, cudaStream_t st, unsigned char** out, uint32_t* epo
     g_na_ptr[dev] = static_cast<unsigned char*>(p);
   }
   *out = g_na_ptr[dev];
-  *epoch = g_na_epoch[dev];
   return SALR_OK;
-}
-
-void noalloc_commit_epoch(int dev, uint32_t epoch) {
-  std::lock_guard<std::mutex> g(g_na_mu);
-  g_na_epoch[dev] = epoch;
 }
 
 }  // namespace
@@ -1420,32 +1409,25 @@ int noalloc_reset(int dev) {
   return cuda_status(e);
 }
 
-namespace {
-
-}  // namespace
-
 extern "C" int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, const void* A_cat,
                                    const void* B_cat, int64_t R, void* Y, void* stream) {
   int rc = check_linear_args(X, M, h, A_cat, B_cat, R, Y);
   if (rc != SALR_OK) return rc;
   if (M > kNoAllocMaxM || h->N > kNoAllocMaxN) return SALR_ERR_UNSUPPORTED;
-  if (device_sms(h->device) > kNoAllocMaxSMs) return SALR_ERR_UNSUPPORTED;
   int dev = 0;
   SALR_TRY(cudaGetDevice(&dev));
   if (dev != h->device) return SALR_ERR_INVALID;
   unsigned char* scr = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t epoch = 0;
-  rc = noalloc_scratch(dev, st, &scr, &epoch);
+  rc = noalloc_scratch(dev, st, &scr);
   if (rc != SALR_OK) return rc;
   StreamParams sp{};
   sp.blob = h->blob;
   sp.offsets = h->offsets;
   sp.Y = static_cast<uint16_t*>(Y);
-  epoch = bind_call(sp, reinterpret_cast<float*>(scr + kNaAcc),
-                    reinterpret_cast<uint32_t*>(scr + kNaCounters),
-                    reinterpret_cast<float*>(scr + kNaTacc),
-                    reinterpret_cast<uint32_t*>(scr + kNaFlags), kNaTBuf, epoch);
+  bind_call(sp, reinterpret_cast<float*>(scr + kNaAcc),
+            reinterpret_cast<uint32_t*>(scr + kNaCounters), reinterpret_cast<float*>(scr + kNaTacc),
+            reinterpret_cast<uint32_t*>(scr + kNaFlags));
   sp.status = h->status;
   sp.N = static_cast<int>(h->N);
   sp.K = static_cast<int>(h->K);
@@ -1464,7 +1446,5 @@ extern "C" int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, cons
     if (!make_map(&ta, A_cat, R, h->K, 64, 64)) return SALR_ERR_CUDA;
     if (!make_map(&tb, B_cat, h->N, R, 64, sp.R16)) return SALR_ERR_CUDA;
   }
-  rc = launch_stream<16>(sp, tx, ta, tb, device_sms(h->device), st);
-  if (rc == SALR_OK) noalloc_commit_epoch(dev, epoch);
-  return rc;
+  return launch_stream<16>(sp, tx, ta, tb, device_sms(h->device), st);
 }

@@ -5,34 +5,16 @@
 // `keep` entries of largest magnitude (ties to the lower column), the mask is stored as a
 // bitmap and the kept values as a compact array, both cut into 128 x 64 blocks that are
 // located through a per-block offset table.  The byte layout is the one written out in
-// include/salr.h.  The dense expansion (salr_decode) uses the layer kernels' expansion
-// functions and lives with them (expand_dense_kernel).
+// include/salr.h.  The scatter places each value where the decoders of salr_decode.cuh
+// look for it; the dense expansion (salr_decode) lives with the layer kernels
+// (expand_dense_kernel).
 #pragma once
 #include <cstdint>
+#include "salr_block.cuh"
+#include "salr_decode.cuh"
 #include "sm100.cuh"
 
 namespace salr {
-
-constexpr int kBlockRows = 128;
-constexpr int kBlockCols = 64;
-constexpr int kBitmapBytes = kBlockRows * kBlockCols / 8;  // 1024
-constexpr int kEncThreads = 256;
-
-__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += t;
-  }
-  return v;
-}
-
-__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 // Exclusive prefix sum over the threads of the block (blockDim.x a multiple of 32,
 // at most 1024).  `sh` holds one slot per warp plus one for the total.
@@ -194,40 +176,47 @@ __global__ void __launch_bounds__(1024) encode_scan_kernel(const uint32_t* __res
   }
 }
 
-// One CTA of 128 threads per block.  Thread r writes the block's row word r; then each
-// warp moves the kept values of its 32 rows, one row at a time: lane l reads columns 2l
-// and 2l + 1 of the row (one 128-byte line per row) and stores the kept ones at their
-// rank.  Thread 0 writes the zero padding.
+// One CTA of 128 threads per block.  Thread r (warp = row quarter, lane = row within it)
+// writes its row's bitmap word, then its kept values, nibble by nibble, at the positions
+// the decoders compute for them (values ordered by quarter, nibble, row, column; see
+// salr_decode.cuh).  Thread 0 writes the zero padding.
 __global__ void __launch_bounds__(kBlockRows) encode_scatter_kernel(
     const uint16_t* __restrict__ W, int K, const uint64_t* __restrict__ bits,
     const uint32_t* __restrict__ offsets, unsigned long long cap16, uint8_t* __restrict__ blob) {
-  __shared__ uint32_t sh[33];
+  __shared__ uint64_t bm[kBlockRows];
   const int b = blockIdx.x, nwords = K / 64;
   if (offsets[b + 1] > cap16 || offsets[b] > offsets[b + 1]) return;
   const int i = b / nwords, j = b % nwords, r = threadIdx.x;
   const int warp = r >> 5, lane = r & 31;
   const uint64_t word = bits[static_cast<size_t>(i * kBlockRows + r) * nwords + j];
-  uint32_t nnz;
-  const uint32_t rstart = block_excl_scan(__popcll(word), sh, &nnz);
+  bm[r] = word;
   uint8_t* base = blob + static_cast<size_t>(offsets[b]) * 16;
   reinterpret_cast<uint64_t*>(base)[r] = word;
+  __syncthreads();
+  const QuarterPos qp = quarter_pos(bm, warp, lane);
   uint16_t* vals = reinterpret_cast<uint16_t*>(base + kBitmapBytes);
-  const uint64_t below = (1ull << (2 * lane)) - 1ull;
-#pragma unroll 4
-  for (int q = 0; q < 32; ++q) {
-    const int rr = 32 * warp + q;
-    const uint64_t wq = __shfl_sync(0xffffffffu, word, q);
-    const uint32_t sq = __shfl_sync(0xffffffffu, rstart, q);
-    const uint32_t pair = reinterpret_cast<const uint32_t*>(
-        W + static_cast<size_t>(i * kBlockRows + rr) * K + j * kBlockCols)[lane];
-    const uint32_t m = static_cast<uint32_t>(wq >> (2 * lane)) & 3u;
-    const uint32_t at = sq + __popcll(wq & below);
-    if (m & 1u) vals[at] = static_cast<uint16_t>(pair & 0xFFFFu);
-    if (m & 2u) vals[at + (m & 1u)] = static_cast<uint16_t>(pair >> 16);
+  const uint4* src = reinterpret_cast<const uint4*>(W + static_cast<size_t>(i * kBlockRows + r) * K +
+                                                    j * kBlockCols);
+  uint32_t pos = qp.qb;
+#pragma unroll
+  for (int c8 = 0; c8 < 8; ++c8) {  // 8 columns: two nibbles
+    const uint4 q4 = src[c8];
+    const uint32_t w4[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int n = 2 * c8 + h;
+      uint32_t at = nib_pos(qp, n, pos);
+      const uint32_t nib = static_cast<uint32_t>(word >> (4 * n)) & 15u;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if ((nib >> c) & 1u) vals[at++] = static_cast<uint16_t>(w4[2 * h + (c >> 1)] >> (16 * (c & 1)));
+    }
   }
   if (r == 0) {
+    uint32_t nnz = 0;
+    for (int rr = 0; rr < kBlockRows; ++rr) nnz += __popcll(bm[rr]);
     const uint32_t end = (offsets[b + 1] - offsets[b]) * 16;
-    for (uint32_t p = kBitmapBytes + 2 * nnz; p < end; ++p) base[p] = 0;
+    for (uint32_t q = kBitmapBytes + 2 * nnz; q < end; ++q) base[q] = 0;
   }
 }
 

@@ -81,7 +81,7 @@ struct PrefillCtrl {
 static_assert(sizeof(PrefillCtrl) <= kPreCtrlBytes, "control block");
 
 // Shared-memory layout: [decoded tiles: sa x 16 KB][X tiles: sx x BNT*128][compact blocks:
-// sc x cbuf][chunk tables: 4 x 4 KB][nibble table][control].
+// sc x cbuf][nibble table][control].
 template <int BNT>
 struct PrefillLayout {
   static constexpr int kXbuf = BNT * 128;
@@ -91,8 +91,7 @@ struct PrefillLayout {
     return c_off(sa, sx) + sc * cbuf;
   }
   __host__ __device__ static int smem_bytes(int sa, int sx, int sc, int cbuf) {
-    return table_off(sa, sx, sc, cbuf) + kPreGroups * 4096 + 128 /*nibbles*/ + kPreCtrlBytes +
-           1024 /*align*/;
+    return table_off(sa, sx, sc, cbuf) + 128 /*nibbles*/ + kPreCtrlBytes + 1024 /*align*/;
   }
 };
 
@@ -169,8 +168,8 @@ __global__ void __launch_bounds__(kPreThreads, 1)
   auto xbuf = [&](int s) { return smem + L::x_off(SA) + s * L::kXbuf; };
   auto cbuf = [&](int s) { return smem + L::c_off(SA, SX) + s * p.cbuf; };
   uint8_t* tables = smem + L::table_off(SA, SX, SC, p.cbuf);
-  uint2* ntab = reinterpret_cast<uint2*>(tables + kPreGroups * 4096);
-  PrefillCtrl* ctrl = reinterpret_cast<PrefillCtrl*>(tables + kPreGroups * 4096 + 128);
+  uint2* ntab = reinterpret_cast<uint2*>(tables);
+  PrefillCtrl* ctrl = reinterpret_cast<PrefillCtrl*>(tables + 128);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, cta = blockIdx.x;
@@ -459,12 +458,12 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     }
   } else {
     // ================================================================ decoders (warps 7-22)
-    // four groups of four warps; group x takes the iterations g = x mod 4, each warp 32
-    // rows of a block (or, for an adapter chunk, the group's leader copies B_cat^T)
-    constexpr int RPW = 128 / WPG;
+    // four groups of four warps; group x takes the iterations g = x mod 4, warp wg of the
+    // group rebuilds rows 32 wg .. + 31 of a block, one row per thread (or, for an adapter
+    // chunk, the group's leader copies B_cat^T)
+    static_assert(WPG == 4, "one warp per 32-row quarter");
     const int dw = warp - 7;
     const int grp = dw / WPG, wg = dw % WPG;
-    uint32_t* cs = reinterpret_cast<uint32_t*>(tables + grp * 4096);
     if (p.R16 > 0 && wg == 0 && lane == 0 && !p.dense) prefetch_tmap(&tmB);
     uint32_t g = 0, adn = 0;
     RingCursor cc, ac;  // walked on every iteration, this group's or not
@@ -481,14 +480,13 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         }
         if (it < w.nk) {
           const uint8_t* cb = cbuf(sc);
-          build_chunk_table<RPW>(reinterpret_cast<const uint64_t*>(cb), cs, wg, lane);
-          __syncwarp();
+          const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb), wg, lane);
           if (!mbar_wait(&ctrl->aempty[sa], ac.ph ^ 1)) {
             pre_timeout(p.status, ctrl);
             ok = false;
             break;
           }
-          expand_rows<RPW>(cb + kBitmapBytes, cs, abuf(sa), wg, lane, ntab);
+          expand_quarter_to_tile(qp, cb, wg, lane, ntab, abuf(sa));
           fence_proxy_async_smem();
         } else {
           if (!mbar_wait(&ctrl->aempty[sa], ac.ph ^ 1)) {
@@ -532,19 +530,22 @@ __global__ void __launch_bounds__(kPreThreads, 1)
 // Dense expansion of the whole encoded weight, [N x K] bf16 row-major with pruned entries
 // +0 (the layer's dense-scratch path and salr_decode).  CTAs of four warps walk the
 // 128 x 64 blocks blockIdx.x, blockIdx.x + gridDim.x, ...: each block is staged in shared
-// memory by cp.async while the previous one is expanded (two buffers), the warps build
-// the chunk table and expand 32 rows each with the layer kernels' device functions, and
-// every 8-column chunk goes straight to global memory (8 lanes write one 128-byte row
-// segment).  About 39 KB of shared memory, so several CTAs share an SM.
+// memory by cp.async while the previous one is expanded (two buffers); each warp rebuilds
+// one 32-row quarter with the layer kernels' device functions into a swizzled shared
+// tile, and the tile then goes out row segment by row segment (8 lanes write one
+// 128-byte row segment).  About 51 KB of shared memory, so four CTAs share an SM.
 constexpr int kExpandMaxBlockBytes = kBitmapBytes + 2 * kBlockRows * kBlockCols;  // dense block
 constexpr int kExpandBuf = kExpandMaxBlockBytes + 32;
+constexpr int kExpandCtasPerSm = 4;
 __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __restrict__ blob,
                                                            const uint32_t* __restrict__ offsets,
                                                            int K, int nblocks,
                                                            uint16_t* __restrict__ out) {
-  __shared__ __align__(16) uint8_t cb[2][kExpandBuf];
-  __shared__ __align__(16) uint32_t cs[kBlockRows * 8];
-  __shared__ uint2 nt[16];
+  extern __shared__ uint4 exp_smem[];
+  uint8_t* const cb0 = reinterpret_cast<uint8_t*>(exp_smem);  // two staging buffers
+  auto cb = [&](int buf) { return cb0 + buf * kExpandBuf; };
+  uint8_t* tile = cb0 + 2 * kExpandBuf;
+  uint2* nt = reinterpret_cast<uint2*>(tile + kPreTileBytes);
   const int nwords = K / 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < 16) nt[threadIdx.x] = nibble_entry(threadIdx.x);
@@ -552,7 +553,7 @@ __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __rest
     const uint32_t o0 = offsets[b], n16 = offsets[b + 1] - o0;
     const uint4* src = reinterpret_cast<const uint4*>(blob) + o0;
     for (uint32_t k = threadIdx.x; k < n16; k += 128)
-      cp_async16(reinterpret_cast<uint4*>(cb[buf]) + k, src + k);
+      cp_async16(reinterpret_cast<uint4*>(cb(buf)) + k, src + k);
   };
   int buf = 0;
   if (static_cast<int>(blockIdx.x) < nblocks) stage(blockIdx.x, 0);
@@ -563,24 +564,22 @@ __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __rest
     cp_async_commit();
     cp_async_wait_one();  // this block's copies (the older group) have landed
     const uint32_t n16 = offsets[b + 1] - offsets[b];
-    if (threadIdx.x < 2) reinterpret_cast<uint4*>(cb[buf])[n16 + threadIdx.x] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x < 2) reinterpret_cast<uint4*>(cb(buf))[n16 + threadIdx.x] = make_uint4(0, 0, 0, 0);
     __syncthreads();
+    const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb(buf)), warp, lane);
+    expand_quarter_to_tile(qp, cb(buf), warp, lane, nt, tile);
+    __syncthreads();  // the tile is complete; this compact buffer is free for block b + 2 grid
     const int i = b / nwords, j = b % nwords;
-    build_chunk_table<32>(reinterpret_cast<const uint64_t*>(cb[buf]), cs, warp, lane);
-    __syncwarp();
-    const uint8_t* vals = cb[buf] + kBitmapBytes;
-    const int c = lane & 7;
-    uint16_t* dst = out + static_cast<size_t>(i) * kBlockRows * K + j * kBlockCols + c * 8;
-#pragma unroll 2
-    for (int st = 0; st < 8; ++st) {
-      const int row = 32 * warp + 4 * st + (lane >> 3);
-      const uint32_t e = cs[row * 8 + c];
-      const ExpandIn in = expand_load(vals, e & 0xFFFFu, e >> 16, nt);
-      *reinterpret_cast<uint4*>(dst + static_cast<size_t>(row) * K) = expand_compute(in);
-    }
-    __syncthreads();  // this buffer and the chunk table are free for the next blocks
+    uint16_t* dst = out + static_cast<size_t>(i) * kBlockRows * K + j * kBlockCols;
+    const int c = threadIdx.x & 7;
+#pragma unroll 4
+    for (int r = threadIdx.x >> 3; r < kBlockRows; r += 16)
+      *reinterpret_cast<uint4*>(dst + static_cast<size_t>(r) * K + c * 8) =
+          *reinterpret_cast<const uint4*>(tile + r * 128 + ((c ^ (r & 7)) << 4));
+    __syncthreads();  // the tile is free for the next block
   }
 }
+constexpr int kExpandSmemBytes = 2 * kExpandBuf + kPreTileBytes + 128;
 
 // ------------------------------------------------------------------------------------
 // t = X A_cat for all tokens, rounded once to bf16 into T [M x 128] (ranks past R16 are

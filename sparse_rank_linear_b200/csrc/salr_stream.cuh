@@ -11,20 +11,20 @@
 //   warp to arrive for a quarter (no waiting) reads its sum, writes the bf16 output and
 //   clears the accumulator and the count for the next call.
 // * Stage 1 decode (SALR technical summary, Methodology 4): decoder warps work in
-//   groups, each group on a different block so that several blocks are in flight.  A
-//   warp first turns the bitmap words of its 32 rows into the offset of every (row,
-//   8-column chunk) in the compact value array, then expands one bitmap byte per lane:
-//   each nibble reads three 32-bit words from the 4-byte boundary at or below its first
-//   value, shifts them by a halfword when that value is odd, and spreads them over its
-//   four columns with byte permutes whose selectors come from a 16-entry table.
-// * Stage 2: tcgen05 bf16 MMAs into a double-buffered TMEM accumulator, pipelined
-//   against the decode through shared-memory stages filled by TMA.
+//   groups, each group on a different block so that several blocks are in flight.  Each
+//   warp of a group rebuilds one 32-row quarter of the block, one row per thread
+//   (salr_decode.cuh), and writes it with tcgen05.st into a TMEM slot: the rebuilt block
+//   never passes through shared memory.
+// * Stage 2: tcgen05 bf16 MMAs with A (the rebuilt block, 128 weight rows x 64) read from
+//   that TMEM slot and B (the X tile) from shared memory, into a double-buffered TMEM
+//   accumulator, pipelined against the decode through a ring of TMEM slots.
 // * Concatenated adapter (Methodology 3): t = X A_cat is computed once per call.  The
 //   lowest CTAs multiply a share of the K dimension each on the tensor cores and add
 //   their parts into an fp32 buffer; when all parts have arrived every row tile reads t
 //   back, rounds it to bf16 once and adds B_cat^T t^T to its accumulator with one more
-//   MMA.  The buffer is double-buffered by call parity: each call clears the other one
-//   for the next call, so nothing waits at the end of a call.
+//   MMA.  The CTAs that read t count themselves out; the last one clears the buffer and
+//   both counts, so the scratch is zero again when the kernel ends, whatever the host
+//   did in between (a replayed graph included).
 // * Consecutive calls overlap (programmatic dependent launch): a CTA fetches its first
 //   compact blocks before waiting for the previous kernel of the stream, and touches X,
 //   the adapters, the scratch and Y only after that wait.
@@ -33,11 +33,14 @@
 // waiting on anything.  Every wait is bounded.
 //
 // Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-9 epilogue in two groups
-// (group 0 also the adapter's t share), 10.. decoders.
+// (group 0 also the adapter's t share), 10.. decoders (a warp may only reach the TMEM
+// lanes 32 (warp % 4) .. + 31, so the four warps of a decoder group, consecutive, cover
+// the four quarters).
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
 #include "salr_codec.cuh"
+#include "salr_decode.cuh"
 #include "sm100.cuh"
 
 namespace salr {
@@ -45,7 +48,7 @@ namespace salr {
 constexpr int kStreamFixedWarps = 10;  // producer, MMA, 2 x 4 epilogue warps
 constexpr int kStreamGroups = 4;  // decoder groups, each decodes a different block
 constexpr int kStreamMaxUnitsPerCta = 4096;
-constexpr int kStreamMaxA = 8;   // decoded-tile ring
+constexpr int kStreamMaxA = 8;   // rebuilt-block ring (TMEM slots)
 constexpr int kStreamMaxC = 16;  // compact-block ring
 
 struct StreamParams {
@@ -54,18 +57,15 @@ struct StreamParams {
   uint16_t* Y;
   float* acc;            // [RT x 128 x BNT] fp32 sums of split row tiles, zero between calls
   uint32_t* counters;    // [RT x 4] segments arrived per split tile and 32-row quarter, zero between calls
-  float* tacc;           // [BNT x R16] fp32 accumulator of t = X A_cat (this call's buffer)
-  float* tacc_next;      // the other buffer, cleared by this call for the next one
-  uint32_t* tflag;       // t parts arrived in this call's buffer
-  uint32_t* tflag_next;  // the other buffer's count, cleared by this call
-  int tzero;             // floats per t buffer
-  uint32_t epoch;        // call count; its parity picks the t buffer
+  float* tacc;           // [BNT x R16] fp32 accumulator of t = X A_cat, zero between calls
+  uint32_t* tflag;       // [2]: t parts arrived, CTAs done reading t; zero between calls
   int* status;
   int N, K, M, R, R16;
   int kblocks;  // K / 64
   int RT;       // N / 128
   int units;    // RT * kblocks
   int tshare;   // CTAs 0 .. tshare-1 compute a share of t (tshare = min(grid, kblocks))
+  int treaders;  // CTAs that start a row tile (and read t): see stream_t_readers
   int cbuf;     // per-stage bytes for one compact block (bitmap + values), multiple of 1024
   int bcbuf;    // bytes of the B_cat^T tile / t-share buffer (0 without adapter), x1024
   int sa;       // entries of the decoded-tile ring (tile + X tile each)
@@ -74,25 +74,27 @@ struct StreamParams {
 
 template <int BNT>
 struct StreamLayout {
-  static constexpr int kAbuf = 16384;
   static constexpr int kXbuf = BNT * 128;
-  static constexpr int kCs = 4096;                     // 128 rows x 8 chunks: offset | byte << 16
-  static constexpr int kAent = kAbuf + kXbuf;          // one decoded-tile ring entry
+  static constexpr int kAent = kXbuf;                  // one ring entry: the block's X tile
   static constexpr int kTbuf = BNT * 256;              // t as [BNT x 128] bf16, two chunks
+  // TMEM columns: two accumulators and the t share (BNT each), then, from a multiple of
+  // 32, the ring of rebuilt blocks (32 columns each: 64 bf16 per lane)
+  __host__ __device__ static constexpr uint32_t a_col() { return (3 * BNT + 31) / 32 * 32; }
+  __host__ __device__ static constexpr uint32_t tmem_cols(int sa) {
+    const uint32_t need = a_col() + 32u * static_cast<uint32_t>(sa);
+    return need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
+  }
   // B_cat^T tile [128 x R16] and, at kernel start, the t-share stage (A_cat block + X)
   __host__ __device__ static int bcat_bytes(int R16) {
     if (R16 == 0) return 0;
     const int a = 256 * R16, b = 16384 + kXbuf;
     return ((a > b ? a : b) + 1023) / 1024 * 1024;
   }
-  // layout: [A ring: sa x (tile, X)] [C ring: sc x cbuf] [chunk tables: groups] [t] [B_cat] [ctrl]
+  // layout: [X ring: sa x X tile] [C ring: sc x cbuf] [t] [B_cat] [ctrl] [nibble table]
   __host__ __device__ static int c_off(int sa) { return sa * kAent; }
-  __host__ __device__ static int cs_off(int cbuf, int sa, int sc) { return c_off(sa) + sc * cbuf; }
-  __host__ __device__ static int fixed_off(int cbuf, int sa, int sc, int groups) {
-    return cs_off(cbuf, sa, sc) + groups * kCs;
-  }
-  __host__ __device__ static int smem_bytes(int cbuf, int bcbuf, int sa, int sc, int groups) {
-    return fixed_off(cbuf, sa, sc, groups) + kTbuf + bcbuf + 1024 /*ctrl*/ + 128 /*nibbles*/ +
+  __host__ __device__ static int fixed_off(int cbuf, int sa, int sc) { return c_off(sa) + sc * cbuf; }
+  __host__ __device__ static int smem_bytes(int cbuf, int bcbuf, int sa, int sc) {
+    return fixed_off(cbuf, sa, sc) + kTbuf + bcbuf + 1024 /*ctrl*/ + 128 /*nibbles*/ +
            1024 /*align*/;
   }
 };
@@ -129,13 +131,23 @@ __device__ __forceinline__ bool wait_global_flag(const uint32_t* flag, uint32_t 
   }
 }
 
+// CTAs of a grid of G over U blocks in storage order (K blocks of KB per row tile) whose
+// contiguous range [c U / G, (c + 1) U / G) holds the first block of some row tile: the
+// CTAs that apply the adapter and so read t.
+__host__ __device__ inline int stream_t_readers(long long U, int G, int KB) {
+  int n = 0;
+  for (int c = 0; c < G; ++c) {
+    const long long a = (static_cast<long long>(c) * U) / G;
+    const long long b = (static_cast<long long>(c + 1) * U) / G;
+    n += ((a + KB - 1) / KB) * KB < b;
+  }
+  return n;
+}
+
 __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ uint2 lds64(const uint8_t* p) {
-  return *reinterpret_cast<const uint2*>(p);
-}
 
 // CTA that owns unit u (block u in storage order) under the even split of U units.
 __device__ __forceinline__ int owner_of(long long u, long long U, int G) {
@@ -143,125 +155,6 @@ __device__ __forceinline__ int owner_of(long long u, long long U, int G) {
   while (c + 1 < G && ((c + 1) * U) / G <= u) ++c;
   while (c > 0 && (c * U) / G > u) --c;
   return c;
-}
-
-// Expansion of a bitmap byte into 8 bf16 columns.  A nibble n (4 columns) whose kept
-// values, in order, sit in the window (W0, W1) from its first one expands as
-//   word 0 (columns 0, 1) = prmt(W0, 0, PAT(n & 3))
-//   word 1 (columns 2, 3) = prmt(prmt(W0, W1, PAIR(popc(n & 3))), 0, PAT(n >> 2))
-// where PAT(v), v the 2-bit mask of two columns, is 0x4444 / 0x4410 / 0x1044 / 0x3210
-// (both zero, first value low, first value high, both values; selector 4 reads the zero
-// operand) and PAIR(s) = 0x3210 + 0x2222 s brings values s, s + 1 to the bottom.  The
-// selectors of the 16 nibbles sit in a 128-byte table in shared memory (conflict-free
-// reads): entry n = {PAT(n & 3) | PAT(n >> 2) << 16, PAIR(popc(n & 3))}.
-__device__ __forceinline__ uint32_t pat2(uint32_t v) {
-  return v == 0 ? 0x4444u : v == 1 ? 0x4410u : v == 2 ? 0x1044u : 0x3210u;
-}
-__device__ __forceinline__ uint2 nibble_entry(uint32_t n) {
-  return make_uint2(pat2(n & 3u) | (pat2(n >> 2) << 16), 0x3210u + 0x2222u * __popc(n & 3u));
-}
-
-// Shared-memory operands of one byte's expansion: each nibble's window is the three
-// 32-bit words from the 4-byte boundary at or below its first value (the low nibble's at
-// halfword p, the high nibble's at q = p + popc(low nibble)); words past the block's values
-// (the value array is readable 24 bytes past its end) only meet columns whose mask bit is
-// clear, which the permutes zero.
-struct ExpandIn {
-  uint32_t a0, a1, a2, c0, c1, c2;  // low / high nibble windows
-  uint2 el, eh;                     // nibble-table entries
-  uint32_t p, q;
-};
-
-__device__ __forceinline__ ExpandIn expand_load(const uint8_t* vals, uint32_t p, uint32_t b,
-                                                const uint2* nt) {
-  ExpandIn in;
-  in.p = p;
-  in.q = p + __popc(b & 15u);
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(vals + ((p & ~1u) << 1));
-  const uint32_t* v = reinterpret_cast<const uint32_t*>(vals + ((in.q & ~1u) << 1));
-  in.a0 = w[0];
-  in.a1 = w[1];
-  in.a2 = w[2];
-  in.c0 = v[0];
-  in.c1 = v[1];
-  in.c2 = v[2];
-  in.el = nt[b & 15u];
-  in.eh = nt[b >> 4];
-  return in;
-}
-
-__device__ __forceinline__ uint4 expand_compute(const ExpandIn& in) {
-  // windows start at the nibbles' first values: shift by one halfword when that is odd
-  const uint32_t sh0 = (in.p & 1u) << 4, sh1 = (in.q & 1u) << 4;
-  const uint32_t L0 = __funnelshift_r(in.a0, in.a1, sh0), L1 = __funnelshift_r(in.a1, in.a2, sh0);
-  const uint32_t H0 = __funnelshift_r(in.c0, in.c1, sh1), H1 = __funnelshift_r(in.c1, in.c2, sh1);
-  uint4 out;
-  out.x = __byte_perm(L0, 0u, in.el.x);
-  out.y = __byte_perm(__byte_perm(L0, L1, in.el.y), 0u, in.el.x >> 16);
-  out.z = __byte_perm(H0, 0u, in.eh.x);
-  out.w = __byte_perm(__byte_perm(H0, H1, in.eh.y), 0u, in.eh.x >> 16);
-  return out;
-}
-
-// Chunk table of one decoder warp's RPW rows (rows RPW*wg ..) of a block: entry (row,
-// 8-column chunk) = offset of the chunk's first kept value in the block's value array |
-// the chunk's bitmap byte << 16.  Thread per row: the rows before the warp's own are
-// counted first, then a warp scan of the rows' counts gives each row's start, and a
-// bytewise popcount prefix the chunk offsets within the row.
-template <int RPW>
-__device__ __forceinline__ void build_chunk_table(const uint64_t* bm, uint32_t* cs, int wg, int lane) {
-  uint32_t base = 0;
-  for (int rr = lane; rr < RPW * wg; rr += 32) base += __popcll(bm[rr]);
-  base = warp_sum(base);
-#pragma unroll
-  for (int h = 0; h < (RPW + 31) / 32; ++h) {
-    const int rl = 32 * h + lane;  // row within the warp's rows (lanes past RPW idle)
-    const bool act = rl < RPW;
-    const int row = RPW * wg + rl;
-    const uint64_t w = act ? bm[row] : 0ull;
-    const uint32_t lo = static_cast<uint32_t>(w), hi = static_cast<uint32_t>(w >> 32);
-    const uint32_t clo = __popc(lo), cnt = clo + __popc(hi);
-    const uint32_t inc = warp_incl_scan(cnt);
-    const uint32_t rs = base + inc - cnt;
-    base += __shfl_sync(0xffffffffu, inc, 31);
-    uint32_t bl = lo - ((lo >> 1) & 0x55555555u);
-    bl = (bl & 0x33333333u) + ((bl >> 2) & 0x33333333u);
-    bl = (bl + (bl >> 4)) & 0x0F0F0F0Fu;
-    uint32_t bh = hi - ((hi >> 1) & 0x55555555u);
-    bh = (bh & 0x33333333u) + ((bh >> 2) & 0x33333333u);
-    bh = (bh + (bh >> 4)) & 0x0F0F0F0Fu;
-    const uint32_t plo = bl * 0x01010100u;
-    const uint32_t phi = bh * 0x01010100u + clo * 0x01010101u;
-    // entry = offset | bitmap byte << 16, two uint4 per row
-    uint4 o0, o1;
-    o0.x = rs + (plo & 0xFFu) + ((lo & 0xFFu) << 16);
-    o0.y = rs + ((plo >> 8) & 0xFFu) + (((lo >> 8) & 0xFFu) << 16);
-    o0.z = rs + ((plo >> 16) & 0xFFu) + (((lo >> 16) & 0xFFu) << 16);
-    o0.w = rs + (plo >> 24) + ((lo >> 24) << 16);
-    o1.x = rs + (phi & 0xFFu) + ((hi & 0xFFu) << 16);
-    o1.y = rs + ((phi >> 8) & 0xFFu) + (((hi >> 8) & 0xFFu) << 16);
-    o1.z = rs + ((phi >> 16) & 0xFFu) + (((hi >> 16) & 0xFFu) << 16);
-    o1.w = rs + (phi >> 24) + ((hi >> 24) << 16);
-    if (act) {
-      reinterpret_cast<uint4*>(cs)[2 * row] = o0;
-      reinterpret_cast<uint4*>(cs)[2 * row + 1] = o1;
-    }
-  }
-}
-
-// Expansion of one decoder warp's RPW rows into the decoded tile (K-major, 128-byte
-// swizzle): 4 rows x 8 chunks per step, one bitmap byte per lane.
-template <int RPW>
-__device__ __forceinline__ void expand_rows(const uint8_t* vals, const uint32_t* cs, uint8_t* ab,
-                                            int wg, int lane, const uint2* nt) {
-  const int c = lane & 7;
-#pragma unroll 2
-  for (int st = 0; st < RPW / 4; ++st) {
-    const int row = RPW * wg + 4 * st + (lane >> 3);
-    const uint32_t e = cs[row * 8 + c];
-    const ExpandIn in = expand_load(vals, e & 0xFFFFu, e >> 16, nt);
-    *reinterpret_cast<uint4*>(ab + row * 128 + ((c ^ (row & 7)) << 4)) = expand_compute(in);
-  }
 }
 
 template <int BNT, int NDEC>
@@ -275,13 +168,9 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int SA = p.sa, SC = p.sc;
-  auto abuf = [&](int s) { return smem + s * L::kAent; };
-  auto xbuf = [&](int s) { return smem + s * L::kAent + L::kAbuf; };
+  auto xbuf = [&](int s) { return smem + s * L::kAent; };
   auto cbuf = [&](int s) { return smem + L::c_off(SA) + s * p.cbuf; };
-  auto csb = [&](int g) {
-    return reinterpret_cast<uint32_t*>(smem + L::cs_off(p.cbuf, SA, SC) + g * L::kCs);
-  };
-  uint8_t* tbuf = smem + L::fixed_off(p.cbuf, SA, SC, kStreamGroups);
+  uint8_t* tbuf = smem + L::fixed_off(p.cbuf, SA, SC);
   uint8_t* bcbuf = tbuf + L::kTbuf;  // B_cat^T tile; at kernel start, the t-share stage
   StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(bcbuf + p.bcbuf);
   uint2* ntab = reinterpret_cast<uint2*>(bcbuf + p.bcbuf + 1024);  // 16 x 8 B nibble table
@@ -296,7 +185,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
   const int KB = p.kblocks;
   // t share of this CTA: K blocks cta, cta + tshare, ... (only CTAs below tshare)
   const int nts = (adapter && cta < p.tshare) ? (KB - cta + p.tshare - 1) / p.tshare : 0;
-  constexpr uint32_t kCols = 4 * BNT < 32 ? 32 : 4 * BNT;  // 2 accumulators + t share
+  const uint32_t kCols = L::tmem_cols(SA);  // 2 accumulators, t share, rebuilt-block ring
   // the producer's first batch of block offsets is requested before the set-up below
   uint32_t offv = 0, offx = 0;
   if (warp == 0) {
@@ -336,6 +225,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem;
   const uint32_t tmem_ts = tmem + 2 * BNT;  // t^T share accumulator [128 ranks x BNT]
+  const uint32_t tmem_a = tmem + L::a_col();  // rebuilt-block ring, 32 columns per slot
 
   if (warp == 0) {
     // ================================================================ TMA producer
@@ -463,11 +353,11 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       };
       // the t share is multiplied as soon as its data has landed (polled between blocks),
       // never ahead of decoded blocks: it is fetched only after the dependency wait
-      // The block loop runs on one thread that shares its SM sub-partition with ALU-bound
-      // decoder warps, so it is kept short: descriptors differ from slot 0's only in the
+      // The block loop runs on one thread that shares its SM sub-partition with decoder
+      // warps, so it is kept short: X descriptors differ from slot 0's only in the
       // start-address field (address >> 4, which never carries past its 14 bits in shared
-      // memory), and the slot index and its phase parity advance without division.
-      const uint64_t adesc0 = smem_desc_sw128(smem_u32(abuf(0)), 16, 1024);
+      // memory), slot s's A operand is TMEM columns 32 s .. of the ring, and the slot index
+      // and its phase parity advance without division.
       const uint64_t xdesc0 = smem_desc_sw128(smem_u32(xbuf(0)), 16, 1024);
       constexpr uint32_t kSlotStep = L::kAent >> 4;
       uint32_t dec0 = smem_u32(&ctrl->dec[0]), xf0 = smem_u32(&ctrl->xfull[0]);
@@ -512,11 +402,12 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
             break;
           }
           tc_fence_after();
-          const uint64_t da = adesc0 + s * kSlotStep, dx = xdesc0 + s * kSlotStep;
-          mma_bf16_ss(acc, da, dx, idesc, kb != kba);
-          mma_bf16_ss(acc, da + 2, dx + 2, idesc, 1u);
-          mma_bf16_ss(acc, da + 4, dx + 4, idesc, 1u);
-          mma_bf16_ss(acc, da + 6, dx + 6, idesc, 1u);
+          const uint32_t ta = tmem_a + 32u * s;
+          const uint64_t dx = xdesc0 + s * kSlotStep;
+          mma_bf16_ts(acc, ta, dx, idesc, kb != kba);
+          mma_bf16_ts(acc, ta + 8, dx + 2, idesc, 1u);
+          mma_bf16_ts(acc, ta + 16, dx + 4, idesc, 1u);
+          mma_bf16_ts(acc, ta + 24, dx + 6, idesc, 1u);
           mma_commit(&ctrl->aempty[s]);
           if (++s == SA) {
             s = 0;
@@ -572,12 +463,6 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(p.Y);
     volatile int* gflag = &ctrl->flag[eg];
     griddep_wait();
-    if (eg == 1 && cta == G - 1) {
-      // ---- 0. clear the other t buffer and its arrival count for the next call
-      float4* z = reinterpret_cast<float4*>(p.tacc_next);
-      for (int e = r; e < p.tzero / 4; e += 128) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (lead) *p.tflag_next = 0u;
-    }
     if (eg == 0) {
       bool ok = true;
       // ---- 1. this CTA's share of t = X A_cat: drain t^T from TMEM into the fp32 buffer
@@ -640,8 +525,30 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
           }
           fence_proxy_async_smem();
         }
+        const bool tok = *gflag != 0;
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->tready);
+        if (tok) {
+          // ---- count this CTA out of t's readers; the last one clears t and both counts
+          //      (every reader's loads of t are complete before its count: the values
+          //      are already in shared memory)
+          __threadfence();
+          named_bar(bar_id, 128);
+          if (lead) {
+            const uint32_t done = atomicAdd(p.tflag + 1, 1u) + 1u;
+            *gflag = done == static_cast<uint32_t>(p.treaders) ? 3 : 1;
+          }
+          named_bar(bar_id, 128);
+          if (*gflag == 3) {
+            __threadfence();
+            float4* z = reinterpret_cast<float4*>(p.tacc);
+            for (int e = r; e < p.M * p.R16 / 4; e += 128) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (lead) {
+              p.tflag[0] = 0u;
+              p.tflag[1] = 0u;
+            }
+          }
+        }
       }
     }
     // ---- 3. segments of this group's parity: drain the accumulator, then write Y or, for
@@ -730,17 +637,16 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     }
   } else {
     // ================================================================ decoders
-    // NDEC warps in kStreamGroups groups; group g decodes blocks g, g + groups, ... so
-    // that several blocks are in flight.  Each warp owns 32 rows of its group's block:
-    // it first builds the value offset of each (row, 8-column chunk) of those rows
-    // (thread per row), then expands them one bitmap byte per lane.
-    constexpr int WPG = NDEC / kStreamGroups;  // warps per group
-    static_assert(WPG == 2 || WPG == 4 || WPG == 8, "rows per warp");
-    constexpr int RPW = 128 / WPG;             // rows per warp
+    // NDEC warps in kStreamGroups groups of four consecutive warps; group g decodes blocks
+    // g, g + groups, ... so that several blocks are in flight.  Warp w of a group rebuilds
+    // rows 32 (w % 4) .. + 31 of its block, one row per thread, into the TMEM lanes of
+    // the same numbers (the only lanes a warp may write).
+    static_assert(NDEC == 4 * kStreamGroups, "four warps, one per row quarter, in each group");
     const int dw = warp - kStreamFixedWarps;
-    const int g = dw / WPG, wg = dw % WPG;
+    const int g = dw >> 2, q = warp & 3;
     const int nunits = u1 - u0;
-    const bool leader = wg == 0 && lane == 0;  // issues the group's X-tile copies
+    const bool leader = (dw & 3) == 0 && lane == 0;  // issues the group's X-tile copies
+    const uint32_t tlane = tmem_a + (static_cast<uint32_t>(32 * q) << 16);
     int last_x = -1;
     griddep_wait();
     for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
@@ -750,24 +656,27 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         break;
       }
       const uint8_t* cb = cbuf(sc);
-      const uint64_t* bm = reinterpret_cast<const uint64_t*>(cb);
-      const uint8_t* vals = cb + kBitmapBytes;
-      uint32_t* cs = csb(g);
-      uint8_t* ab = abuf(sa);
-      build_chunk_table<RPW>(bm, cs, wg, lane);
-      __syncwarp();
-      // ---- the decoded tile's ring entry must be free; the group leader fetches X
+      const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb), q, lane);
+      // ---- the TMEM slot must be free (its last MMAs complete); the group leader fetches X
       if (!mbar_wait(&ctrl->aempty[sa], ((it / SA) & 1) ^ 1)) {
         stream_timeout(p, ctrl);
         break;
       }
+      tc_fence_after();
       if (leader) {
         mbar_arrive_expect_tx(&ctrl->xfull[sa], BNT * 128);
         tma_load_2d(xbuf(sa), &tmX, ((u0 + it) % KB) * 64, 0, &ctrl->xfull[sa]);
         last_x = it;
       }
-      expand_rows<RPW>(vals, cs, ab, wg, lane, ntab);
-      fence_proxy_async_smem();
+      const uint32_t ts = tlane + 32u * sa;
+      uint32_t r[8];
+      expand_quarter(qp, cb + kBitmapBytes, ntab, [&](int n, uint32_t w0, uint32_t w1) {
+        r[2 * (n & 3)] = w0;
+        r[2 * (n & 3) + 1] = w1;
+        if ((n & 3) == 3) tmem_st8(ts + 8 * (n >> 2), r[0], r[1], r[2], r[3], r[4], r[5], r[6], r[7]);
+      });
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&ctrl->dec[sa]);

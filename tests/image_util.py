@@ -23,7 +23,7 @@ def image(w_bits: np.ndarray, sparsity: float) -> bytes:
     return pack(n, k, keep, n * keep, s32, offs, blob)
 
 
-def pack(n, k, keep, nnz, sparsity, offs, blob, version=1, header_bytes=64, magic=MAGIC,
+def pack(n, k, keep, nnz, sparsity, offs, blob, version=2, header_bytes=64, magic=MAGIC,
          zero=0) -> bytes:
     head = HEADER.pack(magic, version, header_bytes, n, k, keep, nnz, sparsity, zero,
                        len(blob))

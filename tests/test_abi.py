@@ -127,7 +127,7 @@ def test_load_rejects_bad_images_on_host(lib):
     bad = {
         "short": good[:63],
         "magic": pk(magic=b"SALRBLK2"),
-        "version": pk(version=2),
+        "version": pk(version=1),  # row-major value order, refused
         "header size": pk(header_bytes=72),
         "reserved word": pk(zero=1),
         "keep": pk(keep=keep + 1, nnz=n * (keep + 1)),
