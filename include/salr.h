@@ -201,10 +201,12 @@ typedef struct {
                           GEMM; 2: weight expansion + t kernel + GEMM on dense weight tiles */
   int32_t kernels;     /* kernel launches per call */
   int32_t token_tile;  /* tokens per MMA tile: 16, 32, 64, 128 or 256 */
+  int32_t tile_rows;   /* weight rows per output tile: 128, or 256 on path 2 when
+                          N % 256 == 0 (two MMAs share each X tile) */
   int32_t grid;        /* CTAs of the layer kernel, at most one per SM */
   int32_t units;       /* work units of the layer kernel: 128 x 64 weight blocks (path 0),
                           else whole tiles plus the K parts of split tiles */
-  int32_t tiles;       /* output tiles of 128 weight rows x token_tile (paths 1, 2) */
+  int32_t tiles;       /* output tiles of tile_rows weight rows x token_tile (paths 1, 2) */
   int32_t whole_tiles; /* tiles computed whole (paths 1, 2) */
   int32_t splits;      /* K parts of each remaining tile (paths 1, 2; 1 = none) */
   int64_t split_sum_bytes;     /* fp32 sums of the split tiles in the handle's workspace */

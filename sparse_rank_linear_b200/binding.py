@@ -26,7 +26,8 @@ _P, _I64, _F, _I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
 class SalrPlan(ctypes.Structure):
     """salr_plan of include/salr.h (field order and types as declared there)."""
     _fields_ = [("path", ctypes.c_int32), ("kernels", ctypes.c_int32),
-                ("token_tile", ctypes.c_int32), ("grid", ctypes.c_int32),
+                ("token_tile", ctypes.c_int32), ("tile_rows", ctypes.c_int32),
+                ("grid", ctypes.c_int32),
                 ("units", ctypes.c_int32), ("tiles", ctypes.c_int32),
                 ("whole_tiles", ctypes.c_int32), ("splits", ctypes.c_int32),
                 ("split_sum_bytes", ctypes.c_int64), ("dense_scratch_bytes", ctypes.c_int64)]

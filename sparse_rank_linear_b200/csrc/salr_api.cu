@@ -32,6 +32,13 @@ constexpr int kSmemLimit = 232448;  // B200 opt-in dynamic shared memory per CTA
 // scratch wins (up_proj M = 512: 104 against 128 us; down_proj M = 512: 107 against
 // 110 us; up_proj M = 1024: 134 against 183 us).
 constexpr int kDenseMinTokenTiles = 2;
+// Full rounds (256-row tiles per SM) from which the dense path takes 256-row weight tiles.
+// SALR_WIDE_MIN_ROUNDS overrides it (tests reach the 256-row kernel on small shapes).
+constexpr int kWideMinRounds = 8;
+int wide_min_rounds() {
+  const char* v = getenv("SALR_WIDE_MIN_ROUNDS");
+  return v && v[0] >= '0' && v[0] <= '9' ? atoi(v) : kWideMinRounds;
+}
 
 // Split-K scratch of the prefill kernel: fp32 tile sums and arrival counts (grown on
 // demand, left zeroed by every call).
@@ -373,6 +380,17 @@ TileSplit tail_split(int tiles, int kb, int sms) {
   return r;
 }
 
+// Bound on the K blocks the busiest CTA multiplies under a work split (see tail_split).
+int64_t split_makespan(int tiles, int kb, int sms, TileSplit ts) {
+  const int64_t s = ts.splits;
+  const int64_t part = (kb + s - 1) / s;
+  if (tiles < sms) return part;  // at most one part per CTA
+  const int64_t whole = static_cast<int64_t>(tiles / sms) * kb;
+  const int64_t rem = tiles - ts.full;
+  if (rem == 0) return whole;
+  return whole + (rem * s + sms - 1) / sms * part;
+}
+
 // The launch plan of salr_linear for M tokens on `sms` SMs: the call itself and
 // salr_linear_plan both take their decisions from here.  N and K are valid shapes
 // (check_shape); for M > 64, K stays within kPreMaxKBlocks blocks of 64.
@@ -380,6 +398,7 @@ struct LinearPlan {
   int path;     // 0 small-M kernel, 1 t + fused decode/GEMM, 2 expansion + t + dense GEMM
   int kernels;  // launches per call
   int bnt;      // tokens per MMA tile
+  int rows;     // weight rows per output tile: 128, or 256 (dense path, N % 256 == 0)
   int RT, KB, TT, tiles;
   int full, splits;  // whole tiles; K parts of each later tile
   int units, grid;
@@ -399,25 +418,42 @@ LinearPlan plan_linear(int64_t N, int64_t K, int64_t M, int64_t R, int sms) {
   }
   p.bnt = M <= 128 ? 128 : 256;
   p.TT = static_cast<int>((M + p.bnt - 1) / p.bnt);
-  p.tiles = p.RT * p.TT;
+  const bool dense = p.TT >= kDenseMinTokenTiles;
+  // Dense weight tiles of 256 rows let two MMAs share every X tile: a third fewer operand
+  // bytes through shared memory per MMA cycle.  Their two accumulators fill the TMEM, so
+  // a unit's epilogue no longer overlaps the next unit's MMAs; that costs a few us per
+  // unit.  Measured on B200 (256-row against 128-row tiles): large M = 8192 (3584 tiles,
+  // 24 rounds) 3.42 against 4.23 ms; up_proj M = 2048 (344 tiles) 214 against 203 us;
+  // down_proj M = 4096 (256 tiles) 379 against 364 us.  So they are taken from
+  // kWideMinRounds full rounds of 256-row tiles on, and only if the busiest CTA then gets
+  // no more 128-row block steps than with 128-row tiles.
+  p.rows = 128;
+  if (dense && p.bnt == 256 && N % 256 == 0) {
+    const int t128 = p.RT * p.TT, t256 = static_cast<int>(N / 256) * p.TT;
+    const int64_t m128 = split_makespan(t128, p.KB, sms, tail_split(t128, p.KB, sms));
+    const int64_t m256 = 2 * split_makespan(t256, p.KB, sms, tail_split(t256, p.KB, sms));
+    if (t256 >= static_cast<int64_t>(wide_min_rounds()) * sms && m256 <= m128) p.rows = 256;
+  }
+  p.tiles = static_cast<int>(N / p.rows) * p.TT;
   const TileSplit ts = tail_split(p.tiles, p.KB, sms);
   p.full = ts.full;
   p.splits = ts.splits;
   p.units = ts.full + (p.tiles - ts.full) * ts.splits;
   p.grid = std::min(p.units, sms);
-  const bool dense = p.TT >= kDenseMinTokenTiles;
   p.path = dense ? 2 : 1;
   p.kernels = 1 + (R > 0 ? 1 : 0) + (dense ? 1 : 0);
-  p.sum_bytes = p.splits > 1 ? static_cast<int64_t>(p.tiles - p.full) * 128 * p.bnt * 4 : 0;
+  p.sum_bytes = p.splits > 1 ? static_cast<int64_t>(p.tiles - p.full) * p.rows * p.bnt * 4 : 0;
   p.dense_bytes = dense ? N * K * 2 : 0;
   return p;
 }
 
-template <int BNT>
+template <int BNT, bool WIDE>
 int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb,
                    const CUtensorMap& tt, const CUtensorMap& tw, int grid, bool after_t,
                    cudaStream_t st) {
   using L = PrefillLayout<BNT>;
+  const auto kern = salr_prefill_kernel<BNT, WIDE>;
+  p.wide = WIDE ? 1 : 0;
   // Ring sizes.  Among 5 or 4 decoded-tile slots and 4 to 2 X slots, take the layout
   // with the most compact-block slots (a multiple of the group count, at most kPreMaxC):
   // compact blocks come from HBM and need the deepest queue, X tiles mostly hit L2.  Ties
@@ -430,14 +466,16 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   // block it - 4, which saw block it - 4 - SA >= it - 2 SA consumed (the MMA consumes in
   // order), so the slot can never be two phases behind.
   int sa = 0, sx = 0, sc = 0;
+  p.atile = p.wide ? 2 * kPreTileBytes : kPreTileBytes;
+  const int au = p.atile / kPreTileBytes;  // 16 KB units per weight-tile slot
   if (p.dense) {
     // dense weight tiles: no compact-block ring.  Four weight-tile slots and as many X
     // slots as fit (up to four): measured against 6 + 3 and 3 + 5 slots on B200, 4 + 4
     // was the fastest (down_proj M = 4096: 380 against 404 and 393 us; up_proj M = 2048
-    // even)
-    sa = 4;
+    // even).  256-row tiles take 32 KB slots: three of them and three X slots.
+    sa = p.wide ? 3 : 4;
     for (sx = kPreMaxX; sx >= 2; --sx)
-      if (L::smem_bytes(sa, sx, 0, p.cbuf) <= kSmemLimit) break;
+      if (L::smem_bytes(sa * au, sx, 0, p.cbuf) <= kSmemLimit) break;
     if (sx < 2) return SALR_ERR_UNSUPPORTED;
     sc = kPreGroups;  // placeholder so the check below passes; no slot is used
   }
@@ -457,13 +495,13 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   p.sa = sa;
   p.sx = sx;
   p.sc = p.dense ? 0 : sc;
-  const int smem = L::smem_bytes(p.sa, p.sx, p.sc, p.cbuf);
+  const int smem = L::smem_bytes(p.sa * au, p.sx, p.sc, p.cbuf);
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return SALR_ERR_UNSUPPORTED;
   if (!attr_set[dev]) {
-    SALR_TRY(cudaFuncSetAttribute(salr_prefill_kernel<BNT>,
+    SALR_TRY(cudaFuncSetAttribute(kern,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit));
     attr_set[dev] = true;
   }
@@ -480,13 +518,13 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = after_t ? 1 : 0;
-  SALR_TRY(cudaLaunchKernelEx(&cfg, salr_prefill_kernel<BNT>, p, tx, tb, tt, tw));
+  SALR_TRY(cudaLaunchKernelEx(&cfg, kern, p, tx, tb, tt, tw));
   return SALR_OK;
 }
 
 // Persistent small-M path: one CTA per SM, launched so that it may overlap the preceding
 // kernel of the stream.
-constexpr int kStreamDecoders = 16;
+constexpr int kStreamDecoders = 4 * kStreamGroups;  // one warp per row quarter in each group
 
 int ensure_stream_scratch(salr_weight_s* h, cudaStream_t st) {
   if (h->sscr.acc) return SALR_OK;
@@ -528,9 +566,11 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   using L = StreamLayout<BNT>;
   constexpr int kThreads = 32 * (kStreamFixedWarps + kStreamDecoders);
   p.bcbuf = L::bcat_bytes(p.R16);
-  // decoded-tile ring: one entry per decoder group plus one; the rest of shared memory
-  // becomes compact-block entries, which set how many blocks are in flight from HBM
-  p.sa = kStreamGroups + 1;
+  // rebuilt-block ring (TMEM slots, each with its X tile in shared memory): two per
+  // decoder group, so that a group only ever waits for the MMAs of its own block before
+  // last; the rest of shared memory becomes compact-block entries, which set how many
+  // blocks are in flight from HBM
+  p.sa = 2 * kStreamGroups;
   const int fixed = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, 0);
   // The compact-block slots come in a multiple of the group count, so that slot s only
   // ever holds blocks of group s mod 4: a group never waits on a slot whose previous fill
@@ -783,6 +823,7 @@ int salr_linear_plan(int64_t N, int64_t K, int64_t M, int64_t R, int32_t sms, sa
   out->path = p.path;
   out->kernels = p.kernels;
   out->token_tile = p.bnt;
+  out->tile_rows = p.path == 0 ? 128 : p.rows;
   out->grid = p.grid;
   out->units = p.units;
   out->tiles = p.tiles;
@@ -862,7 +903,7 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   pp.splits = pl.splits;
   if (pp.splits > 1) {
     const size_t ntail = static_cast<size_t>(pl.tiles - pl.full);
-    rc = ensure_workspace(h, ntail * 128 * bnt, ntail * 4, st);
+    rc = ensure_workspace(h, ntail * pl.rows * bnt, ntail * 4, st);
     if (rc != SALR_OK) return rc;
     pp.acc = h->work.ws;
     pp.counters = h->work.counters;
@@ -878,6 +919,7 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   std::memset(&tw, 0, sizeof(tw));
   uint8_t* wdense = nullptr;
   pp.dense = pl.path == 2 ? 1 : 0;
+  pp.wide = pl.rows == 256 ? 1 : 0;
   if (pp.dense) {
     const cudaError_t e =
         dev_alloc_async(reinterpret_cast<void**>(&wdense), static_cast<size_t>(h->N) * h->K * 2, st);
@@ -919,8 +961,9 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
                     : launch_t<256>(tp, tx, ta, TT * tp.splits, st);
     if (rc != SALR_OK) return release_dense(rc);
   }
-  rc = bnt == 128 ? launch_prefill<128>(pp, tx, tb, tt, tw, grid, R > 0, st)
-                  : launch_prefill<256>(pp, tx, tb, tt, tw, grid, R > 0, st);
+  rc = bnt == 128  ? launch_prefill<128, false>(pp, tx, tb, tt, tw, grid, R > 0, st)
+       : pp.wide    ? launch_prefill<256, true>(pp, tx, tb, tt, tw, grid, R > 0, st)
+                    : launch_prefill<256, false>(pp, tx, tb, tt, tw, grid, R > 0, st);
   return release_dense(rc);
 }
 

@@ -18,7 +18,10 @@
 //   tile by tensor TMA; decoder warps expand the block into the 128-byte-swizzled tile
 //   (stage 1, Methodology 4) with the same device functions as the small-M kernel, and
 //   tcgen05 MMAs multiply it (stage 2).  Dense mode: warp 0 copies the weight tiles from
-//   the dense scratch by TMA into the same slots, and the decoders stay idle.  The
+//   the dense scratch by TMA into the same slots, and the decoders stay idle.  Wide dense
+//   mode takes 256 weight rows per unit: each slot holds two 128-row tiles, two MMAs (one
+//   TMEM accumulator each) share every X tile, and the two accumulators then serve one
+//   unit instead of alternating between units.  The
 //   adapter's up projection B_cat^T t^T runs as extra iterations of the same pipeline
 //   after a unit's K blocks (on split 0).  The epilogue writes Y; a split unit adds into
 //   a token-major fp32 sum in L2 whose last contributor writes Y.
@@ -53,7 +56,7 @@ struct PrefillParams {
   const uint8_t* blob;
   const uint32_t* offsets;
   uint16_t* Y;
-  float* acc;          // [split tiles][128 rows][BNT tokens] fp32 sums, zero between calls
+  float* acc;          // [split tiles][BNT tokens][rows] fp32 sums, zero between calls
   uint32_t* counters;  // [split tiles][4] split arrivals per 32-row quarter, zero between calls
   int* status;
   int N, K, M, R16;
@@ -63,6 +66,9 @@ struct PrefillParams {
   int splits;          // K splits of each tile from `full` on (the split tiles)
   int units;           // split tiles x splits + full (split units first)
   int dense;           // 1: weight tiles come dense from tmW by TMA (no decoding)
+  int wide;            // dense mode with 256-row tiles: each unit is two 128-row halves
+                       // that share the X tiles, one TMEM accumulator per half
+  int atile;           // bytes of a decoded-tile ring slot: 16 KB, or 32 KB when wide
   int cbuf;            // bytes of a compact-block slot, multiple of 1024
   int sc, sa, sx;      // ring depths: compact blocks, decoded tiles, X tiles
 };
@@ -85,6 +91,7 @@ static_assert(sizeof(PrefillCtrl) <= kPreCtrlBytes, "control block");
 template <int BNT>
 struct PrefillLayout {
   static constexpr int kXbuf = BNT * 128;
+  // `sa` counts 16 KB units: ring slots x (atile / 16 KB)
   __host__ __device__ static int x_off(int sa) { return sa * kPreTileBytes; }
   __host__ __device__ static int c_off(int sa, int sx) { return x_off(sa) + sx * kXbuf; }
   __host__ __device__ static int table_off(int sa, int sx, int sc, int cbuf) {
@@ -152,7 +159,7 @@ __device__ __forceinline__ PreUnit pre_unit(const PrefillParams& p, int u) {
 // ranks of t, and its compact-block slot turn carries no data.  Accumulators alternate
 // between two TMEM column ranges, so that the epilogue of one unit overlaps the MMAs of
 // the next.
-template <int BNT>
+template <int BNT, bool WIDE>
 __global__ void __launch_bounds__(kPreThreads, 1)
     salr_prefill_kernel(const __grid_constant__ PrefillParams p,
                         const __grid_constant__ CUtensorMap tmX,
@@ -164,10 +171,14 @@ __global__ void __launch_bounds__(kPreThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int SC = p.sc, SA = p.sa, SX = p.sx;
-  auto abuf = [&](int s) { return smem + s * kPreTileBytes; };
-  auto xbuf = [&](int s) { return smem + L::x_off(SA) + s * L::kXbuf; };
-  auto cbuf = [&](int s) { return smem + L::c_off(SA, SX) + s * p.cbuf; };
-  uint8_t* tables = smem + L::table_off(SA, SX, SC, p.cbuf);
+  const int AU = SA * (p.atile / kPreTileBytes);  // 16 KB units of the decoded-tile ring
+  auto abuf = [&](int s) { return smem + s * p.atile; };
+  auto xbuf = [&](int s) { return smem + L::x_off(AU) + s * L::kXbuf; };
+  auto cbuf = [&](int s) { return smem + L::c_off(AU, SX) + s * p.cbuf; };
+  uint8_t* tables = smem + L::table_off(AU, SX, SC, p.cbuf);
+  // weight rows per unit: 128, or 256 (taken from the parameters in the wide kernel, which
+  // as a run-time value keeps that kernel's registers within bounds)
+  const int ROWS = WIDE ? 128 * (1 + (p.wide & 1)) : 128;
   uint2* ntab = reinterpret_cast<uint2*>(tables);
   PrefillCtrl* ctrl = reinterpret_cast<PrefillCtrl*>(tables + 128);
 
@@ -225,13 +236,18 @@ __global__ void __launch_bounds__(kPreThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&ctrl->dec[sa], kPreTileBytes);
-          if (it < w.nk) {
-            tma_load_2d(abuf(sa), &tmW, (w.kb0 + it) * 64, w.i * 128, &ctrl->dec[sa]);
-          } else {
-            const int c = it - w.nk;
-            tma_load_2d(abuf(sa), &tmB, w.i * 128, c * 64, &ctrl->dec[sa]);
-            tma_load_2d(abuf(sa) + 8192, &tmB, w.i * 128 + 64, c * 64, &ctrl->dec[sa]);
+          mbar_arrive_expect_tx(&ctrl->dec[sa], static_cast<uint32_t>(p.atile));
+#pragma unroll 1
+          for (int hf = 0; hf < ROWS / 128; ++hf) {  // 128-row halves, 16 KB apart
+            uint8_t* dst = abuf(sa) + hf * kPreTileBytes;
+            const int row = w.i * ROWS + hf * 128;
+            if (it < w.nk) {
+              tma_load_2d(dst, &tmW, (w.kb0 + it) * 64, row, &ctrl->dec[sa]);
+            } else {
+              const int c = it - w.nk;
+              tma_load_2d(dst, &tmB, row, c * 64, &ctrl->dec[sa]);
+              tma_load_2d(dst + 8192, &tmB, row + 64, c * 64, &ctrl->dec[sa]);
+            }
           }
           gi = g + 1;
         }
@@ -337,15 +353,20 @@ __global__ void __launch_bounds__(kPreThreads, 1)
       constexpr uint32_t idesc_mn = idesc_bf16(128, BNT, 1, 0);
       const uint64_t adesc0 = smem_desc_sw128(smem_u32(abuf(0)), 16, 1024);
       const uint64_t xdesc0 = smem_desc_sw128(smem_u32(xbuf(0)), 16, 1024);
-      constexpr uint32_t astep = kPreTileBytes >> 4, xstep = L::kXbuf >> 4;
+      const uint32_t astep = static_cast<uint32_t>(p.atile) >> 4;
+      constexpr uint32_t xstep = L::kXbuf >> 4, hstep = kPreTileBytes >> 4;
+      const int halves = ROWS / 128;
       bool ok = true;
       RingCursor ac, xc;
       int t = 0;
       for (int u = cta; u < p.units && ok; u += G, ++t) {
         const PreUnit w = pre_unit(p, u);
-        const int b = t & 1;
+        // two accumulators used by alternate units, or (wide) by the two halves of every
+        // unit: then the epilogue of a unit must drain both before the next one starts
+        const int b = WIDE ? 0 : (t & 1);
+        const uint32_t ph = WIDE ? (t & 1) : ((t >> 1) & 1);
         const uint32_t acc = tmem + static_cast<uint32_t>(b * BNT);
-        if (!mbar_wait(&ctrl->accempty[b], ((t >> 1) & 1) ^ 1) || pre_aborted(ctrl)) {
+        if (!mbar_wait(&ctrl->accempty[b], ph ^ 1) || pre_aborted(ctrl)) {
           pre_timeout(p.status, ctrl);
           break;
         }
@@ -360,20 +381,24 @@ __global__ void __launch_bounds__(kPreThreads, 1)
           }
           tc_fence_after();
           const uint64_t dx = xdesc0 + sx * xstep;
-          if (it < w.nk) {
-            const uint64_t da = adesc0 + sa * astep;
-            mma_bf16_ss(acc, da, dx, idesc, it != 0);
-            mma_bf16_ss(acc, da + 2, dx + 2, idesc, 1u);
-            mma_bf16_ss(acc, da + 4, dx + 4, idesc, 1u);
-            mma_bf16_ss(acc, da + 6, dx + 6, idesc, 1u);
-          } else {
-            // B_cat^T chunk, MN-major: two 64-row halves 8 KB apart, 16 ranks = 2 KB
-            const int c = it - w.nk;
-            const int kk = min(4, (p.R16 - 64 * c) / 16);
-            const uint32_t a0 = smem_u32(abuf(sa));
-            for (int k = 0; k < kk; ++k)
-              mma_bf16_ss(acc, smem_desc_sw128(a0 + 2048 * k, 8192, 1024), dx + 2 * k, idesc_mn,
-                          1u);
+#pragma unroll 1
+          for (int hf = 0; hf < halves; ++hf) {
+            const uint32_t acch = acc + static_cast<uint32_t>(hf * BNT);
+            if (it < w.nk) {
+              const uint64_t da = adesc0 + sa * astep + hf * hstep;
+              mma_bf16_ss(acch, da, dx, idesc, it != 0);
+              mma_bf16_ss(acch, da + 2, dx + 2, idesc, 1u);
+              mma_bf16_ss(acch, da + 4, dx + 4, idesc, 1u);
+              mma_bf16_ss(acch, da + 6, dx + 6, idesc, 1u);
+            } else {
+              // B_cat^T chunk, MN-major: two 64-row halves 8 KB apart, 16 ranks = 2 KB
+              const int c = it - w.nk;
+              const int kk = min(4, (p.R16 - 64 * c) / 16);
+              const uint32_t a0 = smem_u32(abuf(sa) + hf * kPreTileBytes);
+              for (int k = 0; k < kk; ++k)
+                mma_bf16_ss(acch, smem_desc_sw128(a0 + 2048 * k, 8192, 1024), dx + 2 * k,
+                            idesc_mn, 1u);
+            }
           }
           mma_commit(&ctrl->aempty[sa]);
           mma_commit(&ctrl->xempty[sx]);
@@ -388,47 +413,58 @@ __global__ void __launch_bounds__(kPreThreads, 1)
     // ================================================================ epilogue (warps 2-5)
     const int q = warp & 3;  // TMEM lane quarter
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-    const int r = 32 * q + lane;  // weight row within the tile
+    const int r = 32 * q + lane;  // weight row within a 128-row half
+    const int halves = ROWS / 128;
     __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(p.Y);
     int t = 0;
     for (int u = cta; u < p.units; u += G, ++t) {
       const PreUnit w = pre_unit(p, u);
-      const int b = t & 1;
+      const int b = WIDE ? 0 : (t & 1);
+      const uint32_t ph = WIDE ? (t & 1) : ((t >> 1) & 1);
       const uint32_t acc = tmem + static_cast<uint32_t>(b * BNT);
-      bool ok = mbar_wait(&ctrl->accfull[b], (t >> 1) & 1) && !pre_aborted(ctrl);
+      bool ok = mbar_wait(&ctrl->accfull[b], ph) && !pre_aborted(ctrl);
       if (!ok) pre_timeout(p.status, ctrl);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int mvalid = min(BNT, p.M - w.j * BNT);
-      const size_t n = static_cast<size_t>(w.i) * 128 + r;
       const size_t row0 = static_cast<size_t>(w.j) * BNT;
       if (w.ns == 1) {
-        for (int c = 0; c < BNT; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(acc + lane_base + c, v);
-          tmem_ld_wait();
+#pragma unroll 1
+        for (int hf = 0; hf < halves; ++hf) {
+          const size_t n = static_cast<size_t>(w.i) * ROWS + hf * 128 + r;
+          const uint32_t acch = acc + static_cast<uint32_t>(hf * BNT);
+          for (int c = 0; c < BNT; c += 16) {
+            uint32_t v[16];
+            tmem_ld16(acch + lane_base + c, v);
+            tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (c + e < mvalid)
-              Y[(row0 + c + e) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
+            for (int e = 0; e < 16; ++e)
+              if (c + e < mvalid)
+                Y[(row0 + c + e) * p.N + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
+          }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->accempty[b]);
       } else {
         // split K: add into the tile's fp32 sum in L2, count in per warp; the warp that
-        // arrives last for these 32 rows writes Y and clears both.  The sum is token-major
-        // ([token][128 rows]), so that every reduction, load and store of a warp covers
+        // arrives last for these rows writes Y and clears both.  The sum is token-major
+        // ([token][ROWS rows]), so that every reduction, load and store of a warp covers
         // one 128-byte line.
         const size_t st = static_cast<size_t>(w.t - p.full);  // index among the split tiles
-        float* sum = p.acc + st * 128 * BNT + r;
-        for (int c = 0; c < BNT; c += 16) {
-          uint32_t v[16];
-          tmem_ld16(acc + lane_base + c, v);
-          tmem_ld_wait();
+        float* sum = p.acc + st * ROWS * BNT + r;
+#pragma unroll 1
+        for (int hf = 0; hf < halves; ++hf) {
+          const uint32_t acch = acc + static_cast<uint32_t>(hf * BNT);
+          for (int c = 0; c < BNT; c += 16) {
+            uint32_t v[16];
+            tmem_ld16(acch + lane_base + c, v);
+            tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (c + e < mvalid) red_add_f32(sum + (c + e) * 128, __uint_as_float(v[e]));
+            for (int e = 0; e < 16; ++e)
+              if (c + e < mvalid)
+                red_add_f32(sum + hf * 128 + (c + e) * ROWS, __uint_as_float(v[e]));
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -440,17 +476,23 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         if (lane == 0) last = atomicAdd(p.counters + cidx, 1u) == static_cast<uint32_t>(w.ns - 1);
         if (__shfl_sync(0xffffffffu, last, 0)) {
           __threadfence();
-          // 32 tokens per L2 round trip: a chunk's loads all go out before its stores
-          for (int c0 = 0; c0 < mvalid; c0 += 32) {
-            float tv[32];
+#pragma unroll 1
+          for (int hf = 0; hf < halves; ++hf) {
+            const size_t n = static_cast<size_t>(w.i) * ROWS + hf * 128 + r;
+            float* sh = sum + hf * 128;
+            // 32 tokens per L2 round trip: a chunk's loads all go out before its stores
+            for (int c0 = 0; c0 < mvalid; c0 += 32) {
+              float tv[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) tv[e] = c0 + e < mvalid ? __ldcg(sum + (c0 + e) * 128) : 0.f;
+              for (int e = 0; e < 32; ++e)
+                tv[e] = c0 + e < mvalid ? __ldcg(sh + (c0 + e) * ROWS) : 0.f;
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c0 + e < mvalid) {
-                Y[(row0 + c0 + e) * p.N + n] = __float2bfloat16_rn(tv[e]);
-                __stcg(sum + (c0 + e) * 128, 0.f);
-              }
+              for (int e = 0; e < 32; ++e)
+                if (c0 + e < mvalid) {
+                  Y[(row0 + c0 + e) * p.N + n] = __float2bfloat16_rn(tv[e]);
+                  __stcg(sh + (c0 + e) * ROWS, 0.f);
+                }
+            }
           }
           if (lane == 0) p.counters[cidx] = 0u;
         }

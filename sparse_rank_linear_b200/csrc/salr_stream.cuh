@@ -32,10 +32,10 @@
 // The only cross-CTA wait is for t, on the t-share CTAs, which finish their share without
 // waiting on anything.  Every wait is bounded.
 //
-// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-9 epilogue in two groups
-// (group 0 also the adapter's t share), 10.. decoders (a warp may only reach the TMEM
-// lanes 32 (warp % 4) .. + 31, so the four warps of a decoder group, consecutive, cover
-// the four quarters).
+// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 epilogue (also the
+// adapter's t share), 6.. decoders (a warp may only reach the TMEM lanes
+// 32 (warp % 4) .. + 31, so the four warps of a decoder group, consecutive, cover the
+// four quarters).
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -45,10 +45,10 @@
 
 namespace salr {
 
-constexpr int kStreamFixedWarps = 10;  // producer, MMA, 2 x 4 epilogue warps
-constexpr int kStreamGroups = 4;  // decoder groups, each decodes a different block
+constexpr int kStreamFixedWarps = 6;  // producer, MMA, 4 epilogue warps
+constexpr int kStreamGroups = 5;  // decoder groups, each decodes a different block
 constexpr int kStreamMaxUnitsPerCta = 4096;
-constexpr int kStreamMaxA = 8;   // rebuilt-block ring (TMEM slots)
+constexpr int kStreamMaxA = 16;  // rebuilt-block ring (TMEM slots)
 constexpr int kStreamMaxC = 16;  // compact-block ring
 
 struct StreamParams {
@@ -268,6 +268,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       }
     }
     int it = 0, nad = 0, obase = u0;
+    uint32_t ps = 0, pph = 0;  // compact-ring slot and phase of block `it` (lane 0)
     bool stop = false, bc_pending = false;
     for (int u = u0; u < u1 && !stop;) {
       const int i = u / KB, kba = u % KB;
@@ -288,8 +289,8 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
           if (it >= SC) dep_wait();
           if (ts_next < nts && ts_next > 0 && mbar_test_wait(smem_u32(&ctrl->tsfree), (ts_next - 1) & 1))
             issue_ts(ts_next++);
-          const int s = it % SC;
-          if (!mbar_wait(&ctrl->cempty[s], ((it / SC) & 1) ^ 1) || stream_aborted(ctrl)) {
+          const int s = static_cast<int>(ps);
+          if (!mbar_wait(&ctrl->cempty[s], pph ^ 1) || stream_aborted(ctrl)) {
             stream_timeout(p, ctrl);
             fail = 1;
           } else {
@@ -297,6 +298,10 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
             mbar_arrive_expect_tx(&ctrl->cfull[s], cb);
             bulk_g2s(cbuf(s), p.blob + static_cast<size_t>(o0) * 16, cb, &ctrl->cfull[s]);
             if (it == SC - 1) dep_wait();
+          }
+          if (++ps == static_cast<uint32_t>(SC)) {
+            ps = 0;
+            pph ^= 1u;
           }
         }
         if (__shfl_sync(0xffffffffu, fail, 0)) {
@@ -451,10 +456,10 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     }
   } else if (warp < kStreamFixedWarps) {
     // ================================================================ epilogue
-    // Two groups of four warps (2-5 and 6-9); group x drains accumulator x, i.e. the
-    // CTA's segments of that parity, so that two segment epilogues can overlap.  Group 0
-    // also handles this CTA's part of the shared t.
-    const int eg = (warp - 2) >> 2;               // epilogue group
+    // Four warps (2-5): this CTA's part of the shared t first, then the accumulators of
+    // the CTA's segments in order (two TMEM accumulators alternate, so the MMAs of the
+    // next segment run while one is drained).
+    const int eg = 0;                             // epilogue group
     const int bar_id = 1 + eg;                    // named barrier of the group
     const bool lead = threadIdx.x == 64 + 128 * eg;
     const int q = warp & 3;                       // TMEM lane quarter
@@ -559,7 +564,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       const int i = u / KB, kba = u % KB;
       const int kbb = min(KB, kba + (u1 - u));
       const int x = seg & 1;
-      if (x == eg) {
+      {
         bool okw = mbar_wait(&ctrl->accfull[x], (seg >> 1) & 1);
         if (!okw) stream_timeout(p, ctrl);
         okw = __all_sync(0xffffffffu, okw) && !stream_aborted(ctrl);
@@ -648,24 +653,28 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     const bool leader = (dw & 3) == 0 && lane == 0;  // issues the group's X-tile copies
     const uint32_t tlane = tmem_a + (static_cast<uint32_t>(32 * q) << 16);
     int last_x = -1;
+    // ring slots and phases of this group's blocks it = g, g + groups, ...: both rings
+    // hold a multiple of `groups` slots, so the slot advances by `groups` and wraps (with
+    // a phase flip) exactly when it crosses a multiple of the ring size
+    uint32_t sc = g, phc = 0, sa = g, pha = 0;
+    int kbx = (u0 + g) % KB;  // the block's K block, for its X tile
     griddep_wait();
     for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
-      const int sc = it % SC, sa = it % SA;
-      if (!mbar_wait(&ctrl->cfull[sc], (it / SC) & 1)) {
+      if (!mbar_wait(&ctrl->cfull[sc], phc)) {
         stream_timeout(p, ctrl);
         break;
       }
       const uint8_t* cb = cbuf(sc);
       const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb), q, lane);
       // ---- the TMEM slot must be free (its last MMAs complete); the group leader fetches X
-      if (!mbar_wait(&ctrl->aempty[sa], ((it / SA) & 1) ^ 1)) {
+      if (!mbar_wait(&ctrl->aempty[sa], pha ^ 1)) {
         stream_timeout(p, ctrl);
         break;
       }
       tc_fence_after();
       if (leader) {
         mbar_arrive_expect_tx(&ctrl->xfull[sa], BNT * 128);
-        tma_load_2d(xbuf(sa), &tmX, ((u0 + it) % KB) * 64, 0, &ctrl->xfull[sa]);
+        tma_load_2d(xbuf(sa), &tmX, kbx * 64, 0, &ctrl->xfull[sa]);
         last_x = it;
       }
       const uint32_t ts = tlane + 32u * sa;
@@ -682,6 +691,15 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         mbar_arrive(&ctrl->dec[sa]);
         mbar_arrive(&ctrl->cempty[sc]);
       }
+      if ((sc += kStreamGroups) >= static_cast<uint32_t>(SC)) {
+        sc -= SC;
+        phc ^= 1u;
+      }
+      if ((sa += kStreamGroups) >= static_cast<uint32_t>(SA)) {
+        sa -= SA;
+        pha ^= 1u;
+      }
+      for (kbx += kStreamGroups; kbx >= KB;) kbx -= KB;
     }
     if (leader && last_x >= 0 && stream_aborted(ctrl))
       mbar_wait(&ctrl->xfull[last_x % SA], (last_x / SA) & 1);  // own copy lands first

@@ -170,15 +170,26 @@ def test_linear_plan_of_the_workloads(lib):
             d128["units"], d128["grid"]) == (1, 2, 32, 0, 4, 128, 128)
     assert d128["split_sum_bytes"] == 32 * 128 * 128 * 4
     assert d128["dense_scratch_bytes"] == 0
+    # dense path.  256-row tiles only from 8 full rounds of them (up_proj and down_proj
+    # have fewer: 344 and 256 tiles of 256 rows on 148 SMs), so 128-row tiles here
     up = _plan(11008, 4096, 2048, 96)  # 688 tiles = 4 x 148 + 96; 96 x 3 = 288 -> 2 rounds of 1/3
-    assert (up["path"], up["kernels"], up["token_tile"], up["tiles"], up["whole_tiles"],
-            up["splits"], up["units"]) == (2, 3, 256, 688, 592, 3, 592 + 288)
+    assert (up["path"], up["kernels"], up["token_tile"], up["tile_rows"], up["tiles"],
+            up["whole_tiles"], up["splits"], up["units"]) == (2, 3, 256, 128, 688, 592, 3, 880)
     assert up["split_sum_bytes"] == 96 * 128 * 256 * 4
     assert up["dense_scratch_bytes"] == 11008 * 4096 * 2
     dn = _plan(4096, 11008, 4096, 128)  # 512 = 3 x 148 + 68; 68 x 2 = 136 -> 1 round of 1/2
-    assert (dn["tiles"], dn["whole_tiles"], dn["splits"], dn["units"]) == (512, 444, 2, 580)
-    lg = _plan(28672, 8192, 8192, 96)  # 7168 = 48 x 148 + 64
-    assert (lg["tiles"], lg["whole_tiles"], lg["splits"]) == (7168, 7104, 2)
+    assert (dn["tile_rows"], dn["tiles"], dn["whole_tiles"], dn["splits"], dn["units"]) == \
+        (128, 512, 444, 2, 580)
+    # 24 full rounds of 256-row tiles, and the busiest CTA gets no more 128-row block steps
+    # (2 x (24 x 128 + 32)) than with 128-row tiles (48 x 128 + 2 x 32)
+    lg = _plan(28672, 8192, 8192, 96)  # 3584 = 24 x 148 + 32; 32 x 4 = 128 -> 1 round of 1/4
+    assert (lg["tile_rows"], lg["tiles"], lg["whole_tiles"], lg["splits"]) == (256, 3584, 3552, 4)
+    # 256-row tiles would leave up_proj M = 512 at 86 tiles on 148 SMs: 128-row tiles
+    u512 = _plan(11008, 4096, 512)
+    assert (u512["tile_rows"], u512["tiles"], u512["whole_tiles"], u512["splits"]) == (128, 172, 148, 6)
+    # N not a multiple of 256, and the fused path, keep 128-row tiles
+    assert _plan(384, 256, 600)["tile_rows"] == 128
+    assert _plan(28672, 8192, 128, 96)["tile_rows"] == 128
     l128 = _plan(28672, 8192, 128, 96)  # 224 = 148 + 76; 76 x 7 = 532 -> 4 rounds of 1/7
     assert (l128["path"], l128["whole_tiles"], l128["splits"], l128["units"]) == (1, 148, 7, 680)
     u256 = _plan(11008, 4096, 256, 96)  # 86 tiles, 148 // 86 = 1: nothing split
@@ -217,7 +228,10 @@ def test_linear_plan_split_never_lengthens_a_cta(lib, sms):
         M = int(rng.integers(65, 20000))
         p = _plan(128 * RT, 64 * KB, M, 0, sms)
         tiles = p["tiles"]
-        assert tiles == RT * -(-M // p["token_tile"])
+        assert p["tile_rows"] in (128, 256)
+        if p["tile_rows"] == 256:
+            assert p["path"] == 2 and p["token_tile"] == 256 and RT % 2 == 0
+        assert tiles == 128 * RT // p["tile_rows"] * -(-M // p["token_tile"])
         s = p["splits"]
         assert p["units"] == p["whole_tiles"] + (tiles - p["whole_tiles"]) * s
         assert p["grid"] == min(p["units"], sms)
@@ -270,8 +284,8 @@ int main(void) {
   salr_plan p;
   int rc = salr_linear_plan(11008, 4096, 2048, 96, 148, &p);
   if (rc != SALR_OK) { printf("plan %d\n", rc); return 1; }
-  printf("%d %d %d %d %d %d %lld\n", p.path, p.kernels, p.tiles, p.whole_tiles, p.splits,
-         p.units, (long long)p.dense_scratch_bytes);
+  printf("%d %d %d %d %d %d %d %lld\n", p.path, p.kernels, p.tile_rows, p.tiles, p.whole_tiles,
+         p.splits, p.units, (long long)p.dense_scratch_bytes);
   if (strcmp(salr_status_string(SALR_ERR_UNSUPPORTED), "SALR_ERR_UNSUPPORTED") != 0) return 2;
   if (salr_free(NULL) != SALR_ERR_INVALID) return 3;
   return 0;
@@ -290,4 +304,4 @@ def test_header_is_plain_c_and_links_from_a_c_program(lib, tmp_path):
                    check=True, capture_output=True, text=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, out.stdout + out.stderr
-    assert out.stdout.split() == ["2", "3", "688", "592", "3", "880", str(11008 * 4096 * 2)]
+    assert out.stdout.split() == ["2", "3", "128", "688", "592", "3", "880", str(11008 * 4096 * 2)]

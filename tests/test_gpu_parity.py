@@ -312,6 +312,32 @@ def test_linear_split_tail_tiles_full_compare(R, N, K, M):
     h.free()
 
 
+@pytest.mark.parametrize("N,K,M", [(1280, 512, 384), (9728, 256, 384), (9472, 256, 1024),
+                                   (9728, 512, 1100)])
+@pytest.mark.parametrize("R", [0, 72])
+def test_linear_wide_tiles_full_compare(R, N, K, M, monkeypatch):
+    # dense path with 256-row tiles (two MMAs per X tile, two TMEM accumulators per unit):
+    # every tile split in 8 along K, whole tiles in one partial round, exactly one round,
+    # and 148 whole tiles plus 42 split in two with a ragged last token tile.  The library
+    # takes such tiles only from 8 full rounds on; the override reaches them here.
+    monkeypatch.setenv("SALR_WIDE_MIN_ROUNDS", "0")
+    if salr.plan(N, K, M, R)["tile_rows"] != 256:
+        pytest.skip("this GPU's SM count gives 128-row tiles for this shape")
+    wl = synth.Workload("wide", N, K, (R,) if R else (), (M,))
+    w, x = synth.weight(wl), synth.activations(wl, M)
+    ad = synth.adapters(wl)
+    h = salr.encode(to_dev(w), 0.5)
+    A = to_dev(ad[0][0]) if R else None
+    B = to_dev(ad[0][1]) if R else None
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    expect, bound = oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad)
+    for call in range(2):
+        Y = salr.linear(to_dev(x), h, A, B)
+        assert h.sync_status() == 0
+        assert_close(to_bits(Y), expect, bound, f"wide R={R} call {call}")
+    h.free()
+
+
 @pytest.mark.parametrize("M", [256, 64])
 def test_identity_rows_reproduce_decoded_columns_bitexact(M):
     # X = rows of the identity, no adapter: every output is a single product
