@@ -560,11 +560,22 @@ void bind_call(StreamParams& sp, float* acc, uint32_t* counters, float* tacc, ui
   sp.tflag = tflags;
 }
 
+// Compact blocks per bulk copy: as many as make about 40 KB (at most 4).  A bulk copy
+// occupies the SM's copy engine for about 540 cycles whatever its size (measured on B200
+// from L2: 2 to 32 KB per copy, 2 to 8 copies in flight, 1 or 148 CTAs), so copies of
+// single ~9 KB blocks cap a CTA near 17 bytes per cycle, about 5 TB/s over 148 SMs, before
+// anything else shares the engine.
+int stream_blocks_per_copy(uint32_t max16) {
+  const int blockb = static_cast<int>(max16) * 16;
+  const int b = 40960 / (blockb > 0 ? blockb : 1);
+  return b < 1 ? 1 : b > kStreamMaxBpc ? kStreamMaxBpc : b;
+}
+
 template <int BNT>
 int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
                   const CUtensorMap& tb, int sms, cudaStream_t st) {
   using L = StreamLayout<BNT>;
-  constexpr int kThreads = 32 * (kStreamFixedWarps + kStreamDecoders);
+  constexpr int kThreads = 32 * (kStreamFixedWarps + kStreamDecoders + kStreamGroups);
   p.bcbuf = L::bcat_bytes(p.R16);
   // rebuilt-block ring (TMEM slots, each with its X tile in shared memory): two per
   // decoder group, so that a group only ever waits for the MMAs of its own block before
@@ -572,13 +583,12 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   // blocks are in flight from HBM
   p.sa = 2 * kStreamGroups;
   const int fixed = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, 0);
-  // The compact-block slots come in a multiple of the group count, so that slot s only
-  // ever holds blocks of group s mod 4: a group never waits on a slot whose previous fill
-  // it has not consumed itself, and a parity wait can never pass on a phase two fills old.
+  // The rest of shared memory becomes super-slots, one bulk copy of p.bpc blocks each.  A
+  // super-slot is refilled only once every decoder warp of all its blocks has counted out,
+  // so no warp can wait on a fill two phases old.
   int sc = (kSmemLimit - fixed) / p.cbuf;
   if (sc > kStreamMaxC) sc = kStreamMaxC;
-  sc -= sc % kStreamGroups;
-  if (sc < kStreamGroups) return SALR_ERR_UNSUPPORTED;
+  if (sc < 2) return SALR_ERR_UNSUPPORTED;
   p.sc = sc;
   const int smem = L::smem_bytes(p.cbuf, p.bcbuf, p.sa, p.sc);
   static std::atomic<bool> attr_set[64];  // zero-initialised: false
@@ -857,7 +867,9 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
     sp.kblocks = static_cast<int>(h->K / 64);
     sp.RT = static_cast<int>(h->N / 128);
     sp.units = sp.RT * sp.kblocks;
-    sp.cbuf = static_cast<int>((h->max16 * 16 + 32 + 1023) / 1024 * 1024);
+    sp.bpc = stream_blocks_per_copy(h->max16);
+    sp.cbuf = static_cast<int>((sp.bpc * h->max16 * 16 + 32 + 1023) / 1024 * 1024);
+    sp.X = static_cast<const uint16_t*>(X);
     CUtensorMap tx, ta, tb;
     std::memset(&ta, 0, sizeof(ta));
     std::memset(&tb, 0, sizeof(tb));
@@ -1480,7 +1492,9 @@ extern "C" int salr_linear_noalloc(const void* X, int64_t M, salr_handle h, cons
   sp.kblocks = static_cast<int>(h->K / 64);
   sp.RT = static_cast<int>(h->N / 128);
   sp.units = sp.RT * sp.kblocks;
-  sp.cbuf = static_cast<int>((h->max16 * 16 + 32 + 1023) / 1024 * 1024);
+  sp.bpc = stream_blocks_per_copy(h->max16);
+  sp.cbuf = static_cast<int>((sp.bpc * h->max16 * 16 + 32 + 1023) / 1024 * 1024);
+  sp.X = static_cast<const uint16_t*>(X);
   CUtensorMap tx, ta, tb;
   std::memset(&ta, 0, sizeof(ta));
   std::memset(&tb, 0, sizeof(tb));

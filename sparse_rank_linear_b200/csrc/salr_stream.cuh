@@ -32,10 +32,10 @@
 // The only cross-CTA wait is for t, on the t-share CTAs, which finish their share without
 // waiting on anything.  Every wait is bounded.
 //
-// Warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 epilogue (also the
-// adapter's t share), 6.. decoders (a warp may only reach the TMEM lanes
+// Warp roles: 0 TMA producer, 1 TMEM allocator + adapter MMAs, 2-5 epilogue (also the
+// adapter's t share), 6-25 decoders (a warp may only reach the TMEM lanes
 // 32 (warp % 4) .. + 31, so the four warps of a decoder group, consecutive, cover the
-// four quarters).
+// four quarters), 26-30 the MMA issuers of the five decoder groups.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -49,9 +49,12 @@ constexpr int kStreamFixedWarps = 6;  // producer, MMA, 4 epilogue warps
 constexpr int kStreamGroups = 5;  // decoder groups, each decodes a different block
 constexpr int kStreamMaxUnitsPerCta = 4096;
 constexpr int kStreamMaxA = 16;  // rebuilt-block ring (TMEM slots)
-constexpr int kStreamMaxC = 16;  // compact-block ring
+constexpr int kStreamMaxC = 16;  // compact-block ring (super-slots of up to 4 blocks)
+constexpr int kStreamMaxBpc = 4;  // blocks per bulk copy
+constexpr int kStreamCtrlBytes = 2048;
 
 struct StreamParams {
+  const uint16_t* X;     // M x K bf16 activations (X tiles are read with ordinary loads)
   const uint8_t* blob;
   const uint32_t* offsets;
   uint16_t* Y;
@@ -66,7 +69,8 @@ struct StreamParams {
   int units;    // RT * kblocks
   int tshare;   // CTAs 0 .. tshare-1 compute a share of t (tshare = min(grid, kblocks))
   int treaders;  // CTAs that start a row tile (and read t): see stream_t_readers
-  int cbuf;     // per-stage bytes for one compact block (bitmap + values), multiple of 1024
+  int cbuf;     // bytes of a super-slot: bpc compact blocks + 32, multiple of 1024
+  int bpc;      // compact blocks per bulk copy (1 .. 4)
   int bcbuf;    // bytes of the B_cat^T tile / t-share buffer (0 without adapter), x1024
   int sa;       // entries of the decoded-tile ring (tile + X tile each)
   int sc;       // entries of the compact-block ring
@@ -94,22 +98,26 @@ struct StreamLayout {
   __host__ __device__ static int c_off(int sa) { return sa * kAent; }
   __host__ __device__ static int fixed_off(int cbuf, int sa, int sc) { return c_off(sa) + sc * cbuf; }
   __host__ __device__ static int smem_bytes(int cbuf, int bcbuf, int sa, int sc) {
-    return fixed_off(cbuf, sa, sc) + kTbuf + bcbuf + 1024 /*ctrl*/ + 128 /*nibbles*/ +
+    return fixed_off(cbuf, sa, sc) + kTbuf + bcbuf + kStreamCtrlBytes + 128 /*nibbles*/ +
            1024 /*align*/;
   }
 };
 
 struct StreamCtrl {
   uint64_t cfull[kStreamMaxC], cempty[kStreamMaxC];
-  uint64_t dec[kStreamMaxA], xfull[kStreamMaxA], aempty[kStreamMaxA];
-  uint64_t accfull[2], accempty[2];
+  uint64_t dec[kStreamMaxA], aempty[kStreamMaxA];
+  uint64_t gdone[kStreamGroups][2];  // a group's MMAs of a segment on accumulator x done
+  uint64_t gfin[kStreamGroups];      // a group's last MMAs done (before TMEM is freed)
+  uint64_t adone[2];                 // the adapter MMAs of a segment on accumulator x done
+  uint64_t accempty[2];              // accumulator x drained and zeroed by the epilogue
   uint64_t bcfull, bcempty, tready, tsfull, tsfree, tsdone, fin;
   uint32_t tmem;
   int abort;
   int flag[2];
+  uint32_t boff[kStreamMaxC][4];  // byte offset of each block of a super-slot's copy
 };
 
-static_assert(sizeof(StreamCtrl) <= 1024, "control block");
+static_assert(sizeof(StreamCtrl) <= kStreamCtrlBytes, "control block");
 
 __device__ __forceinline__ void stream_timeout(const StreamParams& p, StreamCtrl* c) {
   atomicOr(p.status, DEV_ERR_TIMEOUT);
@@ -158,7 +166,7 @@ __device__ __forceinline__ int owner_of(long long u, long long U, int G) {
 }
 
 template <int BNT, int NDEC>
-__global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
+__global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups), 1)
     salr_stream_kernel(const __grid_constant__ StreamParams p,
                        const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmA,
@@ -173,7 +181,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
   uint8_t* tbuf = smem + L::fixed_off(p.cbuf, SA, SC);
   uint8_t* bcbuf = tbuf + L::kTbuf;  // B_cat^T tile; at kernel start, the t-share stage
   StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(bcbuf + p.bcbuf);
-  uint2* ntab = reinterpret_cast<uint2*>(bcbuf + p.bcbuf + 1024);  // 16 x 8 B nibble table
+  uint2* ntab = reinterpret_cast<uint2*>(bcbuf + p.bcbuf + kStreamCtrlBytes);  // 16 x 8 B
 
   griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -196,17 +204,18 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < SC; ++s) {
       mbar_init(&ctrl->cfull[s], 1);
-      mbar_init(&ctrl->cempty[s], NDEC / kStreamGroups);
+      mbar_init(&ctrl->cempty[s], p.bpc * (NDEC / kStreamGroups));  // every warp of its blocks
     }
     for (int s = 0; s < SA; ++s) {
       mbar_init(&ctrl->dec[s], NDEC / kStreamGroups);
-      mbar_init(&ctrl->xfull[s], 1);
       mbar_init(&ctrl->aempty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&ctrl->accfull[x], 1);
+      for (int g = 0; g < kStreamGroups; ++g) mbar_init(&ctrl->gdone[g][x], 1);
+      mbar_init(&ctrl->adone[x], 1);
       mbar_init(&ctrl->accempty[x], 4);
     }
+    for (int g = 0; g < kStreamGroups; ++g) mbar_init(&ctrl->gfin[g], 1);
     mbar_init(&ctrl->bcfull, 1);
     mbar_init(&ctrl->bcempty, 1);
     mbar_init(&ctrl->tready, 4);
@@ -267,66 +276,84 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         prefetch_tmap(&tmB);
       }
     }
-    int it = 0, nad = 0, obase = u0;
-    uint32_t ps = 0, pph = 0;  // compact-ring slot and phase of block `it` (lane 0)
+    // Copies of `bpc` consecutive blocks at a time (one bulk copy costs the SM's copy
+    // engine about the same time whatever its size, so few large copies stream faster
+    // than many small ones).  Copy j lands in super-slot j % SC; the byte offset of each
+    // of its blocks is written to boff[slot][k] before the copy's barrier arrival.
+    const int nunits = u1 - u0, bpc = p.bpc;
+    int nad = 0, obase = u0, ncopies = 0;
+    uint32_t ps = 0, pph = 0;  // super-slot and phase of the next copy (lane 0)
+    // segment cursor of the B_cat tiles: row tile si holds CTA positions [.., send)
+    int si = u0 / KB, send = min(u1, (u0 / KB + 1) * KB) - u0;
+    bool sfirst = u0 % KB == 0, sleft = nunits > 0;
     bool stop = false, bc_pending = false;
-    for (int u = u0; u < u1 && !stop;) {
-      const int i = u / KB, kba = u % KB;
-      const int kbb = min(KB, kba + (u1 - u));
-      for (int kb = kba; kb < kbb; ++kb, ++it) {
-        const int unit = i * KB + kb;
-        if (unit >= obase + 32) {
-          obase = unit;
-          offv = (obase + lane <= p.units) ? __ldg(p.offsets + obase + lane) : 0u;
-          offx = (obase + 32 <= p.units) ? __ldg(p.offsets + obase + 32) : 0u;
+    for (int it0 = 0; it0 < nunits && !stop; it0 += bpc) {
+      const int nb = min(bpc, nunits - it0);
+      if (u0 + it0 + nb > obase + 32) {
+        obase = u0 + it0;
+        offv = (obase + lane <= p.units) ? __ldg(p.offsets + obase + lane) : 0u;
+        offx = (obase + 32 <= p.units) ? __ldg(p.offsets + obase + 32) : 0u;
+      }
+      const int k0 = u0 + it0 - obase;  // 0 .. 31; k0 + nb <= 32
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t v = __shfl_sync(0xffffffffu, offv, (k0 + k) & 31);
+        o[k] = (k0 + k < 32) ? v : offx;
+      }
+      const uint32_t oe = __shfl_sync(0xffffffffu, offv, (k0 + nb) & 31);
+      const uint32_t o_end = (k0 + nb < 32) ? oe : offx;  // the copy's end
+      int fail = 0;
+      if (lane == 0) {
+        if (ncopies >= SC) dep_wait();
+        if (ts_next < nts && ts_next > 0 && mbar_test_wait(smem_u32(&ctrl->tsfree), (ts_next - 1) & 1))
+          issue_ts(ts_next++);
+        const int s = static_cast<int>(ps);
+        if (!mbar_wait(&ctrl->cempty[s], pph ^ 1) || stream_aborted(ctrl)) {
+          stream_timeout(p, ctrl);
+          fail = 1;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (k < nb) ctrl->boff[s][k] = (o[k] - o[0]) * 16u;
+          const uint32_t cb = (o_end - o[0]) * 16u;
+          mbar_arrive_expect_tx(&ctrl->cfull[s], cb);
+          bulk_g2s(cbuf(s), p.blob + static_cast<size_t>(o[0]) * 16, cb, &ctrl->cfull[s]);
+          if (++ncopies == SC) dep_wait();
         }
-        const int k = unit - obase;
-        const uint32_t o0 = __shfl_sync(0xffffffffu, offv, k);
-        const uint32_t o1n = __shfl_sync(0xffffffffu, offv, (k + 1) & 31);
-        const uint32_t o1 = (k + 1 < 32) ? o1n : offx;
-        int fail = 0;
-        if (lane == 0) {
-          if (it >= SC) dep_wait();
-          if (ts_next < nts && ts_next > 0 && mbar_test_wait(smem_u32(&ctrl->tsfree), (ts_next - 1) & 1))
-            issue_ts(ts_next++);
-          const int s = static_cast<int>(ps);
-          if (!mbar_wait(&ctrl->cempty[s], pph ^ 1) || stream_aborted(ctrl)) {
-            stream_timeout(p, ctrl);
-            fail = 1;
-          } else {
-            const uint32_t cb = (o1 - o0) * 16u;
-            mbar_arrive_expect_tx(&ctrl->cfull[s], cb);
-            bulk_g2s(cbuf(s), p.blob + static_cast<size_t>(o0) * 16, cb, &ctrl->cfull[s]);
-            if (it == SC - 1) dep_wait();
-          }
-          if (++ps == static_cast<uint32_t>(SC)) {
-            ps = 0;
-            pph ^= 1u;
-          }
-        }
-        if (__shfl_sync(0xffffffffu, fail, 0)) {
-          stop = true;
-          break;
+        if (++ps == static_cast<uint32_t>(SC)) {
+          ps = 0;
+          pph ^= 1u;
         }
       }
-      if (!stop && adapter && kba == 0) {
-        int fail = 0;
-        if (lane == 0) {
-          dep_wait();
-          if (!finish_ts() || !mbar_wait(&ctrl->bcempty, (nad & 1) ^ 1)) {
-            stream_timeout(p, ctrl);
-            fail = 1;
-          } else {
-            mbar_arrive_expect_tx(&ctrl->bcfull, 256u * p.R16);
-            tma_load_2d(bcbuf, &tmB, i * 128, 0, &ctrl->bcfull);
-            tma_load_2d(bcbuf + p.R16 * 128, &tmB, i * 128 + 64, 0, &ctrl->bcfull);
-            bc_pending = true;
-          }
-        }
-        ++nad;
-        if (__shfl_sync(0xffffffffu, fail, 0)) stop = true;
+      if (__shfl_sync(0xffffffffu, fail, 0)) {
+        stop = true;
+        break;
       }
-      u = i * KB + kbb;
+      // B_cat tiles of the row tiles whose last block of this CTA has now been requested
+      while (!stop && sleft && send <= it0 + nb) {
+        if (adapter && sfirst) {
+          int bfail = 0;
+          if (lane == 0) {
+            dep_wait();
+            if (!finish_ts() || !mbar_wait(&ctrl->bcempty, (nad & 1) ^ 1)) {
+              stream_timeout(p, ctrl);
+              bfail = 1;
+            } else {
+              mbar_arrive_expect_tx(&ctrl->bcfull, 256u * p.R16);
+              tma_load_2d(bcbuf, &tmB, si * 128, 0, &ctrl->bcfull);
+              tma_load_2d(bcbuf + p.R16 * 128, &tmB, si * 128 + 64, 0, &ctrl->bcfull);
+              bc_pending = true;
+            }
+          }
+          ++nad;
+          if (__shfl_sync(0xffffffffu, bfail, 0)) stop = true;
+        }
+        sleft = send < nunits;
+        ++si;
+        sfirst = true;
+        send = min(send + KB, nunits);
+      }
     }
     if (lane == 0) {
       dep_wait();
@@ -334,19 +361,28 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
       if (stream_aborted(ctrl)) {
         // let copies this thread started land before the CTA may exit
         for (int s = 0; s < SC; ++s)
-          if (it > s) mbar_wait(&ctrl->cfull[(it - 1 - s) % SC], ((it - 1 - s) / SC) & 1);
+          if (ncopies > s) mbar_wait(&ctrl->cfull[(ncopies - 1 - s) % SC], ((ncopies - 1 - s) / SC) & 1);
         if (bc_pending) mbar_wait(&ctrl->bcfull, (nad - 1) & 1);
         if (ts_next > 0) mbar_wait(&ctrl->tsfull, (ts_next - 1) & 1);
       }
     }
   } else if (warp == 1) {
-    // ================================================================ MMA issuer
+    // ================================================================ adapter MMAs
+    // The blocks' MMAs are issued by the decoder groups themselves (one issuing thread
+    // per group: a thread takes ~40 cycles to issue one tcgen05.mma, so one thread for
+    // all of them would cap the block rate).  This thread multiplies this CTA's t shares
+    // as they land, then adds B_cat^T t^T into the accumulator of every segment that
+    // starts a row tile.  All MMAs into an accumulator accumulate; the epilogue zeroes it
+    // after draining it.
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(128, BNT, 0, 0);
       constexpr uint32_t idesc_mn = idesc_bf16(128, BNT, 1, 0);
       bool ok = true;
       int ts_done = 0;  // t-share rounds multiplied so far
-      auto mma_ts = [&]() {
+      while (ok && ts_done < nts) {
+        if (!mbar_wait(&ctrl->tsfull, ts_done & 1) || stream_aborted(ctrl)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t a0 = smem_u32(bcbuf), x0 = smem_u32(bcbuf + 16384);
 #pragma unroll
@@ -355,102 +391,32 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
                       smem_desc_sw128(x0 + 32 * k, 16, 1024), idesc_mn, (ts_done | k) != 0);
         mma_commit(&ctrl->tsfree);
         if (++ts_done == nts) mma_commit(&ctrl->tsdone);
-      };
-      // the t share is multiplied as soon as its data has landed (polled between blocks),
-      // never ahead of decoded blocks: it is fetched only after the dependency wait
-      // The block loop runs on one thread that shares its SM sub-partition with decoder
-      // warps, so it is kept short: X descriptors differ from slot 0's only in the
-      // start-address field (address >> 4, which never carries past its 14 bits in shared
-      // memory), slot s's A operand is TMEM columns 32 s .. of the ring, and the slot index
-      // and its phase parity advance without division.
-      const uint64_t xdesc0 = smem_desc_sw128(smem_u32(xbuf(0)), 16, 1024);
-      constexpr uint32_t kSlotStep = L::kAent >> 4;
-      uint32_t dec0 = smem_u32(&ctrl->dec[0]), xf0 = smem_u32(&ctrl->xfull[0]);
-      int s = 0;
-      uint32_t ph = 0;
+      }
       int seg = 0, nad = 0;
-      for (int u = u0; u < u1 && ok && !stream_aborted(ctrl); ++seg) {
+      for (int u = u0; u < u1 && ok && adapter; ++seg) {
         const int i = u / KB, kba = u % KB;
         const int kbb = min(KB, kba + (u1 - u));
-        const int x = seg & 1;
-        if (!mbar_wait(&ctrl->accempty[x], ((seg >> 1) & 1) ^ 1)) {
-          stream_timeout(p, ctrl);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t acc = tmem + x * BNT;
-        for (int kb = kba; kb < kbb; ++kb) {
-          if (ts_done < nts && mbar_test_wait(smem_u32(&ctrl->tsfull), ts_done & 1)) mma_ts();
-          if (ts_done < nts) {
-            // while the block is still being decoded, take the t share once it has landed
-            const long long t0 = clock64();
-            while (!mbar_test_wait(dec0 + 8 * s, ph)) {
-              if (ts_done < nts && mbar_test_wait(smem_u32(&ctrl->tsfull), ts_done & 1)) mma_ts();
-              if (clock64() - t0 > kWaitLimitCycles || stream_aborted(ctrl)) {
-                ok = false;
-                break;
-              }
-              __nanosleep(32);
-            }
-            if (!ok) {
-              stream_timeout(p, ctrl);
-              break;
-            }
-          } else if (!mbar_try_wait(dec0 + 8 * s, ph) && !mbar_wait(&ctrl->dec[s], ph)) {
-            stream_timeout(p, ctrl);
-            ok = false;
-            break;
-          }
-          if (!mbar_try_wait(xf0 + 8 * s, ph) && !mbar_wait(&ctrl->xfull[s], ph)) {
-            stream_timeout(p, ctrl);
+        if (kba == 0) {
+          const int x = seg & 1;
+          if (!mbar_wait(&ctrl->accempty[x], (seg >> 1) & 1) || !mbar_wait(&ctrl->tready, 0) ||
+              !mbar_wait(&ctrl->bcfull, nad & 1) || stream_aborted(ctrl)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t ta = tmem_a + 32u * s;
-          const uint64_t dx = xdesc0 + s * kSlotStep;
-          mma_bf16_ts(acc, ta, dx, idesc, kb != kba);
-          mma_bf16_ts(acc, ta + 8, dx + 2, idesc, 1u);
-          mma_bf16_ts(acc, ta + 16, dx + 4, idesc, 1u);
-          mma_bf16_ts(acc, ta + 24, dx + 6, idesc, 1u);
-          mma_commit(&ctrl->aempty[s]);
-          if (++s == SA) {
-            s = 0;
-            ph ^= 1u;
-          }
-        }
-        if (!ok) break;
-        if (adapter && kba == 0) {
-          while (ok && ts_done < nts) {
-            if (!mbar_wait(&ctrl->tsfull, ts_done & 1)) {
-              ok = false;
-              break;
-            }
-            mma_ts();
-          }
-          if (!ok || !mbar_wait(&ctrl->tready, 0) || !mbar_wait(&ctrl->bcfull, nad & 1)) {
-            stream_timeout(p, ctrl);
-            break;
-          }
-          tc_fence_after();
+          const uint32_t acc = tmem + x * BNT;
           const uint32_t b0 = smem_u32(bcbuf), t0 = smem_u32(tbuf);
           for (int k = 0; k < p.R16 / 16; ++k)
             mma_bf16_ss(acc, smem_desc_sw128(b0 + 2048 * k, p.R16 * 128, 1024),
                         smem_desc_sw128(t0 + (k >> 2) * (BNT * 128) + (k & 3) * 32, 16, 1024),
                         idesc_mn, 1);
           mma_commit(&ctrl->bcempty);
+          mma_commit(&ctrl->adone[x]);
           ++nad;
         }
-        mma_commit(&ctrl->accfull[x]);
         u = i * KB + kbb;
       }
-      while (ok && !stream_aborted(ctrl) && ts_done < nts) {
-        if (!mbar_wait(&ctrl->tsfull, ts_done & 1)) {
-          stream_timeout(p, ctrl);
-          break;
-        }
-        mma_ts();
-      }
+      if (!ok) stream_timeout(p, ctrl);
       mma_commit(&ctrl->fin);
       if (!mbar_wait(&ctrl->fin, 0)) stream_timeout(p, ctrl);
     }
@@ -467,6 +433,19 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     const int r = 32 * q + lane;  // weight row within the tile; rank index for t
     __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(p.Y);
     volatile int* gflag = &ctrl->flag[eg];
+    // ---- 0. both accumulators start at zero (every MMA into them accumulates); their
+    //         accempty phase 0 lets the first two segments' MMAs in
+    auto zero_acc = [&](int x) {
+#pragma unroll
+      for (int c = 0; c < BNT; c += 8)
+        tmem_st8(tmem + x * BNT + lane_base + c, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->accempty[x]);
+    };
+    zero_acc(0);
+    zero_acc(1);
     griddep_wait();
     if (eg == 0) {
       bool ok = true;
@@ -556,16 +535,33 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
         }
       }
     }
-    // ---- 3. segments of this group's parity: drain the accumulator, then write Y or, for
-    //         a split tile, add the partial into the tile's fp32 sum in L2; the last of
-    //         the tile's segments to count itself in writes Y and clears the sum
+    // ---- 3. the CTA's segments in order: wait until every decoder group with blocks in
+    //         the segment (and the adapter, if the segment applies it) has seen its MMAs
+    //         complete, drain the accumulator, zero it for its next segment, then write Y
+    //         or, for a split tile, add the partial into the tile's fp32 sum in L2; the
+    //         last of the tile's segments to count itself in writes Y and clears the sum
     int seg = 0;
+    uint32_t gph = 0, aph = 0;  // phase parities of gdone[g][x] (bit 2g + x), adone[x] (bit x)
     for (int u = u0; u < u1; ++seg) {
       const int i = u / KB, kba = u % KB;
       const int kbb = min(KB, kba + (u1 - u));
       const int x = seg & 1;
       {
-        bool okw = mbar_wait(&ctrl->accfull[x], (seg >> 1) & 1);
+        const int itA = u - u0, nb = kbb - kba;  // the segment's blocks, by CTA position
+        bool okw = true;
+#pragma unroll
+        for (int g = 0; g < kStreamGroups; ++g) {
+          const int gg = (itA + g) % kStreamGroups;  // groups of blocks itA, itA + 1, ...
+          if (g < nb) {
+            const uint32_t bit = 1u << (2 * gg + x);
+            okw = okw && mbar_wait(&ctrl->gdone[gg][x], (gph & bit) ? 1u : 0u);
+            gph ^= bit;
+          }
+        }
+        if (adapter && kba == 0) {
+          okw = okw && mbar_wait(&ctrl->adone[x], (aph >> x) & 1u);
+          aph ^= 1u << x;
+        }
         if (!okw) stream_timeout(p, ctrl);
         okw = __all_sync(0xffffffffu, okw) && !stream_aborted(ctrl);
         named_bar(bar_id, 128);
@@ -595,9 +591,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
                               __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->accempty[x]);
+        zero_acc(x);
         if (!whole) {
           // Each warp counts its 32 rows of the tile in on its own: its additions are
           // performed first (fence), and the warp that arrives last for these rows reads
@@ -648,61 +642,149 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC), 1)
     // the same numbers (the only lanes a warp may write).
     static_assert(NDEC == 4 * kStreamGroups, "four warps, one per row quarter, in each group");
     const int dw = warp - kStreamFixedWarps;
-    const int g = dw >> 2, q = warp & 3;
     const int nunits = u1 - u0;
-    const bool leader = (dw & 3) == 0 && lane == 0;  // issues the group's X-tile copies
-    const uint32_t tlane = tmem_a + (static_cast<uint32_t>(32 * q) << 16);
-    int last_x = -1;
-    // ring slots and phases of this group's blocks it = g, g + groups, ...: both rings
-    // hold a multiple of `groups` slots, so the slot advances by `groups` and wraps (with
-    // a phase flip) exactly when it crosses a multiple of the ring size
-    uint32_t sc = g, phc = 0, sa = g, pha = 0;
-    int kbx = (u0 + g) % KB;  // the block's K block, for its X tile
-    griddep_wait();
-    for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
-      if (!mbar_wait(&ctrl->cfull[sc], phc)) {
-        stream_timeout(p, ctrl);
-        break;
+    // ring slots and phases of group g's blocks it = g, g + groups, ...: both rings hold a
+    // multiple of `groups` slots, so the slot advances by `groups` and wraps (with a phase
+    // flip) exactly when it crosses a multiple of the ring size
+    if (dw < NDEC) {
+      const int g = dw >> 2, q = warp & 3;
+      const uint32_t tlane = tmem_a + (static_cast<uint32_t>(32 * q) << 16);
+      // block it lives in copy it / bpc (super-slot sc, phase phc) at block kc of it
+      const int bpc = p.bpc;
+      uint32_t sc = 0, phc = 0, sa = g, pha = 0;
+      int kc = g;
+      for (; kc >= bpc; kc -= bpc)
+        if (++sc == static_cast<uint32_t>(SC)) {
+          sc = 0;
+          phc ^= 1u;
+        }
+      griddep_wait();
+      for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
+        if (!mbar_wait(&ctrl->cfull[sc], phc)) {
+          stream_timeout(p, ctrl);
+          break;
+        }
+        const uint8_t* cb = cbuf(sc) + ctrl->boff[sc][kc];
+        const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb), q, lane);
+        // ---- the TMEM slot must be free: the MMAs of its previous block have completed
+        if (!mbar_wait(&ctrl->aempty[sa], pha ^ 1)) {
+          stream_timeout(p, ctrl);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ts = tlane + 32u * sa;
+        uint32_t r[8];
+        expand_quarter(qp, cb + kBitmapBytes, ntab, [&](int n, uint32_t w0, uint32_t w1) {
+          r[2 * (n & 3)] = w0;
+          r[2 * (n & 3) + 1] = w1;
+          if ((n & 3) == 3) tmem_st8(ts + 8 * (n >> 2), r[0], r[1], r[2], r[3], r[4], r[5], r[6], r[7]);
+        });
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&ctrl->dec[sa]);
+          mbar_arrive(&ctrl->cempty[sc]);
+        }
+        for (kc += kStreamGroups; kc >= bpc; kc -= bpc)
+          if (++sc == static_cast<uint32_t>(SC)) {
+            sc = 0;
+            phc ^= 1u;
+          }
+        if ((sa += kStreamGroups) >= static_cast<uint32_t>(SA)) {
+          sa -= SA;
+          pha ^= 1u;
+        }
       }
-      const uint8_t* cb = cbuf(sc);
-      const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb), q, lane);
-      // ---- the TMEM slot must be free (its last MMAs complete); the group leader fetches X
-      if (!mbar_wait(&ctrl->aempty[sa], pha ^ 1)) {
-        stream_timeout(p, ctrl);
-        break;
+    } else {
+      // ============================================================== MMA issuers
+      // One warp per decoder group (a thread needs ~40 cycles to issue one tcgen05.mma,
+      // and warps issue in parallel).  For each of its group's blocks, once the TMEM slot
+      // is free: the warp loads the block's X tile (BNT tokens x 64, rows past M zero)
+      // with ordinary loads into the slot's 128-byte-swizzled X buffer (a TMA per block
+      // would cost the SM's copy engine as much as a compact-block copy); then lane 0,
+      // once the four quarters are in TMEM, issues the block's four MMAs into the
+      // accumulator of the block's segment.  Every MMA accumulates (the epilogue zeroes an
+      // accumulator after draining it).  After the group's last block of a segment, lane 0
+      // commits gdone[g][x] for the epilogue.
+      const int g = dw - NDEC;
+      uint32_t sa = g, pha = 0;
+      int kbx = (u0 + g) % KB;  // the block's K block, for its X tile
+      int seg = 0, seg_waited = -1;  // segment `seg` holds CTA positions [.., segEnd)
+      int segEnd = min(u1, (u0 / KB + 1) * KB) - u0;
+      constexpr uint32_t idesc = idesc_bf16(128, BNT, 0, 0);
+      const uint64_t xdesc0 = smem_desc_sw128(smem_u32(xbuf(0)), 16, 1024);
+      constexpr uint32_t kSlotStep = L::kAent >> 4;  // X descriptors differ in the address only
+      constexpr int kXChunks = BNT * 8 / 32;  // 16-byte chunks of an X tile per lane
+      static_assert(kXChunks % 4 == 0, "X chunks per lane in fours");
+      bool issued = false;
+      griddep_wait();
+      for (int it = g; it < nunits; it += kStreamGroups) {
+        while (it >= segEnd) {
+          ++seg;
+          segEnd = min(segEnd + KB, nunits);
+        }
+        const int x = seg & 1;
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&ctrl->aempty[sa], pha ^ 1) && !stream_aborted(ctrl);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          if (lane == 0) stream_timeout(p, ctrl);
+          break;
+        }
+        // ---- X tile of the block: row m (token) at m * 128, chunk c at (c ^ (m & 7)) * 16
+        uint8_t* xb = xbuf(sa);
+#pragma unroll
+        for (int t0 = 0; t0 < kXChunks; t0 += 4) {  // 4 loads in flight per lane at a time
+          uint4 v[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int e = lane + 32 * (t0 + t), m = e >> 3, c = e & 7;
+            v[t] = m < p.M ? __ldg(reinterpret_cast<const uint4*>(
+                                 p.X + static_cast<size_t>(m) * p.K + kbx * 64) + c)
+                           : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int e = lane + 32 * (t0 + t), m = e >> 3, c = e & 7;
+            *reinterpret_cast<uint4*>(xb + m * 128 + ((c ^ (m & 7)) << 4)) = v[t];
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (seg_waited != seg) {
+            ok = mbar_wait(&ctrl->accempty[x], (seg >> 1) & 1);
+            seg_waited = seg;
+          }
+          ok = ok && mbar_wait(&ctrl->dec[sa], pha);
+          if (!ok) {
+            stream_timeout(p, ctrl);
+          } else {
+            tc_fence_after();
+            const uint32_t acc = tmem + x * BNT, ta = tmem_a + 32u * sa;
+            const uint64_t dx = xdesc0 + sa * kSlotStep;
+            mma_bf16_ts(acc, ta, dx, idesc, 1u);
+            mma_bf16_ts(acc, ta + 8, dx + 2, idesc, 1u);
+            mma_bf16_ts(acc, ta + 16, dx + 4, idesc, 1u);
+            mma_bf16_ts(acc, ta + 24, dx + 6, idesc, 1u);
+            mma_commit(&ctrl->aempty[sa]);
+            if (it + kStreamGroups >= segEnd) mma_commit(&ctrl->gdone[g][x]);
+            issued = true;
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        if ((sa += kStreamGroups) >= static_cast<uint32_t>(SA)) {
+          sa -= SA;
+          pha ^= 1u;
+        }
+        for (kbx += kStreamGroups; kbx >= KB;) kbx -= KB;
       }
-      tc_fence_after();
-      if (leader) {
-        mbar_arrive_expect_tx(&ctrl->xfull[sa], BNT * 128);
-        tma_load_2d(xbuf(sa), &tmX, kbx * 64, 0, &ctrl->xfull[sa]);
-        last_x = it;
+      // every MMA this thread issued has completed before the TMEM can be freed
+      if (lane == 0 && issued) {
+        mma_commit(&ctrl->gfin[g]);
+        if (!mbar_wait(&ctrl->gfin[g], 0)) stream_timeout(p, ctrl);
       }
-      const uint32_t ts = tlane + 32u * sa;
-      uint32_t r[8];
-      expand_quarter(qp, cb + kBitmapBytes, ntab, [&](int n, uint32_t w0, uint32_t w1) {
-        r[2 * (n & 3)] = w0;
-        r[2 * (n & 3) + 1] = w1;
-        if ((n & 3) == 3) tmem_st8(ts + 8 * (n >> 2), r[0], r[1], r[2], r[3], r[4], r[5], r[6], r[7]);
-      });
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&ctrl->dec[sa]);
-        mbar_arrive(&ctrl->cempty[sc]);
-      }
-      if ((sc += kStreamGroups) >= static_cast<uint32_t>(SC)) {
-        sc -= SC;
-        phc ^= 1u;
-      }
-      if ((sa += kStreamGroups) >= static_cast<uint32_t>(SA)) {
-        sa -= SA;
-        pha ^= 1u;
-      }
-      for (kbx += kStreamGroups; kbx >= KB;) kbx -= KB;
     }
-    if (leader && last_x >= 0 && stream_aborted(ctrl))
-      mbar_wait(&ctrl->xfull[last_x % SA], (last_x / SA) & 1);  // own copy lands first
   }
 
   tc_fence_before();

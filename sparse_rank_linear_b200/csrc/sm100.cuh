@@ -226,14 +226,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 
 // Store 8 consecutive 32-bit TMEM columns of this thread's lane (shape 32x32b: thread i
-// of the warp writes lane 32 (warp % 4) + i).
+// of the warp writes lane 32 (warp % 4) + i).  No memory clobber: the store touches only
+// tensor memory, so ordinary loads may be scheduled across it; it stays ordered with the
+// other tcgen05 and mbarrier instructions (all volatile asm).
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2,
                                          uint32_t r3, uint32_t r4, uint32_t r5, uint32_t r6,
                                          uint32_t r7) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-      "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(r4), "r"(r5), "r"(r6), "r"(r7)
-      : "memory");
+      "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(r4), "r"(r5), "r"(r6), "r"(r7));
 }
 
 // Wait until this thread's tcgen05.st have completed.
