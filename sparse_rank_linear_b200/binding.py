@@ -10,7 +10,9 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libsalr.so")
+# The built library; SALR_LIBRARY names another build of it (the bounds-checked debug
+# build, libsalr_checks.so) to load instead.
+LIB_PATH = os.environ.get("SALR_LIBRARY") or os.path.join(HERE, "libsalr.so")
 
 SALR_OK = 0
 SALR_ERR_INVALID = 1

@@ -33,23 +33,30 @@ def command(out: str = LIB, extra=()) -> list:
             *[os.path.join(CSRC, s) for s in SOURCES], "-o", out, "-cudart", "static"]
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps.append(os.path.join(ROOT, "include", "salr.h"))
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if force or stale():
-        cmd = command()
+# Debug build: every data-derived offset in the kernels is checked; a failed check sets
+# the range bit of the handle's status word (salr_sync_status then reports an error)
+# instead of touching memory out of bounds.  Load it with SALR_LIBRARY=<this path>.
+LIB_CHECKS = os.path.join(HERE, "libsalr_checks.so")
+
+
+def build(force: bool = False, verbose: bool = False, checks: bool = False) -> str:
+    out = LIB_CHECKS if checks else LIB
+    if force or stale(out):
+        cmd = command(out, ("-DSALR_CHECKS",) if checks else ())
         if verbose:
             print(" ".join(cmd))
         subprocess.run(cmd, check=True)
-    return LIB
+    return out
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
+    build(force="--force" in sys.argv, verbose=True, checks="--checks" in sys.argv)

@@ -325,7 +325,7 @@ cudaError_t launch_expand(const salr_weight_s* h, uint16_t* out, cudaStream_t st
   }
   const long long g = std::min<long long>(h->nblocks, 1ll * kExpandCtasPerSm * device_sms(h->device));
   expand_dense_kernel<<<static_cast<unsigned>(g < 1 ? 1 : g), 128, kExpandSmemBytes, st>>>(
-      h->blob, h->offsets, static_cast<int>(h->K), static_cast<int>(h->nblocks), out);
+      h->blob, h->offsets, static_cast<int>(h->K), static_cast<int>(h->nblocks), out, h->status);
   return cudaGetLastError();
 }
 
@@ -560,6 +560,27 @@ void bind_call(StreamParams& sp, float* acc, uint32_t* counters, float* tacc, ui
   sp.tflag = tflags;
 }
 
+// The bound on device-side waits, in SM cycles: kWaitLimitCycles (about 1 s), or
+// SALR_WAIT_LIMIT_CYCLES (failure tests make waits run out quickly with it).  Copied to
+// the device on the call's stream whenever it differs from the value last sent there.
+cudaError_t apply_wait_limit(cudaStream_t st) {
+  static std::atomic<long long> sent[64];  // 0: the module's initial value
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return e;
+  const char* v = getenv("SALR_WAIT_LIMIT_CYCLES");
+  long long want = v && v[0] >= '0' && v[0] <= '9' ? atoll(v) : kWaitLimitCycles;
+  if (want < 1000) want = 1000;
+  const long long have = sent[dev].load() == 0 ? kWaitLimitCycles : sent[dev].load();
+  if (want == have) return cudaSuccess;
+  static long long staged[64];  // stays valid while the copy is queued
+  staged[dev] = want;
+  e = cudaMemcpyToSymbolAsync(g_wait_limit, &staged[dev], sizeof(long long), 0,
+                              cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) sent[dev] = want;
+  return e;
+}
+
 // Compact blocks per bulk copy: as many as make about 40 KB (at most 4).  A bulk copy
 // occupies the SM's copy engine for about 540 cycles whatever its size (measured on B200
 // from L2: 2 to 32 KB per copy, 2 to 8 copies in flight, 1 or 148 CTAs), so copies of
@@ -604,6 +625,11 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   const int grid = static_cast<int>(units < sms ? units : sms);
   p.tshare = grid < p.kblocks ? grid : p.kblocks;
   p.treaders = stream_t_readers(units, grid, p.kblocks);
+  // SALR_FAIL_T_WAIT=1 (failure tests only): the readers of t wait for one part more
+  // than are ever added, so their bounded wait runs out and the call reports a timeout
+  const char* ft = getenv("SALR_FAIL_T_WAIT");
+  p.twant = p.tshare + (ft && ft[0] == '1' ? 1 : 0);
+  SALR_TRY(apply_wait_limit(st));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -782,7 +808,8 @@ int salr_encode(const void* W, int64_t N, int64_t K, float sparsity, void* strea
   encode_scan_kernel<<<1, 1024, 0, st>>>(size16, static_cast<int>(nblocks), cap16, h->offsets,
                                          h->status);
   encode_scatter_kernel<<<static_cast<unsigned>(nblocks), kBlockRows, 0, st>>>(
-      static_cast<const uint16_t*>(W), static_cast<int>(K), bits, h->offsets, cap16, h->blob);
+      static_cast<const uint16_t*>(W), static_cast<int>(K), bits, h->offsets, cap16, h->blob,
+      h->status);
   if ((e = cudaGetLastError()) != cudaSuccess) return fail(cuda_status(e));
 
   uint32_t total16 = 0;

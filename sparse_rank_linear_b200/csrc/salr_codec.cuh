@@ -182,7 +182,8 @@ __global__ void __launch_bounds__(1024) encode_scan_kernel(const uint32_t* __res
 // salr_decode.cuh).  Thread 0 writes the zero padding.
 __global__ void __launch_bounds__(kBlockRows) encode_scatter_kernel(
     const uint16_t* __restrict__ W, int K, const uint64_t* __restrict__ bits,
-    const uint32_t* __restrict__ offsets, unsigned long long cap16, uint8_t* __restrict__ blob) {
+    const uint32_t* __restrict__ offsets, unsigned long long cap16, uint8_t* __restrict__ blob,
+    int* status) {
   __shared__ uint64_t bm[kBlockRows];
   const int b = blockIdx.x, nwords = K / 64;
   if (offsets[b + 1] > cap16 || offsets[b] > offsets[b + 1]) return;
@@ -195,6 +196,9 @@ __global__ void __launch_bounds__(kBlockRows) encode_scatter_kernel(
   __syncthreads();
   const QuarterPos qp = quarter_pos(bm, warp, lane);
   uint16_t* vals = reinterpret_cast<uint16_t*>(base + kBitmapBytes);
+  const uint32_t cap_vals = ((offsets[b + 1] - offsets[b]) * 16 - kBitmapBytes) / 2;
+  (void)cap_vals;
+  (void)status;
   const uint4* src = reinterpret_cast<const uint4*>(W + static_cast<size_t>(i * kBlockRows + r) * K +
                                                     j * kBlockCols);
   uint32_t pos = qp.qb;
@@ -209,7 +213,11 @@ __global__ void __launch_bounds__(kBlockRows) encode_scatter_kernel(
       const uint32_t nib = static_cast<uint32_t>(word >> (4 * n)) & 15u;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        if ((nib >> c) & 1u) vals[at++] = static_cast<uint16_t>(w4[2 * h + (c >> 1)] >> (16 * (c & 1)));
+        if ((nib >> c) & 1u) {
+          if (SALR_CHECK(at < cap_vals, status))
+            vals[at] = static_cast<uint16_t>(w4[2 * h + (c >> 1)] >> (16 * (c & 1)));
+          ++at;
+        }
     }
   }
   if (r == 0) {

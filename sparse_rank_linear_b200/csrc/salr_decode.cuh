@@ -24,6 +24,7 @@
 #pragma once
 #include <cstdint>
 #include "salr_block.cuh"
+#include "sm100.cuh"
 
 namespace salr {
 
@@ -92,14 +93,26 @@ __device__ __forceinline__ uint32_t nib_pos(const QuarterPos& qp, int n, uint32_
 // 4n+2, 4n+3 (w1) as bf16 pairs, low half the lower column, for n = 0 .. 15.  The value
 // array must be readable 12 bytes past its last value (the windows of the last runs);
 // bytes read there only meet columns whose mask bit is clear.
+// status / vals_bytes: the status word and the bytes readable from vals (the block, its
+// padding and whatever the caller's buffer holds after it), for the checks of debug
+// builds: a window that would reach past vals_bytes is flagged and read from the start.
 template <class Sink>
 __device__ __forceinline__ void expand_quarter(const QuarterPos& qp, const uint8_t* vals,
-                                               const uint2* nt, Sink&& sink) {
+                                               const uint2* nt, Sink&& sink,
+                                               int* status = nullptr,
+                                               uint32_t vals_bytes = 0xFFFFFFFFu) {
   const uint32_t* v32 = reinterpret_cast<const uint32_t*>(vals);
   uint32_t base = qp.qb;
+  (void)status;
+  (void)vals_bytes;
 #pragma unroll
   for (int n = 0; n < 16; ++n) {
+#ifdef SALR_CHECKS
+    uint32_t p = nib_pos(qp, n, base);
+    if (!SALR_CHECK(((p >> 1) + 3) * 4 <= vals_bytes, status)) p = 0;
+#else
     const uint32_t p = nib_pos(qp, n, base);
+#endif
     const uint32_t nib = static_cast<uint32_t>(qp.word >> (4 * n)) & 15u;
     const uint32_t* w = v32 + (p >> 1);
     const uint32_t a0 = w[0], a1 = w[1], a2 = w[2];
@@ -116,17 +129,21 @@ __device__ __forceinline__ void expand_quarter(const QuarterPos& qp, const uint8
 // bank groups, so the stores are conflict-free.
 __device__ __forceinline__ void expand_quarter_to_tile(const QuarterPos& qp, const uint8_t* blk,
                                                        int q, int lane, const uint2* nt,
-                                                       uint8_t* tile) {
+                                                       uint8_t* tile, int* status = nullptr,
+                                                       uint32_t blk_bytes = 0xFFFFFFFFu) {
   const int row = 32 * q + lane;
   uint8_t* dst = tile + row * 128;
   uint32_t r[4];
-  expand_quarter(qp, blk + kBitmapBytes, nt, [&](int n, uint32_t w0, uint32_t w1) {
-    r[2 * (n & 1)] = w0;
-    r[2 * (n & 1) + 1] = w1;
-    if (n & 1)
-      *reinterpret_cast<uint4*>(dst + ((((n >> 1) ^ (row & 7))) << 4)) =
-          make_uint4(r[0], r[1], r[2], r[3]);
-  });
+  expand_quarter(
+      qp, blk + kBitmapBytes, nt,
+      [&](int n, uint32_t w0, uint32_t w1) {
+        r[2 * (n & 1)] = w0;
+        r[2 * (n & 1) + 1] = w1;
+        if (n & 1)
+          *reinterpret_cast<uint4*>(dst + ((((n >> 1) ^ (row & 7))) << 4)) =
+              make_uint4(r[0], r[1], r[2], r[3]);
+      },
+      status, blk_bytes - kBitmapBytes);
 }
 
 }  // namespace salr

@@ -528,7 +528,8 @@ __global__ void __launch_bounds__(kPreThreads, 1)
             ok = false;
             break;
           }
-          expand_quarter_to_tile(qp, cb, wg, lane, ntab, abuf(sa));
+          expand_quarter_to_tile(qp, cb, wg, lane, ntab, abuf(sa), p.status,
+                                 static_cast<uint32_t>(p.cbuf));
           fence_proxy_async_smem();
         } else {
           if (!mbar_wait(&ctrl->aempty[sa], ac.ph ^ 1)) {
@@ -582,7 +583,8 @@ constexpr int kExpandCtasPerSm = 4;
 __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __restrict__ blob,
                                                            const uint32_t* __restrict__ offsets,
                                                            int K, int nblocks,
-                                                           uint16_t* __restrict__ out) {
+                                                           uint16_t* __restrict__ out,
+                                                           int* status) {
   extern __shared__ uint4 exp_smem[];
   uint8_t* const cb0 = reinterpret_cast<uint8_t*>(exp_smem);  // two staging buffers
   auto cb = [&](int buf) { return cb0 + buf * kExpandBuf; };
@@ -592,7 +594,9 @@ __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __rest
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < 16) nt[threadIdx.x] = nibble_entry(threadIdx.x);
   auto stage = [&](int b, int buf) {
-    const uint32_t o0 = offsets[b], n16 = offsets[b + 1] - o0;
+    const uint32_t o0 = offsets[b];
+    uint32_t n16 = offsets[b + 1] - o0;
+    if (!SALR_CHECK(n16 * 16 + 32 <= static_cast<uint32_t>(kExpandBuf), status)) n16 = 0;
     const uint4* src = reinterpret_cast<const uint4*>(blob) + o0;
     for (uint32_t k = threadIdx.x; k < n16; k += 128)
       cp_async16(reinterpret_cast<uint4*>(cb(buf)) + k, src + k);
@@ -605,11 +609,13 @@ __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __rest
     if (bn < nblocks) stage(bn, buf ^ 1);
     cp_async_commit();
     cp_async_wait_one();  // this block's copies (the older group) have landed
-    const uint32_t n16 = offsets[b + 1] - offsets[b];
+    uint32_t n16 = offsets[b + 1] - offsets[b];
+    if (n16 * 16 + 32 > static_cast<uint32_t>(kExpandBuf)) n16 = 0;  // flagged when staged
     if (threadIdx.x < 2) reinterpret_cast<uint4*>(cb(buf))[n16 + threadIdx.x] = make_uint4(0, 0, 0, 0);
     __syncthreads();
     const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb(buf)), warp, lane);
-    expand_quarter_to_tile(qp, cb(buf), warp, lane, nt, tile);
+    // readable: the block and the two zeroed 16-byte chunks after it
+    expand_quarter_to_tile(qp, cb(buf), warp, lane, nt, tile, status, n16 * 16 + 32);
     __syncthreads();  // the tile is complete; this compact buffer is free for block b + 2 grid
     const int i = b / nwords, j = b % nwords;
     uint16_t* dst = out + static_cast<size_t>(i) * kBlockRows * K + j * kBlockCols;

@@ -69,6 +69,7 @@ struct StreamParams {
   int units;    // RT * kblocks
   int tshare;   // CTAs 0 .. tshare-1 compute a share of t (tshare = min(grid, kblocks))
   int treaders;  // CTAs that start a row tile (and read t): see stream_t_readers
+  int twant;     // t parts the readers wait for: tshare (more only in failure tests)
   int cbuf;     // bytes of a super-slot: bpc compact blocks + 32, multiple of 1024
   int bpc;      // compact blocks per bulk copy (1 .. 4)
   int bcbuf;    // bytes of the B_cat^T tile / t-share buffer (0 without adapter), x1024
@@ -134,7 +135,7 @@ __device__ __forceinline__ bool wait_global_flag(const uint32_t* flag, uint32_t 
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
     if (v == want) return true;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
+    if (clock64() - t0 > wait_limit()) return false;
     __nanosleep(64);
   }
 }
@@ -309,7 +310,11 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
         if (ts_next < nts && ts_next > 0 && mbar_test_wait(smem_u32(&ctrl->tsfree), (ts_next - 1) & 1))
           issue_ts(ts_next++);
         const int s = static_cast<int>(ps);
-        if (!mbar_wait(&ctrl->cempty[s], pph ^ 1) || stream_aborted(ctrl)) {
+        if (!SALR_CHECK(o_end >= o[0] && (o_end - o[0]) * 16u + 32u <= static_cast<uint32_t>(p.cbuf),
+                        p.status)) {
+          *reinterpret_cast<volatile int*>(&ctrl->abort) = 1;
+          fail = 1;
+        } else if (!mbar_wait(&ctrl->cempty[s], pph ^ 1) || stream_aborted(ctrl)) {
           stream_timeout(p, ctrl);
           fail = 1;
         } else {
@@ -480,7 +485,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
       for (int u = u0; u < u1; u = (u / KB + 1) * KB)
         if (u % KB == 0) has_adapter_seg = true;
       if (adapter && has_adapter_seg) {
-        if (lead) *gflag = wait_global_flag(p.tflag, static_cast<uint32_t>(p.tshare)) ? 1 : 0;
+        if (lead) *gflag = wait_global_flag(p.tflag, static_cast<uint32_t>(p.twant)) ? 1 : 0;
         named_bar(bar_id, 128);
         if (*gflag == 0) {
           if (lead) stream_timeout(p, ctrl);
@@ -570,6 +575,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
         if (*gflag != 2) break;
         tc_fence_after();
         const size_t n = static_cast<size_t>(i) * 128 + r;
+        if (!SALR_CHECK(n < static_cast<size_t>(p.N), p.status)) break;
         const bool whole = kba == 0 && kbb == KB;
         float* sum = p.acc + n * BNT;
 #pragma unroll
@@ -674,11 +680,15 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
         tc_fence_after();
         const uint32_t ts = tlane + 32u * sa;
         uint32_t r[8];
-        expand_quarter(qp, cb + kBitmapBytes, ntab, [&](int n, uint32_t w0, uint32_t w1) {
-          r[2 * (n & 3)] = w0;
-          r[2 * (n & 3) + 1] = w1;
-          if ((n & 3) == 3) tmem_st8(ts + 8 * (n >> 2), r[0], r[1], r[2], r[3], r[4], r[5], r[6], r[7]);
-        });
+        expand_quarter(
+            qp, cb + kBitmapBytes, ntab,
+            [&](int n, uint32_t w0, uint32_t w1) {
+              r[2 * (n & 3)] = w0;
+              r[2 * (n & 3) + 1] = w1;
+              if ((n & 3) == 3)
+                tmem_st8(ts + 8 * (n >> 2), r[0], r[1], r[2], r[3], r[4], r[5], r[6], r[7]);
+            },
+            p.status, static_cast<uint32_t>(p.cbuf) - ctrl->boff[sc][kc] - kBitmapBytes);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -733,6 +743,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
         }
         // ---- X tile of the block: row m (token) at m * 128, chunk c at (c ^ (m & 7)) * 16
         uint8_t* xb = xbuf(sa);
+        if (!SALR_CHECK(kbx >= 0 && kbx < KB && sa < static_cast<uint32_t>(SA), p.status)) kbx = 0;
 #pragma unroll
         for (int t0 = 0; t0 < kXChunks; t0 += 4) {  // 4 loads in flight per lane at a time
           uint4 v[4];

@@ -11,9 +11,25 @@ namespace salr {
 // Status bits a kernel may record in the handle's device status word.
 enum : int { DEV_ERR_NAN = 1, DEV_ERR_TIMEOUT = 2, DEV_ERR_RANGE = 4, DEV_ERR_FORMAT = 8 };
 
+// Debug builds (compiled with -DSALR_CHECKS) test the offsets the kernels derive from
+// data (decoder windows, copy sizes, output and partial-sum indices): a failed check
+// records DEV_ERR_RANGE in the status word and the access is skipped, never trapped.
+// Release builds compile the checks away.
+#ifdef SALR_CHECKS
+#define SALR_CHECK(cond, status) ((cond) ? true : (atomicOr((status), DEV_ERR_RANGE), false))
+#else
+#define SALR_CHECK(cond, status) true
+#endif
+
 // Upper bound on how long any single wait may spin, in SM clock cycles (~1 s at the
-// B200's 1.9 GHz boost clock).  A correct pipeline never comes near it.
+// B200's 1.9 GHz boost clock).  A correct pipeline never comes near it.  The bound in
+// force is g_wait_limit, read only once a wait did not succeed at once; the host may
+// lower it (failure tests make a wait run out quickly).
 constexpr long long kWaitLimitCycles = 2000000000LL;
+__device__ long long g_wait_limit = kWaitLimitCycles;
+__device__ __forceinline__ long long wait_limit() {
+  return *static_cast<volatile long long*>(&g_wait_limit);
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -71,10 +87,10 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
-  const long long t0 = clock64();
+  const long long t0 = clock64(), lim = wait_limit();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(a, parity)) return true;
-    if ((i & 255u) == 0 && clock64() - t0 > kWaitLimitCycles) return false;
+    if ((i & 255u) == 0 && clock64() - t0 > lim) return false;
   }
 }
 
