@@ -194,14 +194,14 @@ __global__ void __launch_bounds__(kBlockRows) encode_scatter_kernel(
   uint8_t* base = blob + static_cast<size_t>(offsets[b]) * 16;
   reinterpret_cast<uint64_t*>(base)[r] = word;
   __syncthreads();
-  const QuarterPos qp = quarter_pos(bm, warp, lane);
+  const QuarterRuns qr = quarter_runs(bm, warp, lane);
   uint16_t* vals = reinterpret_cast<uint16_t*>(base + kBitmapBytes);
   const uint32_t cap_vals = ((offsets[b + 1] - offsets[b]) * 16 - kBitmapBytes) / 2;
   (void)cap_vals;
   (void)status;
   const uint4* src = reinterpret_cast<const uint4*>(W + static_cast<size_t>(i * kBlockRows + r) * K +
                                                     j * kBlockCols);
-  uint32_t pos = qp.qb;
+  uint32_t pos = qr.first;
 #pragma unroll
   for (int c8 = 0; c8 < 8; ++c8) {  // 8 columns: two nibbles
     const uint4 q4 = src[c8];
@@ -209,7 +209,8 @@ __global__ void __launch_bounds__(kBlockRows) encode_scatter_kernel(
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int n = 2 * c8 + h;
-      uint32_t at = nib_pos(qp, n, pos);
+      uint32_t at = pos;
+      pos += nib_byte(qr.gap, n);
       const uint32_t nib = static_cast<uint32_t>(word >> (4 * n)) & 15u;
 #pragma unroll
       for (int c = 0; c < 4; ++c)

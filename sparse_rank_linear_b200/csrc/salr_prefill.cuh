@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kPreThreads, 1)
   // weight rows per unit: 128, or 256 (taken from the parameters in the wide kernel, which
   // as a run-time value keeps that kernel's registers within bounds)
   const int ROWS = WIDE ? 128 * (1 + (p.wide & 1)) : 128;
-  uint2* ntab = reinterpret_cast<uint2*>(tables);
+  uint2* ntab = reinterpret_cast<uint2*>(tables);  // 1 KB aligned
   PrefillCtrl* ctrl = reinterpret_cast<PrefillCtrl*>(tables + 128);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -522,14 +522,14 @@ __global__ void __launch_bounds__(kPreThreads, 1)
         }
         if (it < w.nk) {
           const uint8_t* cb = cbuf(sc);
-          const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb), wg, lane);
+          const QuarterRuns qr = quarter_runs(reinterpret_cast<const uint64_t*>(cb), wg, lane);
           if (!mbar_wait(&ctrl->aempty[sa], ac.ph ^ 1)) {
             pre_timeout(p.status, ctrl);
             ok = false;
             break;
           }
-          expand_quarter_to_tile(qp, cb, wg, lane, ntab, abuf(sa), p.status,
-                                 static_cast<uint32_t>(p.cbuf));
+          expand_runs_to_tile(qr, smem_u32(cb + kBitmapBytes), wg, lane, smem_u32(ntab), abuf(sa),
+                              p.status, static_cast<uint32_t>(p.cbuf) - kBitmapBytes);
           fence_proxy_async_smem();
         } else {
           if (!mbar_wait(&ctrl->aempty[sa], ac.ph ^ 1)) {
@@ -589,7 +589,8 @@ __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __rest
   uint8_t* const cb0 = reinterpret_cast<uint8_t*>(exp_smem);  // two staging buffers
   auto cb = [&](int buf) { return cb0 + buf * kExpandBuf; };
   uint8_t* tile = cb0 + 2 * kExpandBuf;
-  uint2* nt = reinterpret_cast<uint2*>(tile + kPreTileBytes);
+  uint2* nt = reinterpret_cast<uint2*>((reinterpret_cast<uintptr_t>(tile + kPreTileBytes) + 255) &
+                                       ~static_cast<uintptr_t>(255));  // 256-byte aligned
   const int nwords = K / 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < 16) nt[threadIdx.x] = nibble_entry(threadIdx.x);
@@ -613,9 +614,11 @@ __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __rest
     if (n16 * 16 + 32 > static_cast<uint32_t>(kExpandBuf)) n16 = 0;  // flagged when staged
     if (threadIdx.x < 2) reinterpret_cast<uint4*>(cb(buf))[n16 + threadIdx.x] = make_uint4(0, 0, 0, 0);
     __syncthreads();
-    const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb(buf)), warp, lane);
+    const QuarterRuns qr = quarter_runs(reinterpret_cast<const uint64_t*>(cb(buf)), warp, lane);
     // readable: the block and the two zeroed 16-byte chunks after it
-    expand_quarter_to_tile(qp, cb(buf), warp, lane, nt, tile, status, n16 * 16 + 32);
+    const uint32_t readable = n16 * 16 + 32;
+    expand_runs_to_tile(qr, smem_u32(cb(buf) + kBitmapBytes), warp, lane, smem_u32(nt), tile, status,
+                        readable > kBitmapBytes ? readable - kBitmapBytes : 0u);
     __syncthreads();  // the tile is complete; this compact buffer is free for block b + 2 grid
     const int i = b / nwords, j = b % nwords;
     uint16_t* dst = out + static_cast<size_t>(i) * kBlockRows * K + j * kBlockCols;
@@ -627,7 +630,7 @@ __global__ void __launch_bounds__(128) expand_dense_kernel(const uint8_t* __rest
     __syncthreads();  // the tile is free for the next block
   }
 }
-constexpr int kExpandSmemBytes = 2 * kExpandBuf + kPreTileBytes + 128;
+constexpr int kExpandSmemBytes = 2 * kExpandBuf + kPreTileBytes + 256 + 128;  // table aligned up
 
 // ------------------------------------------------------------------------------------
 // t = X A_cat for all tokens, rounded once to bf16 into T [M x 128] (ranks past R16 are

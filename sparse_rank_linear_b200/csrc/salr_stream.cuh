@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
   uint8_t* tbuf = smem + L::fixed_off(p.cbuf, SA, SC);
   uint8_t* bcbuf = tbuf + L::kTbuf;  // B_cat^T tile; at kernel start, the t-share stage
   StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(bcbuf + p.bcbuf);
-  uint2* ntab = reinterpret_cast<uint2*>(bcbuf + p.bcbuf + kStreamCtrlBytes);  // 16 x 8 B
+  uint2* ntab = reinterpret_cast<uint2*>(bcbuf + p.bcbuf + kStreamCtrlBytes);  // 16 x 8 B, 1 KB aligned
 
   griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -654,6 +654,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
     // flip) exactly when it crosses a multiple of the ring size
     if (dw < NDEC) {
       const int g = dw >> 2, q = warp & 3;
+      const uint32_t tab_sa = smem_u32(ntab);
       const uint32_t tlane = tmem_a + (static_cast<uint32_t>(32 * q) << 16);
       // block it lives in copy it / bpc (super-slot sc, phase phc) at block kc of it
       const int bpc = p.bpc;
@@ -671,7 +672,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
           break;
         }
         const uint8_t* cb = cbuf(sc) + ctrl->boff[sc][kc];
-        const QuarterPos qp = quarter_pos(reinterpret_cast<const uint64_t*>(cb), q, lane);
+        const QuarterRuns qr = quarter_runs(reinterpret_cast<const uint64_t*>(cb), q, lane);
         // ---- the TMEM slot must be free: the MMAs of its previous block have completed
         if (!mbar_wait(&ctrl->aempty[sa], pha ^ 1)) {
           stream_timeout(p, ctrl);
@@ -680,8 +681,8 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
         tc_fence_after();
         const uint32_t ts = tlane + 32u * sa;
         uint32_t r[8];
-        expand_quarter(
-            qp, cb + kBitmapBytes, ntab,
+        expand_runs(
+            qr, smem_u32(cb + kBitmapBytes), tab_sa,
             [&](int n, uint32_t w0, uint32_t w1) {
               r[2 * (n & 3)] = w0;
               r[2 * (n & 3) + 1] = w1;
