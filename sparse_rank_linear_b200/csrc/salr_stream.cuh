@@ -60,7 +60,7 @@ struct StreamParams {
   uint16_t* Y;
   float* acc;            // [RT x 128 x BNT] fp32 sums of split row tiles, zero between calls
   uint32_t* counters;    // [RT x 4] segments arrived per split tile and 32-row quarter, zero between calls
-  float* tacc;           // [BNT x R16] fp32 accumulator of t = X A_cat, zero between calls
+  float* tacc;           // [R16 x BNT] fp32 accumulator of t = X A_cat (rank-major), zero between calls
   uint32_t* tflag;       // [2]: t parts arrived, CTAs done reading t; zero between calls
   int* status;
   int N, K, M, R, R16;
@@ -202,31 +202,51 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
     offx = (u0 + 32 <= p.units) ? __ldg(p.offsets + u0 + 32) : 0u;
   }
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < SC; ++s) {
-      mbar_init(&ctrl->cfull[s], 1);
-      mbar_init(&ctrl->cempty[s], p.bpc * (NDEC / kStreamGroups));  // every warp of its blocks
+  {
+    // one barrier per thread (a thread initialising them all in turn took microseconds)
+    constexpr int WPG = NDEC / kStreamGroups;
+    int i = threadIdx.x;
+    uint64_t* b = nullptr;
+    uint32_t cnt = 1;
+    if (i < SC) {
+      b = &ctrl->cfull[i];
+    } else if ((i -= SC) < SC) {
+      b = &ctrl->cempty[i];
+      cnt = p.bpc * WPG;  // every warp of its blocks
+    } else if ((i -= SC) < SA) {
+      b = &ctrl->dec[i];
+      cnt = WPG;
+    } else if ((i -= SA) < SA) {
+      b = &ctrl->aempty[i];
+    } else if ((i -= SA) < 2 * kStreamGroups) {
+      b = &ctrl->gdone[i >> 1][i & 1];
+    } else if ((i -= 2 * kStreamGroups) < kStreamGroups) {
+      b = &ctrl->gfin[i];
+    } else if ((i -= kStreamGroups) < 2) {
+      b = &ctrl->adone[i];
+    } else if ((i -= 2) < 2) {
+      b = &ctrl->accempty[i];
+      cnt = 4;
+    } else {
+      switch (i - 2) {
+        case 0: b = &ctrl->bcfull; break;
+        case 1: b = &ctrl->bcempty; break;
+        case 2: b = &ctrl->tready; cnt = 4; break;
+        case 3: b = &ctrl->tsfull; break;
+        case 4: b = &ctrl->tsfree; break;
+        case 5: b = &ctrl->tsdone; break;
+        case 6: b = &ctrl->fin; break;
+        default: break;
+      }
     }
-    for (int s = 0; s < SA; ++s) {
-      mbar_init(&ctrl->dec[s], NDEC / kStreamGroups);
-      mbar_init(&ctrl->aempty[s], 1);
+    if (b) {
+      mbar_init(b, cnt);
+      fence_mbar_init();
     }
-    for (int x = 0; x < 2; ++x) {
-      for (int g = 0; g < kStreamGroups; ++g) mbar_init(&ctrl->gdone[g][x], 1);
-      mbar_init(&ctrl->adone[x], 1);
-      mbar_init(&ctrl->accempty[x], 4);
+    if (threadIdx.x == 0) {
+      ctrl->abort = 0;
+      ctrl->flag[0] = ctrl->flag[1] = 0;
     }
-    for (int g = 0; g < kStreamGroups; ++g) mbar_init(&ctrl->gfin[g], 1);
-    mbar_init(&ctrl->bcfull, 1);
-    mbar_init(&ctrl->bcempty, 1);
-    mbar_init(&ctrl->tready, 4);
-    mbar_init(&ctrl->tsfull, 1);
-    mbar_init(&ctrl->tsfree, 1);
-    mbar_init(&ctrl->tsdone, 1);
-    mbar_init(&ctrl->fin, 1);
-    ctrl->abort = 0;
-    ctrl->flag[0] = ctrl->flag[1] = 0;
-    fence_mbar_init();
   }
   if (threadIdx.x < 16) ntab[threadIdx.x] = nibble_entry(threadIdx.x);
   if (warp == 1) tmem_alloc(&ctrl->tmem, kCols);
@@ -423,7 +443,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
       }
       if (!ok) stream_timeout(p, ctrl);
       mma_commit(&ctrl->fin);
-      if (!mbar_wait(&ctrl->fin, 0)) stream_timeout(p, ctrl);
+      if (!mbar_wait_idle(&ctrl->fin, 0, 200)) stream_timeout(p, ctrl);
     }
   } else if (warp < kStreamFixedWarps) {
     // ================================================================ epilogue
@@ -436,6 +456,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
     const int q = warp & 3;                       // TMEM lane quarter
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     const int r = 32 * q + lane;  // weight row within the tile; rank index for t
+    bool t_read = false;          // this CTA has read t (it is one of t's readers)
     __nv_bfloat16* Y = reinterpret_cast<__nv_bfloat16*>(p.Y);
     volatile int* gflag = &ctrl->flag[eg];
     // ---- 0. both accumulators start at zero (every MMA into them accumulates); their
@@ -465,10 +486,13 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
             uint32_t v[16];
             tmem_ld16(tmem_ts + lane_base + c, v);
             tmem_ld_wait();
-            if (r < p.R) {
+            if (r < p.R) {  // t is kept rank-major, [R16 x BNT]
 #pragma unroll
-              for (int e = 0; e < 16; ++e)
-                if (c + e < p.M) atomicAdd(&p.tacc[(c + e) * p.R16 + r], __uint_as_float(v[e]));
+              for (int e = 0; e < 16; e += 4)
+                if (c + e < p.M)
+                  red_add_v4f32(p.tacc + r * BNT + c + e, __uint_as_float(v[e]),
+                                __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                                __uint_as_float(v[e + 3]));
             }
           }
         }
@@ -490,54 +514,38 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
         if (*gflag == 0) {
           if (lead) stream_timeout(p, ctrl);
         } else {
-          // 8 entries per thread per L2 round trip: a batch's loads go out before its
-          // shared-memory stores
-          for (int e0 = r; e0 < BNT * p.R16; e0 += 128 * 8) {
-            float v[8];
+          // four tokens of one rank per 16-byte load, 4 loads per thread per L2 round
+          // trip: a batch's loads go out before its shared-memory stores
+          constexpr int kPerRank = BNT / 4;
+          for (int f0 = r; f0 < kPerRank * p.R16; f0 += 128 * 4) {
+            float4 v[4];
 #pragma unroll
-            for (int g = 0; g < 8; ++g) {
-              const int e = e0 + 128 * g;
-              const int m = e / p.R16, j = e % p.R16;
-              v[g] = (e < BNT * p.R16 && m < p.M && j < p.R) ? __ldcg(&p.tacc[m * p.R16 + j])
-                                                            : 0.0f;
+            for (int g = 0; g < 4; ++g) {
+              const int f = f0 + 128 * g, j = f / kPerRank, m = 4 * (f % kPerRank);
+              v[g] = (f < kPerRank * p.R16 && m < p.M && j < p.R)
+                         ? __ldcg(reinterpret_cast<const float4*>(p.tacc + j * BNT + m))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int g = 0; g < 8; ++g) {
-              const int e = e0 + 128 * g;
-              if (e >= BNT * p.R16) continue;
-              const int m = e / p.R16, j = e % p.R16;
+            for (int g = 0; g < 4; ++g) {
+              const int f = f0 + 128 * g, j = f / kPerRank, m0 = 4 * (f % kPerRank);
+              if (f >= kPerRank * p.R16) continue;
               const int chunk = j >> 6, cc = j & 63;
-              uint8_t* dst = tbuf + chunk * (BNT * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
-                             (((cc >> 3) ^ (m & 7)) << 4) + (cc & 7) * 2;
-              *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v[g]);
+              const float tv[4] = {v[g].x, v[g].y, v[g].z, v[g].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int m = m0 + e;
+                uint8_t* dst = tbuf + chunk * (BNT * 128) + (m >> 3) * 1024 + (m & 7) * 128 +
+                               (((cc >> 3) ^ (m & 7)) << 4) + (cc & 7) * 2;
+                *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(tv[e]);
+              }
             }
           }
           fence_proxy_async_smem();
         }
-        const bool tok = *gflag != 0;
+        t_read = *gflag != 0;
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->tready);
-        if (tok) {
-          // ---- count this CTA out of t's readers; the last one clears t and both counts
-          //      (every reader's loads of t are complete before its count: the values
-          //      are already in shared memory)
-          __threadfence();
-          named_bar(bar_id, 128);
-          if (lead) {
-            const uint32_t done = atomicAdd(p.tflag + 1, 1u) + 1u;
-            *gflag = done == static_cast<uint32_t>(p.treaders) ? 3 : 1;
-          }
-          named_bar(bar_id, 128);
-          if (*gflag == 3) {
-            __threadfence();
-            float4* z = reinterpret_cast<float4*>(p.tacc);
-            for (int e = r; e < p.M * p.R16 / 4; e += 128) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (lead) {
-              p.tflag[0] = 0u;
-              p.tflag[1] = 0u;
-            }
-          }
-        }
       }
     }
     // ---- 3. the CTA's segments in order: wait until every decoder group with blocks in
@@ -559,12 +567,12 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
           const int gg = (itA + g) % kStreamGroups;  // groups of blocks itA, itA + 1, ...
           if (g < nb) {
             const uint32_t bit = 1u << (2 * gg + x);
-            okw = okw && mbar_wait(&ctrl->gdone[gg][x], (gph & bit) ? 1u : 0u);
+            okw = okw && mbar_wait_idle(&ctrl->gdone[gg][x], (gph & bit) ? 1u : 0u, 64);
             gph ^= bit;
           }
         }
         if (adapter && kba == 0) {
-          okw = okw && mbar_wait(&ctrl->adone[x], (aph >> x) & 1u);
+          okw = okw && mbar_wait_idle(&ctrl->adone[x], (aph >> x) & 1u, 64);
           aph ^= 1u << x;
         }
         if (!okw) stream_timeout(p, ctrl);
@@ -640,6 +648,25 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
       }
       u = i * KB + kbb;
     }
+    // ---- 4. count this CTA out of t's readers; the last one clears t and both counts.
+    //      Every warp's loads of t completed before its tready arrival, which the adapter
+    //      MMAs and so the drain of the adapter segment above waited for.
+    if (t_read && warp == 2 + 4 * eg) {
+      uint32_t last = 0;
+      if (lane == 0) {
+        __threadfence();
+        last = atomicAdd(p.tflag + 1, 1u) + 1u == static_cast<uint32_t>(p.treaders);
+      }
+      if (__shfl_sync(0xffffffffu, last, 0)) {
+        __threadfence();
+        float4* z = reinterpret_cast<float4*>(p.tacc);
+        for (int e = lane; e < BNT * p.R16 / 4; e += 32) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane == 0) {
+          p.tflag[0] = 0u;
+          p.tflag[1] = 0u;
+        }
+      }
+    }
   } else {
     // ================================================================ decoders
     // NDEC warps in kStreamGroups groups of four consecutive warps; group g decodes blocks
@@ -665,7 +692,9 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
           sc = 0;
           phc ^= 1u;
         }
-      griddep_wait();
+      // no wait for the preceding kernel here: the decoders read only the compact blocks
+      // (which no kernel that lets this one start early writes) and this CTA's TMEM, so
+      // the first blocks are rebuilt while that kernel finishes
       for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
         if (!mbar_wait(&ctrl->cfull[sc], phc)) {
           stream_timeout(p, ctrl);
@@ -768,7 +797,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
             ok = mbar_wait(&ctrl->accempty[x], (seg >> 1) & 1);
             seg_waited = seg;
           }
-          ok = ok && mbar_wait(&ctrl->dec[sa], pha);
+          ok = ok && mbar_wait_idle(&ctrl->dec[sa], pha, 100);
           if (!ok) {
             stream_timeout(p, ctrl);
           } else {

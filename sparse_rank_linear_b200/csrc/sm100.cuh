@@ -94,6 +94,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// The same for a wait expected to last long (a whole segment, the rest of the kernel):
+// between tests the thread sleeps about `ns` nanoseconds, leaving its issue slots to the
+// warps that do the work.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const long long t0 = clock64(), lim = wait_limit();
+  for (;;) {
+    __nanosleep(ns);
+    if (mbar_try_wait(a, parity)) return true;
+    if (clock64() - t0 > lim) return false;
+  }
+}
+
 // Programmatic dependent launch.  launch_dependents lets the next kernel of the stream
 // (launched with programmatic stream serialization) start its CTAs as this grid's CTAs
 // exit; wait blocks until every preceding grid has completed and its memory operations
