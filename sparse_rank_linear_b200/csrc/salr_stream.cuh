@@ -158,11 +158,20 @@ __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
 }
 
 
+// a * b / c rounded down, a * b < 2^32 when fits32 (32-bit division is several times
+// cheaper than the 64-bit routine; the even split of U units over G CTAs fits whenever
+// U * G < 2^32, about 29 M blocks on 148 SMs)
+__device__ __forceinline__ int mul_div(long long a, long long b, long long c, bool fits32) {
+  return fits32 ? static_cast<int>(static_cast<uint32_t>(a) * static_cast<uint32_t>(b) /
+                                   static_cast<uint32_t>(c))
+                : static_cast<int>((a * b) / c);
+}
+
 // CTA that owns unit u (block u in storage order) under the even split of U units.
-__device__ __forceinline__ int owner_of(long long u, long long U, int G) {
-  int c = static_cast<int>((u * G) / U);
-  while (c + 1 < G && ((c + 1) * U) / G <= u) ++c;
-  while (c > 0 && (c * U) / G > u) --c;
+__device__ __forceinline__ int owner_of(long long u, long long U, int G, bool fits32) {
+  int c = mul_div(u, G, U, fits32);
+  while (c + 1 < G && mul_div(c + 1, U, G, fits32) <= u) ++c;
+  while (c > 0 && mul_div(c, U, G, fits32) > u) --c;
   return c;
 }
 
@@ -189,8 +198,9 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
   const bool adapter = p.R > 0;
   const int G = gridDim.x, cta = blockIdx.x;
   const long long U = p.units;
-  const int u0 = static_cast<int>((static_cast<long long>(cta) * U) / G);
-  const int u1 = static_cast<int>((static_cast<long long>(cta + 1) * U) / G);
+  const bool fits32 = U * G < (1ll << 32);
+  const int u0 = mul_div(cta, U, G, fits32);
+  const int u1 = mul_div(cta + 1, U, G, fits32);
   const int KB = p.kblocks;
   // t share of this CTA: K blocks cta, cta + tshare, ... (only CTAs below tshare)
   const int nts = (adapter && cta < p.tshare) ? (KB - cta + p.tshare - 1) / p.tshare : 0;
@@ -202,10 +212,11 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
     offx = (u0 + 32 <= p.units) ? __ldg(p.offsets + u0 + 32) : 0u;
   }
 
-  {
-    // one barrier per thread (a thread initialising them all in turn took microseconds)
+  if (warp >= 2 && warp < kStreamFixedWarps) {
+    // one barrier per thread of the epilogue warps: the init fence waits for the thread's
+    // earlier memory operations, so it is kept away from the producer's offset loads
     constexpr int WPG = NDEC / kStreamGroups;
-    int i = threadIdx.x;
+    int i = threadIdx.x - 64;
     uint64_t* b = nullptr;
     uint32_t cnt = 1;
     if (i < SC) {
@@ -243,7 +254,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
       mbar_init(b, cnt);
       fence_mbar_init();
     }
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 64) {
       ctrl->abort = 0;
       ctrl->flag[0] = ctrl->flag[1] = 0;
     }
@@ -614,9 +625,9 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
           __syncwarp();
           uint32_t last = 0;
           if (lane == 0) {
-            const int c_first = owner_of(static_cast<long long>(i) * KB, U, G);
+            const int c_first = owner_of(static_cast<long long>(i) * KB, U, G, fits32);
             const int segs =
-                owner_of(static_cast<long long>(i) * KB + KB - 1, U, G) - c_first + 1;
+                owner_of(static_cast<long long>(i) * KB + KB - 1, U, G, fits32) - c_first + 1;
             last = atomicAdd(p.counters + 4 * i + q, 1u) == static_cast<uint32_t>(segs - 1);
           }
           if (__shfl_sync(0xffffffffu, last, 0)) {
@@ -696,7 +707,9 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
       // (which no kernel that lets this one start early writes) and this CTA's TMEM, so
       // the first blocks are rebuilt while that kernel finishes
       for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
-        if (!mbar_wait(&ctrl->cfull[sc], phc)) {
+        // (the first wait lasts until the first copies land: sleeping leaves the issue
+        // slots to the producer meanwhile)
+        if (!(it == g ? mbar_wait_idle(&ctrl->cfull[sc], phc, 32) : mbar_wait(&ctrl->cfull[sc], phc))) {
           stream_timeout(p, ctrl);
           break;
         }
