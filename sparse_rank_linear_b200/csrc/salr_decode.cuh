@@ -61,6 +61,12 @@ __device__ __forceinline__ uint32_t nib_byte(const uint32_t (&e)[4], int n) {
   return __byte_perm(e[(n & 1) + 2 * (n >> 3)], 0u, 0x4440u | ((n >> 1) & 3));
 }
 
+__device__ __forceinline__ uint32_t mad_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // Runs of lane `lane`'s row 32q + lane.  bm: the block's 128 bitmap words.  Called by all
 // 32 lanes of a warp.
 __device__ __forceinline__ QuarterRuns quarter_runs(const uint64_t* bm, int q, int lane) {
@@ -76,12 +82,21 @@ __device__ __forceinline__ QuarterRuns quarter_runs(const uint64_t* bm, int q, i
   const uint32_t lo = static_cast<uint32_t>(x), hi = static_cast<uint32_t>(x >> 32);
   const uint32_t e[4] = {lo & 0x0F0F0F0Fu, (lo >> 4) & 0x0F0F0F0Fu, hi & 0x0F0F0F0Fu,
                          (hi >> 4) & 0x0F0F0F0Fu};
+  // four inclusive warp scans side by side; each step adds the value from `o` lanes down
+  // as a multiply-add by a 0/1 lane mask (on the FMA pipe: the integer pipe is the
+  // decoder's bottleneck)
+  uint32_t s[4] = {e[0], e[1], e[2], e[3]};
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t m = lane >= o ? 1u : 0u;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s[k] = mad_u32(__shfl_up_sync(0xffffffffu, s[k], o), m, s[k]);
+  }
   uint32_t ex[4], rest[4];  // per nibble: values in earlier rows / in this and later rows
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const uint32_t s = warp_incl_scan(e[k]);
-    ex[k] = s - e[k];
-    rest[k] = __shfl_sync(0xffffffffu, s, 31) - ex[k];  // no borrow: the total >= ex, bytewise
+    ex[k] = s[k] - e[k];
+    rest[k] = __shfl_sync(0xffffffffu, s[k], 31) - ex[k];  // no borrow: the total >= ex, bytewise
   }
   // gap(n) = rest(n) + ex(n + 1) <= 4 (32 - lane) + 4 lane: no carry between bytes.  The
   // next nibble of an even one is the same byte of the next word; of an odd one, the next

@@ -707,16 +707,16 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
       // (which no kernel that lets this one start early writes) and this CTA's TMEM, so
       // the first blocks are rebuilt while that kernel finishes
       for (int it = g; it < nunits && !stream_aborted(ctrl); it += kStreamGroups) {
-        // (the first wait lasts until the first copies land: sleeping leaves the issue
-        // slots to the producer meanwhile)
-        if (!(it == g ? mbar_wait_idle(&ctrl->cfull[sc], phc, 32) : mbar_wait(&ctrl->cfull[sc], phc))) {
+        // (waiting warps sleep between tests, leaving the issue slots to the warps at work;
+        // the first wait lasts until the first copies land)
+        if (!mbar_wait_idle(&ctrl->cfull[sc], phc, it == g ? 32 : 20)) {
           stream_timeout(p, ctrl);
           break;
         }
         const uint8_t* cb = cbuf(sc) + ctrl->boff[sc][kc];
         const QuarterRuns qr = quarter_runs(reinterpret_cast<const uint64_t*>(cb), q, lane);
         // ---- the TMEM slot must be free: the MMAs of its previous block have completed
-        if (!mbar_wait(&ctrl->aempty[sa], pha ^ 1)) {
+        if (!mbar_wait_idle(&ctrl->aempty[sa], pha ^ 1, 20)) {
           stream_timeout(p, ctrl);
           break;
         }
@@ -779,7 +779,7 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
         }
         const int x = seg & 1;
         int ok = 1;
-        if (lane == 0) ok = mbar_wait(&ctrl->aempty[sa], pha ^ 1) && !stream_aborted(ctrl);
+        if (lane == 0) ok = mbar_wait_idle(&ctrl->aempty[sa], pha ^ 1, 20) && !stream_aborted(ctrl);
         if (!__shfl_sync(0xffffffffu, ok, 0)) {
           if (lane == 0) stream_timeout(p, ctrl);
           break;
