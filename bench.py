@@ -534,9 +534,10 @@ def roofline_of(wl, M, keep, kern_ms, region_ms, peaks, peak_src, traffic_key, p
                                f" ({'timed region of %.0f ms, under the power cap' % region_ms if long_region else 'short timed region: burst'})")
         roof["frac_of_burst_peak"] = achieved / peaks["bf16_tflops"]
     if M <= 64:
-        kname = f"salr_stream_kernel<{16 if M <= 16 else 32 if M <= 32 else 64},16>"
+        kname = f"salr_stream_kernel<{16 if M <= 16 else 32 if M <= 32 else 64},20>"
     else:
-        kname = f"salr_prefill_kernel<{128 if M <= 128 else 256}>"
+        wide = int(plan.get("tile_rows", 128) == 256)
+        kname = f"salr_prefill_kernel<{128 if M <= 128 else 256},{wide}>"
     roof["traffic"] = traffic_for(kname, traffic_key)
     roof["kernel"] = kname
     roof["kernels_per_call"] = plan["kernels"]
