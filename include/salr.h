@@ -29,6 +29,20 @@
  *   - The library never traps or spins without a bound on the GPU.  Errors found on the
  *     device (a NaN in W, a pipeline wait that ran out of time) are recorded in the
  *     handle's status word; salr_encode reports them itself, salr_sync_status reads them.
+ *   - Bounds-checked build: compiled with -DSALR_CHECKS (python -m
+ *     sparse_rank_linear_b200.build --checks gives libsalr_checks.so, which the Python
+ *     binding loads when SALR_LIBRARY names it), every shared- or global-memory offset
+ *     the kernels derive from the data (block offsets and sizes, value positions, tile
+ *     rows, ring indices) is checked before use; a failed check skips the access and
+ *     sets a range bit that salr_sync_status reports as SALR_ERR_INVALID.
+ *   - Environment, read at each call: SALR_WAIT_LIMIT_CYCLES=n bounds every device wait
+ *     at n SM cycles (default 2e9, about one second; failure tests lower it);
+ *     SALR_FAIL_T_WAIT=1 makes the small-M kernel's readers of t wait for one part more
+ *     than is ever added (failure tests only: the call then reports SALR_ERR_TIMEOUT);
+ *     SALR_WIDE_MIN_ROUNDS=n sets how many full rounds of 256-row tiles the dense-scratch
+ *     path needs before it uses them (default 8; tests set 0 to reach them on small
+ *     shapes); SALR_COOPERATIVE=1 launches the small-M kernel cooperatively instead of
+ *     with programmatic stream serialization; SALR_FAKE_OOM=1 makes allocations fail.
  *
  * Shape rules (v1): N % 128 == 0, 128 <= N <= 2^22, K % 64 == 0, 64 <= K <= 32768,
  * R % 8 == 0, R <= 128, 1 <= M <= 2^24, at most 2^27 output tiles of 128 x 128
@@ -157,19 +171,18 @@ SALR_API int salr_linear_host(const void* X_host, int64_t M, salr_handle h, cons
  * No counterpart in the SALR paper: this is an interface variant of this library, not
  * part of the method.  It computes the same layer as salr_linear (same arguments, same
  * arithmetic and tolerance) for M <= 16 and N <= 32768, and never allocates device
- * memory: the scratch it needs (fp32 partial sums and their arrival counts, the two
- * fp32 t = X A_cat accumulators and their counts, about 2 MiB) is one fixed array in the
+ * memory: the scratch it needs (fp32 partial sums and their arrival counts, the fp32
+ * t = X A_cat accumulator and its counts, about 2 MiB) is one fixed array in the
  * library's device code, present on every GPU that loads the library until the process
  * exits.  Meant for
  * callers whose device memory is planned up front and who may not allocate during
  * inference (a failing or stalling cudaMalloc is not acceptable there).  The handle and
  * all inputs and outputs are still the caller's.
  *
- * Returns SALR_ERR_UNSUPPORTED for M > 16 or N > 32768 (or a GPU with more than 160
- * SMs).  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress), clears the array on `stream` and should come before any
- * stream capture.  Each call then leaves the array ready for the next one; after a call
- * that gave up (salr_sync_status reports it) the array is cleared again.  All calls
+ * Returns SALR_ERR_UNSUPPORTED for M > 16 or N > 32768.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) and clears the array on
+ * `stream`.  Each call then leaves the array ready for the next one; after a call that
+ * gave up (salr_sync_status reports it) the array is cleared again.  All calls
  * on one device share the one array, so calls whose executions overlap on the GPU
  * (different streams, or different threads) race and give wrong results: order them on
  * one stream.

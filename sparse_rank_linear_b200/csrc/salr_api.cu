@@ -1422,7 +1422,8 @@ int salr_sync_status(salr_handle h, void* stream) {
   const int nrc = noalloc_reset(h->device);
   if (nrc != SALR_OK) return nrc;
   if (status & DEV_ERR_TIMEOUT) return SALR_ERR_TIMEOUT;
-  if (status & DEV_ERR_NAN) return SALR_ERR_INVALID;
+  // a NaN, or (in the bounds-checked build) an offset or size out of range
+  if (status & (DEV_ERR_NAN | DEV_ERR_RANGE | DEV_ERR_FORMAT)) return SALR_ERR_INVALID;
   return SALR_ERR_UNSUPPORTED;
 }
 

@@ -88,3 +88,31 @@ def test_noalloc_without_adapter_and_limits(lib):
     Y17 = torch.empty(17, 384, dtype=torch.bfloat16, device="cuda")
     assert call_noalloc(lib, X17, h, None, None, Y17) == 2
     h.free()
+
+
+def test_noalloc_recovers_after_a_wait_runs_out(lib, monkeypatch):
+    # the readers of t wait for one part more than is ever added, under a short bound:
+    # the call gives up and reports SALR_ERR_TIMEOUT; salr_sync_status clears the fixed
+    # array, and the next calls match the oracle again
+    wl = synth.WORKLOADS["q_proj"]
+    w, x, ad = synth.weight(wl), synth.activations(wl, 16), synth.adapters(wl)
+    h = salr.encode(to_dev(w), 0.5)
+    A = to_dev(np.concatenate([a for a, _ in ad], axis=1))
+    B = to_dev(np.concatenate([b for _, b in ad], axis=0))
+    X = to_dev(x)
+    Y = torch.empty(16, wl.N, dtype=torch.bfloat16, device="cuda")
+    monkeypatch.setenv("SALR_WAIT_LIMIT_CYCLES", "400000")
+    monkeypatch.setenv("SALR_FAIL_T_WAIT", "1")
+    assert call_noalloc(lib, X, h, A, B, Y) == 0
+    assert h.sync_status() == 5  # SALR_ERR_TIMEOUT
+    monkeypatch.delenv("SALR_FAIL_T_WAIT")
+    monkeypatch.delenv("SALR_WAIT_LIMIT_CYCLES")
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    ref, s = oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad)
+    for call in range(2):
+        Y = torch.full((16, wl.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        assert call_noalloc(lib, X, h, A, B, Y) == 0
+        assert h.sync_status() == 0
+        ok, rel, worst = oracle.check_tolerance(to_bits(Y), ref, s)
+        assert ok, f"call {call} after the timeout: rel_fro={rel:.2e} worst={worst:.2e}"
+    h.free()
