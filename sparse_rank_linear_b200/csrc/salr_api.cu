@@ -522,6 +522,25 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   return SALR_OK;
 }
 
+// Order of the prefill kernel's output tiles.  Taken token tile first, the tiles in flight
+// sweep all of X every few row tiles: harmless while X stays in L2, but with X larger than
+// about half of it each sweep goes back to DRAM (large M = 8192: about 6 GB of reads per
+// call for 0.6 GB of operands).  Taken in groups of g row tiles, token tile by token
+// tile, the `grid` tiles in flight touch g weight row tiles and about grid / g X tiles,
+// and a group reads X once; g = sqrt(grid * X tile / weight tile) makes the tiles in
+// flight the fewest bytes.  0 keeps the plain order.
+int tile_group_rows(int rtiles, int TT, int rows, int bnt, int64_t K, int grid) {
+  const char* v = getenv("SALR_TILE_GROUP_ROWS");  // tests: a group size on small shapes
+  if (v && v[0] >= '0' && v[0] <= '9') {
+    const int g = atoi(v);
+    return g > rtiles ? rtiles : g;
+  }
+  const double wtile = 2.0 * rows * K, xtile = 2.0 * bnt * K;
+  if (TT * xtile <= 48.0 * (1 << 20) || TT < 2) return 0;
+  int g = static_cast<int>(std::lround(std::sqrt(grid * xtile / wtile)));
+  return g < 1 ? 1 : g > rtiles ? rtiles : g;
+}
+
 // Persistent small-M path: one CTA per SM, launched so that it may overlap the preceding
 // kernel of the stream.
 constexpr int kStreamDecoders = 4 * kStreamGroups;  // one warp per row quarter in each group
@@ -959,6 +978,8 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   uint8_t* wdense = nullptr;
   pp.dense = pl.path == 2 ? 1 : 0;
   pp.wide = pl.rows == 256 ? 1 : 0;
+  pp.rtiles = static_cast<int>(h->N / pl.rows);
+  pp.group_rows = tile_group_rows(pp.rtiles, TT, pl.rows, bnt, h->K, grid);
   if (pp.dense) {
     const cudaError_t e =
         dev_alloc_async(reinterpret_cast<void**>(&wdense), static_cast<size_t>(h->N) * h->K * 2, st);

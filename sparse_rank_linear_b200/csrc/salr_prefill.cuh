@@ -69,6 +69,11 @@ struct PrefillParams {
   int wide;            // dense mode with 256-row tiles: each unit is two 128-row halves
                        // that share the X tiles, one TMEM accumulator per half
   int atile;           // bytes of a decoded-tile ring slot: 16 KB, or 32 KB when wide
+  int rtiles;          // weight row tiles (of 128 or 256 rows)
+  int group_rows;      // 0: tile t is (row tile t / TT, token tile t % TT).  Otherwise the
+                       // tiles go in groups of group_rows row tiles, token tile by token
+                       // tile, so that the tiles in flight share a few weight and X tiles
+                       // that stay in L2
   int cbuf;            // bytes of a compact-block slot, multiple of 1024
   int sc, sa, sx;      // ring depths: compact blocks, decoded tiles, X tiles
 };
@@ -141,8 +146,15 @@ __device__ __forceinline__ PreUnit pre_unit(const PrefillParams& p, int u) {
     w.sidx = u % p.splits;
     w.ns = p.splits;
   }
-  w.j = w.t % p.TT;
-  w.i = w.t / p.TT;
+  if (p.group_rows > 0) {
+    const int per = p.group_rows * p.TT, g = w.t / per, r = w.t - g * per;
+    const int rows = min(p.group_rows, p.rtiles - g * p.group_rows);  // the last group's
+    w.i = g * p.group_rows + r % rows;
+    w.j = r / rows;
+  } else {
+    w.j = w.t % p.TT;
+    w.i = w.t / p.TT;
+  }
   w.kb0 = static_cast<int>(static_cast<long long>(w.sidx) * p.kblocks / w.ns);
   const int kb1 = static_cast<int>(static_cast<long long>(w.sidx + 1) * p.kblocks / w.ns);
   w.nk = kb1 - w.kb0;

@@ -338,6 +338,28 @@ def test_linear_wide_tiles_full_compare(R, N, K, M, monkeypatch):
     h.free()
 
 
+@pytest.mark.parametrize("N,K,M,g,wide", [(640, 256, 600, 2, False), (1536, 512, 1100, 4, False),
+                                          (1280, 512, 1100, 2, True)])
+def test_linear_grouped_tile_order_full_compare(N, K, M, g, wide, monkeypatch):
+    # output tiles taken in groups of g row tiles, token tile by token tile (the order the
+    # library takes when X outgrows the L2), with a short last group and a ragged last
+    # token tile, on 128- and 256-row tiles
+    monkeypatch.setenv("SALR_TILE_GROUP_ROWS", str(g))
+    if wide:
+        monkeypatch.setenv("SALR_WIDE_MIN_ROUNDS", "0")
+        if salr.plan(N, K, M, 72)["tile_rows"] != 256:
+            pytest.skip("this GPU's SM count gives 128-row tiles for this shape")
+    wl = synth.Workload("grouped", N, K, (72,), (M,))
+    w, x, ad = synth.weight(wl), synth.activations(wl, M), synth.adapters(wl)
+    h = salr.encode(to_dev(w), 0.5)
+    wp = oracle.prune(w, oracle.magnitude_mask(w, 0.5))
+    Y = salr.linear(to_dev(x), h, to_dev(ad[0][0]), to_dev(ad[0][1]))
+    assert h.sync_status() == 0
+    assert_close(to_bits(Y), oracle.linear(x, wp, ad), oracle.abs_bound(x, wp, ad),
+                 f"grouped tiles g={g}")
+    h.free()
+
+
 @pytest.mark.parametrize("M", [256, 64])
 def test_identity_rows_reproduce_decoded_columns_bitexact(M):
     # X = rows of the identity, no adapter: every output is a single product
