@@ -224,6 +224,9 @@ typedef struct {
   int32_t splits;      /* K parts of each remaining tile (paths 1, 2; 1 = none) */
   int64_t split_sum_bytes;     /* fp32 sums of the split tiles in the handle's workspace */
   int64_t dense_scratch_bytes; /* transient dense bf16 weight (path 2), else 0 */
+  int32_t group_rows;  /* paths 1, 2: 0 when the output tiles go token tile first; else
+                          they go in groups of this many row tiles, token tile by token
+                          tile (when X outgrows about half the L2) */
 } salr_plan;
 SALR_API int salr_linear_plan(int64_t N, int64_t K, int64_t M, int64_t R, int32_t sms,
                               salr_plan* out);

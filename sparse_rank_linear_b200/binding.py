@@ -32,7 +32,8 @@ class SalrPlan(ctypes.Structure):
                 ("grid", ctypes.c_int32),
                 ("units", ctypes.c_int32), ("tiles", ctypes.c_int32),
                 ("whole_tiles", ctypes.c_int32), ("splits", ctypes.c_int32),
-                ("split_sum_bytes", ctypes.c_int64), ("dense_scratch_bytes", ctypes.c_int64)]
+                ("split_sum_bytes", ctypes.c_int64), ("dense_scratch_bytes", ctypes.c_int64),
+                ("group_rows", ctypes.c_int32)]
 SIGNATURES = {
     "salr_encode": (_I, [_P, _I64, _I64, _F, _P, ctypes.POINTER(_P)]),
     "salr_decode": (_I, [_P, _P, _P]),

@@ -394,6 +394,25 @@ int64_t split_makespan(int tiles, int kb, int sms, TileSplit ts) {
 // The launch plan of salr_linear for M tokens on `sms` SMs: the call itself and
 // salr_linear_plan both take their decisions from here.  N and K are valid shapes
 // (check_shape); for M > 64, K stays within kPreMaxKBlocks blocks of 64.
+// Order of the prefill kernel's output tiles.  Taken token tile first, the tiles in flight
+// sweep all of X every few row tiles: harmless while X stays in L2, but with X larger than
+// about half of it each sweep goes back to DRAM (large M = 8192: about 6 GB of reads per
+// call for 0.6 GB of operands).  Taken in groups of g row tiles, token tile by token
+// tile, the `grid` tiles in flight touch g weight row tiles and about grid / g X tiles,
+// and a group reads X once; g = sqrt(grid * X tile / weight tile) makes the tiles in
+// flight the fewest bytes.  0 keeps the plain order.
+int tile_group_rows(int rtiles, int TT, int rows, int bnt, int64_t K, int grid) {
+  const char* v = getenv("SALR_TILE_GROUP_ROWS");  // tests: a group size on small shapes
+  if (v && v[0] >= '0' && v[0] <= '9') {
+    const int g = atoi(v);
+    return g > rtiles ? rtiles : g;
+  }
+  const double wtile = 2.0 * rows * K, xtile = 2.0 * bnt * K;
+  if (TT * xtile <= 48.0 * (1 << 20) || TT < 2) return 0;
+  int g = static_cast<int>(std::lround(std::sqrt(grid * xtile / wtile)));
+  return g < 1 ? 1 : g > rtiles ? rtiles : g;
+}
+
 struct LinearPlan {
   int path;     // 0 small-M kernel, 1 t + fused decode/GEMM, 2 expansion + t + dense GEMM
   int kernels;  // launches per call
@@ -403,6 +422,7 @@ struct LinearPlan {
   int full, splits;  // whole tiles; K parts of each later tile
   int units, grid;
   int64_t sum_bytes, dense_bytes;
+  int group_rows;  // prefill tile order (tile_group_rows)
 };
 LinearPlan plan_linear(int64_t N, int64_t K, int64_t M, int64_t R, int sms) {
   LinearPlan p{};
@@ -444,6 +464,7 @@ LinearPlan plan_linear(int64_t N, int64_t K, int64_t M, int64_t R, int sms) {
   p.kernels = 1 + (R > 0 ? 1 : 0) + (dense ? 1 : 0);
   p.sum_bytes = p.splits > 1 ? static_cast<int64_t>(p.tiles - p.full) * p.rows * p.bnt * 4 : 0;
   p.dense_bytes = dense ? N * K * 2 : 0;
+  p.group_rows = tile_group_rows(static_cast<int>(N / p.rows), p.TT, p.rows, p.bnt, K, p.grid);
   return p;
 }
 
@@ -520,25 +541,6 @@ int launch_prefill(PrefillParams p, const CUtensorMap& tx, const CUtensorMap& tb
   cfg.numAttrs = after_t ? 1 : 0;
   SALR_TRY(cudaLaunchKernelEx(&cfg, kern, p, tx, tb, tt, tw));
   return SALR_OK;
-}
-
-// Order of the prefill kernel's output tiles.  Taken token tile first, the tiles in flight
-// sweep all of X every few row tiles: harmless while X stays in L2, but with X larger than
-// about half of it each sweep goes back to DRAM (large M = 8192: about 6 GB of reads per
-// call for 0.6 GB of operands).  Taken in groups of g row tiles, token tile by token
-// tile, the `grid` tiles in flight touch g weight row tiles and about grid / g X tiles,
-// and a group reads X once; g = sqrt(grid * X tile / weight tile) makes the tiles in
-// flight the fewest bytes.  0 keeps the plain order.
-int tile_group_rows(int rtiles, int TT, int rows, int bnt, int64_t K, int grid) {
-  const char* v = getenv("SALR_TILE_GROUP_ROWS");  // tests: a group size on small shapes
-  if (v && v[0] >= '0' && v[0] <= '9') {
-    const int g = atoi(v);
-    return g > rtiles ? rtiles : g;
-  }
-  const double wtile = 2.0 * rows * K, xtile = 2.0 * bnt * K;
-  if (TT * xtile <= 48.0 * (1 << 20) || TT < 2) return 0;
-  int g = static_cast<int>(std::lround(std::sqrt(grid * xtile / wtile)));
-  return g < 1 ? 1 : g > rtiles ? rtiles : g;
 }
 
 // Persistent small-M path: one CTA per SM, launched so that it may overlap the preceding
@@ -887,6 +889,7 @@ int salr_linear_plan(int64_t N, int64_t K, int64_t M, int64_t R, int32_t sms, sa
   out->splits = p.path == 0 ? 1 : p.splits;
   out->split_sum_bytes = p.sum_bytes;
   out->dense_scratch_bytes = p.dense_bytes;
+  out->group_rows = p.group_rows;
   return SALR_OK;
 }
 
@@ -979,7 +982,7 @@ int salr_linear(const void* X, int64_t M, salr_handle h, const void* A_cat, cons
   pp.dense = pl.path == 2 ? 1 : 0;
   pp.wide = pl.rows == 256 ? 1 : 0;
   pp.rtiles = static_cast<int>(h->N / pl.rows);
-  pp.group_rows = tile_group_rows(pp.rtiles, TT, pl.rows, bnt, h->K, grid);
+  pp.group_rows = pl.group_rows;
   if (pp.dense) {
     const cudaError_t e =
         dev_alloc_async(reinterpret_cast<void**>(&wdense), static_cast<size_t>(h->N) * h->K * 2, st);

@@ -177,13 +177,19 @@ def test_linear_plan_of_the_workloads(lib):
             up["whole_tiles"], up["splits"], up["units"]) == (2, 3, 256, 128, 688, 592, 3, 880)
     assert up["split_sum_bytes"] == 96 * 128 * 256 * 4
     assert up["dense_scratch_bytes"] == 11008 * 4096 * 2
+    # X of 16 MB stays in L2: token tile first
+    assert up["group_rows"] == 0
     dn = _plan(4096, 11008, 4096, 128)  # 512 = 3 x 148 + 68; 68 x 2 = 136 -> 1 round of 1/2
     assert (dn["tile_rows"], dn["tiles"], dn["whole_tiles"], dn["splits"], dn["units"]) == \
         (128, 512, 444, 2, 580)
+    # X of 90 MB: groups of round(sqrt(148 x 5.6 MB / 2.8 MB)) = 17 row tiles
+    assert dn["group_rows"] == 17
     # 24 full rounds of 256-row tiles, and the busiest CTA gets no more 128-row block steps
     # (2 x (24 x 128 + 32)) than with 128-row tiles (48 x 128 + 2 x 32)
     lg = _plan(28672, 8192, 8192, 96)  # 3584 = 24 x 148 + 32; 32 x 4 = 128 -> 1 round of 1/4
     assert (lg["tile_rows"], lg["tiles"], lg["whole_tiles"], lg["splits"]) == (256, 3584, 3552, 4)
+    # X of 134 MB, 256-row tiles as large as its token tiles: groups of round(sqrt(148)) = 12
+    assert lg["group_rows"] == 12
     # 256-row tiles would leave up_proj M = 512 at 86 tiles on 148 SMs: 128-row tiles
     u512 = _plan(11008, 4096, 512)
     assert (u512["tile_rows"], u512["tiles"], u512["whole_tiles"], u512["splits"]) == (128, 172, 148, 6)
