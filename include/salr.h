@@ -41,8 +41,11 @@
  *     than is ever added (failure tests only: the call then reports SALR_ERR_TIMEOUT);
  *     SALR_WIDE_MIN_ROUNDS=n sets how many full rounds of 256-row tiles the dense-scratch
  *     path needs before it uses them (default 8; tests set 0 to reach them on small
- *     shapes); SALR_COOPERATIVE=1 launches the small-M kernel cooperatively instead of
- *     with programmatic stream serialization; SALR_FAKE_OOM=1 makes allocations fail.
+ *     shapes); SALR_TILE_GROUP_ROWS=n sets the prefill kernel's tile group (tests);
+ *     SALR_STREAM_SKEW=S (0 .. 192, default 0) makes the small-M kernel's CTA ranges
+ *     shrink with the CTA index; SALR_COOPERATIVE=1 launches the small-M kernel
+ *     cooperatively instead of with programmatic stream serialization; SALR_FAKE_OOM=1
+ *     makes allocations fail.
  *
  * Shape rules (v1): N % 128 == 0, 128 <= N <= 2^22, K % 64 == 0, 64 <= K <= 32768,
  * R % 8 == 0, R <= 128, 1 <= M <= 2^24, at most 2^27 output tiles of 128 x 128

@@ -645,7 +645,13 @@ int launch_stream(StreamParams p, const CUtensorMap& tx, const CUtensorMap& ta,
   const long long units = p.units;
   const int grid = static_cast<int>(units < sms ? units : sms);
   p.tshare = grid < p.kblocks ? grid : p.kblocks;
-  p.treaders = stream_t_readers(units, grid, p.kblocks);
+  // SALR_STREAM_SKEW=S (0 .. 255): ranges that shrink with the CTA index (stream_split)
+  const char* sk = getenv("SALR_STREAM_SKEW");
+  const int skew = sk && sk[0] >= '0' && sk[0] <= '9' ? atoi(sk) : 0;
+  // (at most 192: the last CTA keeps at least a quarter of the first one's share; none
+  // below 4 blocks a CTA)
+  p.skew = units < 4ll * grid ? 0 : skew < 0 ? 0 : skew > 192 ? 192 : skew;
+  p.treaders = stream_t_readers(units, grid, p.kblocks, p.skew);
   // SALR_FAIL_T_WAIT=1 (failure tests only): the readers of t wait for one part more
   // than are ever added, so their bounded wait runs out and the call reports a timeout
   const char* ft = getenv("SALR_FAIL_T_WAIT");

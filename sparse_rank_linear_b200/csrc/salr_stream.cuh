@@ -69,6 +69,7 @@ struct StreamParams {
   int units;    // RT * kblocks
   int tshare;   // CTAs 0 .. tshare-1 compute a share of t (tshare = min(grid, kblocks))
   int treaders;  // CTAs that start a row tile (and read t): see stream_t_readers
+  int skew;      // S of stream_split (0: equal ranges)
   int twant;     // t parts the readers wait for: tshare (more only in failure tests)
   int cbuf;     // bytes of a super-slot: bpc compact blocks + 32, multiple of 1024
   int bpc;      // compact blocks per bulk copy (1 .. 4)
@@ -140,14 +141,24 @@ __device__ __forceinline__ bool wait_global_flag(const uint32_t* flag, uint32_t 
   }
 }
 
-// CTAs of a grid of G over U blocks in storage order (K blocks of KB per row tile) whose
-// contiguous range [c U / G, (c + 1) U / G) holds the first block of some row tile: the
-// CTAs that apply the adapter and so read t.
-__host__ __device__ inline int stream_t_readers(long long U, int G, int KB) {
+// First block of CTA c when U blocks in storage order are cut into one contiguous range
+// per CTA of a grid of G.  S = 0: equal ranges, c U / G.  S > 0: the ranges shrink
+// linearly with the CTA index, CTA G - 1 taking about (1 - S / 256) of CTA 0's share
+// (F(c) = U c (512 G - S c) / (G (512 G - S G)), S < 256): with programmatic launch the
+// CTAs of a call start in index order as the SMs of the previous call free up, so the
+// later ones have less time.
+__host__ __device__ inline long long stream_split(long long U, int G, int S, int c) {
+  if (S == 0) return (static_cast<long long>(c) * U) / G;
+  return (U * c * (512ll * G - static_cast<long long>(S) * c)) /
+         (static_cast<long long>(G) * (512ll * G - static_cast<long long>(S) * G));
+}
+
+// CTAs whose range holds the first block of some row tile (K blocks of KB per row tile):
+// the CTAs that apply the adapter and so read t.
+__host__ __device__ inline int stream_t_readers(long long U, int G, int KB, int S) {
   int n = 0;
   for (int c = 0; c < G; ++c) {
-    const long long a = (static_cast<long long>(c) * U) / G;
-    const long long b = (static_cast<long long>(c + 1) * U) / G;
+    const long long a = stream_split(U, G, S, c), b = stream_split(U, G, S, c + 1);
     n += ((a + KB - 1) / KB) * KB < b;
   }
   return n;
@@ -165,14 +176,6 @@ __device__ __forceinline__ int mul_div(long long a, long long b, long long c, bo
   return fits32 ? static_cast<int>(static_cast<uint32_t>(a) * static_cast<uint32_t>(b) /
                                    static_cast<uint32_t>(c))
                 : static_cast<int>((a * b) / c);
-}
-
-// CTA that owns unit u (block u in storage order) under the even split of U units.
-__device__ __forceinline__ int owner_of(long long u, long long U, int G, bool fits32) {
-  int c = mul_div(u, G, U, fits32);
-  while (c + 1 < G && mul_div(c + 1, U, G, fits32) <= u) ++c;
-  while (c > 0 && mul_div(c, U, G, fits32) > u) --c;
-  return c;
 }
 
 template <int BNT, int NDEC>
@@ -199,8 +202,9 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
   const int G = gridDim.x, cta = blockIdx.x;
   const long long U = p.units;
   const bool fits32 = U * G < (1ll << 32);
-  const int u0 = mul_div(cta, U, G, fits32);
-  const int u1 = mul_div(cta + 1, U, G, fits32);
+  const int u0 = p.skew ? static_cast<int>(stream_split(U, G, p.skew, cta)) : mul_div(cta, U, G, fits32);
+  const int u1 = p.skew ? static_cast<int>(stream_split(U, G, p.skew, cta + 1))
+                        : mul_div(cta + 1, U, G, fits32);
   const int KB = p.kblocks;
   // t share of this CTA: K blocks cta, cta + tshare, ... (only CTAs below tshare)
   const int nts = (adapter && cta < p.tshare) ? (KB - cta + p.tshare - 1) / p.tshare : 0;
@@ -618,17 +622,16 @@ __global__ void __launch_bounds__(32 * (kStreamFixedWarps + NDEC + kStreamGroups
         }
         zero_acc(x);
         if (!whole) {
-          // Each warp counts its 32 rows of the tile in on its own: its additions are
-          // performed first (fence), and the warp that arrives last for these rows reads
-          // their sum, writes Y and clears the sum and the count for the next call.
+          // Each warp counts its 32 rows of the tile in on its own, by the K blocks its
+          // segment covers: its additions are performed first (fence), and the warp whose
+          // count completes the tile's K blocks reads the sum of these rows, writes Y and
+          // clears the sum and the count for the next call.
           __threadfence();
           __syncwarp();
           uint32_t last = 0;
           if (lane == 0) {
-            const int c_first = owner_of(static_cast<long long>(i) * KB, U, G, fits32);
-            const int segs =
-                owner_of(static_cast<long long>(i) * KB + KB - 1, U, G, fits32) - c_first + 1;
-            last = atomicAdd(p.counters + 4 * i + q, 1u) == static_cast<uint32_t>(segs - 1);
+            const uint32_t nb = static_cast<uint32_t>(kbb - kba);
+            last = atomicAdd(p.counters + 4 * i + q, nb) + nb == static_cast<uint32_t>(KB);
           }
           if (__shfl_sync(0xffffffffu, last, 0)) {
 #pragma unroll
