@@ -4,12 +4,13 @@
 // HBM-bound regime (M <= 64) where decoding the bitmap blocks is the whole cost:
 //
 // * Work split: the weight's 128 x 64 blocks, in storage order, are cut into one
-//   contiguous range per CTA (one CTA per SM, every SM the same number of blocks).  A
-//   range covers one or more row-tile segments.  A segment that does not cover a whole
-//   row tile adds its fp32 partial into the tile's fp32 accumulator with vector
-//   reductions performed in L2, fences, and counts itself in per 32-row quarter; the last
-//   warp to arrive for a quarter (no waiting) reads its sum, writes the bf16 output and
-//   clears the accumulator and the count for the next call.
+//   contiguous range per CTA (one CTA per SM, every SM the same number of blocks unless
+//   the skew of stream_split is set).  A range covers one or more row-tile segments.  A
+//   segment that does not cover a whole row tile adds its fp32 partial into the tile's
+//   fp32 accumulator with vector reductions performed in L2, fences, and adds the number
+//   of K blocks it covers to its 32-row quarter's count; the warp whose addition
+//   completes the tile (no waiting) reads its sum, writes the bf16 output and clears the
+//   accumulator and the count for the next call.
 // * Stage 1 decode (SALR technical summary, Methodology 4): decoder warps work in
 //   groups, each group on a different block so that several blocks are in flight.  Each
 //   warp of a group rebuilds one 32-row quarter of the block, one row per thread
@@ -26,8 +27,8 @@
 //   both counts, so the scratch is zero again when the kernel ends, whatever the host
 //   did in between (a replayed graph included).
 // * Consecutive calls overlap (programmatic dependent launch): a CTA fetches its first
-//   compact blocks before waiting for the previous kernel of the stream, and touches X,
-//   the adapters, the scratch and Y only after that wait.
+//   compact blocks and rebuilds its first blocks before waiting for the previous kernel
+//   of the stream, and touches X, the adapters, the scratch and Y only after that wait.
 //
 // The only cross-CTA wait is for t, on the t-share CTAs, which finish their share without
 // waiting on anything.  Every wait is bounded.
