@@ -14,6 +14,9 @@
 // * salr_prefill_kernel: persistent, one CTA per SM over the work units (128-row weight
 //   tile, token tile, K split).  Tiles are whole while every CTA gets one; the tiles of a
 //   last, partial round are split along K so that their parts even out over the CTAs.
+//   Tiles go token tile first or, when X outgrows about half the L2, in groups of row
+//   tiles, token tile by token tile, so that the tiles in flight share few weight and X
+//   tiles (pre_unit).
 //   Fused mode: each 128 x 64 bitmap block arrives by one bulk copy and the matching X
 //   tile by tensor TMA; decoder warps expand the block into the 128-byte-swizzled tile
 //   (stage 1, Methodology 4) with the same device functions as the small-M kernel, and
